@@ -1,0 +1,386 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test checks the oracle against something it does not share code with: the pages'
+printed numbers (tests/golden/), exhaustive enumeration of binary16 values, brute-force
+search over all codes, an independent bit reader (numpy.unpackbits), closed forms of
+softmax attention, a library attention routine (torch scaled_dot_product_attention in
+float64), and a 50-digit mpmath evaluation.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+# all finite binary16 values in increasing order (+inf appended), from numpy's own decoder
+_ALL16 = np.arange(0, 0x10000, dtype=np.uint32).astype(np.uint16)
+_VALS16 = _ALL16.view(np.float16).astype(np.float64)
+_FIN = np.isfinite(_VALS16)
+_ORDER = np.argsort(_VALS16[_FIN], kind="stable")
+_SORTED_VALS = _VALS16[_FIN][_ORDER]
+_SORTED_BITS = _ALL16[_FIN][_ORDER]
+
+
+def _smallest_f16_at_least(x: float):
+    """Brute force over every binary16 value: the smallest one >= x (value, bits)."""
+    i = np.searchsorted(_SORTED_VALS, x, side="left")
+    if i == len(_SORTED_VALS):
+        return math.inf, 0x7C00
+    return _SORTED_VALS[i], int(_SORTED_BITS[i])
+
+
+def _read_examples(path):
+    ex, cur = [], None
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        if line.startswith("example"):
+            cur = {"name": line.split()[1]}
+            ex.append(cur)
+            continue
+        k, v = [s.strip() for s in line.split("=", 1)]
+        cur[k] = v
+    return ex
+
+
+def _read_kv(path):
+    out = {}
+    for line in open(path):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            k, v = [s.strip() for s in line.split("=", 1)]
+            out[k] = int(v)
+    return out
+
+
+# --------------------------------------------------------------------------
+# binary16 helpers
+# --------------------------------------------------------------------------
+
+def test_f16_decode_matches_numpy(oracle_mod):
+    for h in list(range(0, 0x7C00, 97)) + [0, 1, 0x3FF, 0x400, 0x3C00, 0x7BFF, 0x8001, 0xBC00]:
+        ref = np.array([h], dtype=np.uint16).view(np.float16).astype(np.float64)[0]
+        assert oracle_mod.f16_bits_to_f64(h) == ref
+
+
+def test_f16_round_up_is_smallest_value_at_least(oracle_mod):
+    rng = np.random.default_rng(0)
+    xs = []
+    # exact binary16 values, their float32 neighbours and midpoints, across all binades
+    for h in range(1, 0x7C00, 37):
+        v = np.float32(_VALS16[h])
+        xs += [v, np.nextafter(v, np.float32(np.inf)), np.nextafter(v, np.float32(0))]
+        if h + 1 < 0x7C00:
+            xs.append(np.float32((_VALS16[h] + _VALS16[h + 1]) / 2))
+    xs += list(rng.uniform(0, 70000, 2000).astype(np.float32))
+    xs += list((10.0 ** rng.uniform(-12, -4, 2000)).astype(np.float32))   # subnormal range
+    xs += [np.float32(65504.0), np.float32(65504.5), np.float32(65520.0), np.float32(1e-30)]
+    xs += list(-rng.uniform(0, 70000, 500).astype(np.float32))             # negatives
+    for x in xs:
+        want_val, want_bits = _smallest_f16_at_least(float(x))
+        got = oracle_mod.f32_to_f16_ru(float(x))
+        if float(x) == 0.0:
+            assert oracle_mod.f16_bits_to_f64(got) == 0.0
+            continue
+        assert oracle_mod.f16_bits_to_f64(got) == want_val, (x, hex(got), want_val)
+
+
+# --------------------------------------------------------------------------
+# quantiser
+# --------------------------------------------------------------------------
+
+def test_golden_worked_examples(oracle_mod):
+    for ex in _read_examples(os.path.join(GOLDEN, "quant_worked_examples.txt")):
+        b = int(ex["b"])
+        v = np.array([float(x) for x in ex["v"].split()], dtype=np.float32)[None, :]
+        scales, codes = oracle_mod.quantize(v, b)
+        assert int(scales[0]) == int(ex["scale_bits"], 16), ex["name"]
+        assert codes[0].tolist() == [int(x) for x in ex["codes"].split()], ex["name"]
+        rows = oracle_mod.pack(codes, b)
+        want = bytes(int(x, 16) for x in ex["row"].split())
+        assert rows[0].tobytes() == want, ex["name"]
+        assert oracle_mod.unpack(rows, v.shape[1], b).tolist() == codes.tolist()
+
+
+def _brute_codes(v, s, q):
+    """Argmin over every integer code in [-q, q] of |fp32(v/s) - code|, ties to even."""
+    out = np.zeros(v.shape, dtype=np.int64)
+    cand = np.arange(-q, q + 1, dtype=np.int64)
+    for i, x in enumerate(v):
+        t = np.float32(x) / np.float32(s)        # one IEEE binary32 division
+        if q > 1000:                              # b = 16: search a window around t
+            c0 = int(np.floor(np.float64(t)))
+            cc = np.arange(max(-q, c0 - 2), min(q, c0 + 3), dtype=np.int64)
+        else:
+            cc = cand
+        dist = np.abs(np.float64(t) - cc.astype(np.float64))
+        best = dist.min()
+        ties = cc[dist == best]
+        even = ties[ties % 2 == 0]
+        out[i] = even[0] if len(even) else ties[0]
+    return out
+
+
+@pytest.mark.parametrize("b", [2, 4, 8, 16])
+def test_quantizer_against_brute_force_and_bounds(oracle_mod, b):
+    rng = np.random.default_rng(b)
+    q = 2 ** (b - 1) - 1
+    T, n = 24, 80
+    v = rng.standard_normal((T, n)).astype(np.float32)
+    v[3] *= 1e-3
+    v[4] *= 1e4
+    v[5, :] = 0.0
+    v[6, 7] = 5.0                       # one dominant value
+    v[7] = rng.standard_t(3, n).astype(np.float32)
+    scales, codes = oracle_mod.quantize(v, b)
+    for t in range(T):
+        A = float(np.max(np.abs(v[t])))
+        s = oracle_mod.f16_bits_to_f64(int(scales[t]))
+        if A == 0.0:
+            assert s == 0.0 and not codes[t].any()
+            continue
+        # scale: smallest binary16 value not below the binary32 quotient A/q
+        quot = float(np.float32(A) / np.float32(q))
+        want_s, _ = _smallest_f16_at_least(quot)
+        assert s == want_s
+        # codes: brute force over all codes
+        assert np.array_equal(codes[t], _brute_codes(v[t], s, q)), t
+        assert np.abs(codes[t]).max() <= q
+        # dequantisation error <= s/2, up to the binary32 rounding of the quotient v/s
+        err = np.abs(v[t].astype(np.float64) - codes[t] * s)
+        bound = s / 2 + np.abs(v[t].astype(np.float64)) * 2.0 ** -23
+        assert np.all(err <= bound), (t, (err - bound).max())
+
+
+def test_quantizer_ties_round_to_even(oracle_mod):
+    # s = 0.125 exactly: A = 127 * 0.125 at b = 8
+    s = 0.125
+    ks = np.arange(-120, 120)
+    v = np.concatenate([[127 * s], (ks + 0.5) * s]).astype(np.float32)
+    scales, codes = oracle_mod.quantize(v[None, :], 8)
+    assert oracle_mod.f16_bits_to_f64(int(scales[0])) == s
+    c = codes[0][1:]
+    lo, hi = ks, ks + 1
+    want = np.where(lo % 2 == 0, lo, hi)
+    assert np.array_equal(c, want)
+
+
+def test_quantizer_scale_is_shared_by_latent_and_rope(oracle_mod):
+    # one scale per token over [c[:d] || k^R]: a large rope value sets the scale for the latent
+    c = np.zeros((1, 64), dtype=np.float32)
+    c[0, :32] = 0.01
+    kr = np.zeros((1, 16), dtype=np.float32)
+    kr[0, 3] = 100.0
+    rows, scales, codes = oracle_mod.quantize_rows(c, kr, 32, 8)
+    s = oracle_mod.f16_bits_to_f64(int(scales[0]))
+    assert s >= 100.0 / 127
+    assert codes.shape == (1, 48)
+    assert codes[0, 32 + 3] == 127 and np.all(codes[0, :32] == 0)
+
+
+# --------------------------------------------------------------------------
+# packing
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("b", [2, 4, 8, 16])
+@pytest.mark.parametrize("n", [48, 80, 192, 576])
+def test_pack_against_numpy_bit_reader(oracle_mod, b, n):
+    rng = np.random.default_rng(n * 31 + b)
+    q = 2 ** (b - 1) - 1
+    codes = rng.integers(-q, q + 1, size=(5, n)).astype(np.int32)
+    rows = oracle_mod.pack(codes, b)
+    rb = rows.shape[1]
+    assert rb % 16 == 0 and rb * 8 >= n * b and (rb - 16) * 8 < n * b
+    bits = np.unpackbits(rows, axis=1, bitorder="little")           # independent reader
+    fields = bits[:, : n * b].reshape(5, n, b).astype(np.int64)
+    u = (fields << np.arange(b, dtype=np.int64)).sum(axis=2)
+    assert np.array_equal(u - 2 ** (b - 1), codes)
+    assert not bits[:, n * b:].any()                                  # zero padding
+
+
+def test_row_bytes_of_the_configured_shapes(oracle_mod):
+    # tiny: d=32,b=8 -> 48 B; d=64,b=4 -> 40 B padded to 48 B; 14B shapes need no padding
+    assert oracle_mod.row_bytes(32 + 16, 8) == 48
+    assert oracle_mod.row_bytes(64 + 16, 4) == 48
+    for d in (128, 256, 384, 512):
+        for b in (2, 4, 8, 16):
+            assert oracle_mod.row_bytes(d + 64, b) == (d + 64) * b // 8
+
+
+# --------------------------------------------------------------------------
+# attention
+# --------------------------------------------------------------------------
+
+def _sdpa(q_lat, q_rope, rows, d, sigma):
+    """torch's attention routine in float64: keys [c || kR], values c[:d]."""
+    Q = torch.from_numpy(np.concatenate([q_lat, q_rope], axis=1))[None, None]
+    K = torch.from_numpy(rows)[None, None]
+    V = torch.from_numpy(rows[:, :d])[None, None]
+    out = torch.nn.functional.scaled_dot_product_attention(Q, K, V, scale=sigma)[0, 0].numpy()
+    lse = torch.logsumexp(sigma * (Q[0, 0] @ K[0, 0].T), dim=-1).numpy()
+    return out, lse
+
+
+def test_attention_matches_library_routine(oracle_mod):
+    rng = np.random.default_rng(5)
+    H, d, dR, T = 6, 32, 16, 77
+    q_lat = rng.standard_normal((H, d))
+    q_rope = rng.standard_normal((H, dR))
+    rows = rng.standard_normal((T, d + dR)) * 1.5
+    sigma = 1 / math.sqrt(d + dR)
+    out, lse = oracle_mod.attend(q_lat, q_rope, rows, np.arange(T), sigma)
+    ref, ref_lse = _sdpa(q_lat, q_rope, rows, d, sigma)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_closed_forms(oracle_mod):
+    rng = np.random.default_rng(6)
+    H, d, dR, T = 3, 16, 8, 10
+    rows = rng.standard_normal((T, d + dR))
+    q_lat = rng.standard_normal((H, d))
+    q_rope = rng.standard_normal((H, dR))
+    # single token: out = c_hat[:d], lse = its score
+    out, lse = oracle_mod.attend(q_lat, q_rope, rows, [4], 0.3)
+    for h in range(H):
+        np.testing.assert_allclose(out[h], rows[4, :d], rtol=0, atol=1e-15)
+        z = 0.3 * (q_lat[h] @ rows[4, :d] + q_rope[h] @ rows[4, d:])
+        assert abs(lse[h] - z) < 1e-12
+    # zero query: uniform weights, out = mean, lse = log T
+    out, lse = oracle_mod.attend(np.zeros((H, d)), np.zeros((H, dR)), rows, np.arange(T), 1.0)
+    np.testing.assert_allclose(out, np.tile(rows[:, :d].mean(0), (H, 1)), atol=1e-14)
+    np.testing.assert_allclose(lse, math.log(T), atol=1e-14)
+    # two tokens: logistic weights
+    out, _ = oracle_mod.attend(q_lat, q_rope, rows, [1, 7], 0.5)
+    for h in range(H):
+        z1 = 0.5 * (q_lat[h] @ rows[1, :d] + q_rope[h] @ rows[1, d:])
+        z7 = 0.5 * (q_lat[h] @ rows[7, :d] + q_rope[h] @ rows[7, d:])
+        w1 = 1 / (1 + math.exp(z7 - z1))
+        np.testing.assert_allclose(out[h], w1 * rows[1, :d] + (1 - w1) * rows[7, :d], atol=1e-13)
+    # empty token set (reading R5)
+    out, lse = oracle_mod.attend(q_lat, q_rope, rows, [], 1.0)
+    assert not out.any() and np.all(np.isneginf(lse))
+
+
+def test_attention_invariances(oracle_mod):
+    rng = np.random.default_rng(7)
+    H, d, dR, T = 4, 32, 16, 50
+    rows = rng.standard_normal((T, d + dR))
+    q_lat, q_rope = rng.standard_normal((H, d)), rng.standard_normal((H, dR))
+    out, lse = oracle_mod.attend(q_lat, q_rope, rows, np.arange(T), 0.2)
+    perm = rng.permutation(T)
+    out2, lse2 = oracle_mod.attend(q_lat, q_rope, rows[perm], np.arange(T), 0.2)
+    np.testing.assert_allclose(out2, out, atol=1e-13)
+    np.testing.assert_allclose(lse2, lse, atol=1e-13)
+    # keep list == attention over the host-compacted rows
+    keep = np.sort(rng.choice(T, 13, replace=False)).astype(np.int32)
+    o_k, l_k = oracle_mod.attend(q_lat, q_rope, rows, keep, 0.2)
+    o_c, l_c = oracle_mod.attend(q_lat, q_rope, rows[keep], np.arange(13), 0.2)
+    np.testing.assert_allclose(o_k, o_c, atol=0)
+    np.testing.assert_allclose(l_k, l_c, atol=0)
+
+
+def test_attention_high_precision_brute_force(oracle_mod):
+    mp = pytest.importorskip("mpmath")
+    mp.mp.dps = 50
+    rng = np.random.default_rng(8)
+    H, d, dR, T = 2, 4, 2, 3
+    rows = rng.standard_normal((T, d + dR)) * 3
+    q_lat, q_rope = rng.standard_normal((H, d)) * 2, rng.standard_normal((H, dR))
+    sigma = 0.7
+    out, lse = oracle_mod.attend(q_lat, q_rope, rows, np.arange(T), sigma)
+    for h in range(H):
+        z = [mp.mpf(sigma) * (mp.fsum(mp.mpf(q_lat[h, j]) * mp.mpf(rows[t, j]) for j in range(d))
+                              + mp.fsum(mp.mpf(q_rope[h, j]) * mp.mpf(rows[t, d + j]) for j in range(dR)))
+             for t in range(T)]
+        e = [mp.e ** zt for zt in z]
+        Z = mp.fsum(e)
+        for j in range(d):
+            o = mp.fsum(e[t] * mp.mpf(rows[t, j]) for t in range(T)) / Z
+            assert abs(float(o) - out[h, j]) <= 1e-13 * max(1.0, abs(float(o)))
+        assert abs(float(mp.log(Z)) - lse[h]) <= 1e-13
+
+
+def test_full_width_16_bit_cache_matches_unquantised_attention(oracle_mod):
+    """b = 16, d = r: attention over the quantised cache equals plain MLA attention on the
+    original inputs, up to the quantisation error (|v - v_hat| <= s/2 with s ~ A/32767)."""
+    rng = np.random.default_rng(9)
+    H, r, dR, T = 8, 64, 16, 200
+    c = rng.standard_normal((T, r)).astype(np.float32)
+    kr = rng.standard_normal((T, dR)).astype(np.float32)
+    q_lat = rng.standard_normal((H, r))
+    q_rope = rng.standard_normal((H, dR))
+    sigma = 1 / math.sqrt(r + dR)
+    _, scales, codes = oracle_mod.quantize_rows(c, kr, r, 16)
+    out, lse = oracle_mod.decode_sequence(q_lat, q_rope, codes, scales, r, sigma)
+    exact = np.concatenate([c, kr], axis=1).astype(np.float64)
+    ref, ref_lse = _sdpa(q_lat, q_rope, exact, r, sigma)
+    # per-element error <= A/32767/2 ~ 7e-5 here; the output moves by about as much
+    for h in range(H):
+        assert np.abs(out[h] - ref[h]).max() <= 2e-3 * np.abs(ref[h]).max()
+        assert np.abs(out[h] - ref[h]).max() <= 1e-3
+    np.testing.assert_allclose(lse, ref_lse, atol=1e-3)
+
+
+def test_inheriting_layer_reads_anchor_cache(oracle_mod):
+    """Depth axis: a layer that inherits uses its anchor's rows; same query -> same output."""
+    rng = np.random.default_rng(10)
+    c = rng.standard_normal((40, 64)).astype(np.float32)
+    kr = rng.standard_normal((40, 16)).astype(np.float32)
+    _, s, k = oracle_mod.quantize_rows(c, kr, 32, 8)
+    q_lat, q_rope = rng.standard_normal((4, 64)), rng.standard_normal((4, 16))
+    a = oracle_mod.decode_sequence(q_lat, q_rope, k, s, 32, 0.1)
+    b = oracle_mod.decode_sequence(q_lat, q_rope, k.copy(), s.copy(), 32, 0.1)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+# --------------------------------------------------------------------------
+# cost model
+# --------------------------------------------------------------------------
+
+def test_cost_model_closed_forms(oracle_mod):
+    g = _read_kv(os.path.join(GOLDEN, "cost_model_closed_forms.txt"))
+    c0 = oracle_mod.c0_bits(48, 8, 128)
+    assert c0 == g["c0_bits_14b"]
+    assert c0 // 8 == g["c0_bytes_14b"] == 192 * 1024
+    assert 32 * 8192 * (c0 // 8) == g["cache_32x8k_bytes_14b"] == 48 * 2 ** 30
+    D, B = (64, 128, 256, 512), (2, 4, 8, 16)
+    assert 1 + len(D) * len(B) == g["n_actions"]
+    # M3 Ultra composition: 12 anchors of rank 128 (+ d_R = 64) at 4 bits, scale-free cost,
+    # plus the 0.5 bit / element of a grouped scale -> 151.7 ~ 152x
+    anchor = [4 * (l // 4) for l in range(48)]
+    d = [128 if l % 4 == 0 else 0 for l in range(48)]
+    b = [4 if l % 4 == 0 else 0 for l in range(48)]
+    bits4 = oracle_mod.bits_per_token(anchor, d, b, 64, with_scale=False)
+    assert bits4 == 12 * 192 * 4
+    assert round(c0 / (bits4 * 4.5 / 4)) == g["m3_ultra_ratio_rounded"]
+    assert 4 * 8 == g["composed_eviction_ratio"]
+
+
+def test_cost_model_counts_anchors_only(oracle_mod):
+    anchor, d, b = [0, 0, 2, 2], [32, 0, 64, 0], [8, 0, 4, 0]
+    assert oracle_mod.bits_per_token(anchor, d, b, 16) == (48 * 8 + 16) + (80 * 4 + 16)
+    assert oracle_mod.bits_per_token(anchor, d, b, 16, with_scale=False) == 48 * 8 + 80 * 4
+
+
+def test_workload_tables_meet_their_budgets(oracle_mod):
+    import workloads
+    tabs = workloads.load_tables()
+    for key, t in tabs.items():
+        a = t["anchor"]
+        assert a[0] == 0
+        last = 0
+        for l in range(len(a)):
+            if a[l] == l:
+                last = l
+                assert t["d"][l] > 0 and t["b"][l] in (2, 4, 8, 16)
+            assert a[l] == last
+        if "budget_bits" in t:
+            bits = oracle_mod.bits_per_token(a, t["d"], t["b"], 64)
+            assert bits == t["bits_per_token"]
+            full = len(a) * ((512 + 64) * 16 + 16)
+            assert bits <= t["budget_bits"] or (bits == full and t["budget_bits"] >= full)
