@@ -1,0 +1,447 @@
+"""Benchmark of the compressed-KV MLA decode step (KV-Kaizen cache) on B200.
+
+One step = the whole hot path over one batch: every anchor layer appends one token through
+kvk_quant_write (quantise-on-write), then every layer runs kvk_mla_decode (split decode +
+log-sum-exp merge) over its anchor's packed cache.  Workload: the 14B shape at the 4x
+budget (48 layers, 40 heads, r = 512, d_R = 64, 32 sequences x 8192 tokens, seeded table),
+synthetic seeded inputs generated on the device.
+
+Prints one JSON line.  `value` is the compressed-cache bytes the decode reads per step
+(algorithmic, sum over layers of batch * tokens * (row_bytes + 2)) per second of the whole
+step, appends included.  Inputs are larger than L2 (the per-layer cache is ~300 MB).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvk|reference]
+                  [--workload 14b_4x] [--graph]
+
+Under torchrun (N > 1) every rank runs an independent replica (the path is data-parallel
+over sequences with no exchange step); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+LOG2 = 0.6931471805599453
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="kvk", choices=["kvk", "reference"])
+    p.add_argument("--workload", default="14b_4x")
+    p.add_argument("--graph", action="store_true", help="replay the step as a CUDA graph")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def dist_setup(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+        pg = dist
+    return rank, world, local, pg
+
+
+def max_over_ranks(x: float, pg, device) -> float:
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg, device=None):
+    if pg is not None:
+        if device is not None and device.type == "cuda":
+            pg.barrier(device_ids=[device.index])
+        else:
+            pg.barrier()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def physical_gpu_index(local: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        parts = [x.strip() for x in vis.split(",") if x.strip()]
+        if local < len(parts):
+            return parts[local]
+    return str(local)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# workload construction (device-side seeded generation)
+# ---------------------------------------------------------------------------
+
+class DecodeWorkload:
+    def __init__(self, name, device, pkg):
+        self.w = w = workloads.WORKLOADS[name]
+        self.t = t = workloads.table(name)
+        self.device = device
+        self.pkg = pkg
+        self.B, self.T, self.H = w.batch, w.tokens, w.n_heads
+        self.lay = pkg.Layout(t["anchor"], t["d"], t["b"], w.r, w.d_rope, self.B, self.T,
+                              device=device)
+        self.anchors = [l for l in range(w.n_layers) if t["anchor"][l] == l]
+        zero = torch.zeros(self.B, dtype=torch.int32, device=device)
+        for l in self.anchors:            # prefill (not timed)
+            c = workloads.latent(w, l, self.B, self.T, device=device)
+            kr = workloads.rope_key(w, l, self.B, self.T, device=device)
+            self.lay.quant_write(l, c, kr, zero)
+            del c, kr
+        torch.cuda.synchronize(device)
+        # per-step inputs: one new token per anchor (written at the last position), queries
+        self.app_pos = torch.full((self.B,), self.T - 1, dtype=torch.int32, device=device)
+        self.app = {l: (workloads.latent(w, l, self.B, 1, device=device, kind="append"),
+                        workloads.rope_key(w, l, self.B, 1, device=device, kind="append"))
+                    for l in self.anchors}
+        self.q = {l: workloads.queries(w, l, self.B, device=device) for l in range(w.n_layers)}
+        self.lens = torch.full((self.B,), self.T, dtype=torch.int32, device=device)
+        self.sigma = {l: workloads.softmax_scale(t["d"][t["anchor"][l]], w.d_rope)
+                      for l in range(w.n_layers)}
+        self.out = {l: torch.empty(self.B, self.H, t["d"][t["anchor"][l]], dtype=torch.float32,
+                                   device=device) for l in range(w.n_layers)}
+        wsb = max(self.lay.workspace_bytes(l, self.B, self.H) for l in range(w.n_layers))
+        self.ws = torch.empty(wsb, dtype=torch.uint8, device=device)
+        self.bytes_per_layer = []
+        for l in range(w.n_layers):
+            info = self.lay.layer_info(l)
+            self.bytes_per_layer.append(self.B * self.T * (info["row_bytes"] + 2))
+        self.decode_bytes = sum(self.bytes_per_layer)
+        self.launches_per_step = len(self.anchors) + 2 * w.n_layers
+
+    def step(self, events=None):
+        from compressed_decode_attention_kvk_b200 import kvk
+        h = self.lay.handle
+        for l in self.anchors:
+            c, kr = self.app[l]
+            kvk.kvk_quant_write(h, l, c, kr, self.app_pos)
+        for l in range(self.w.n_layers):
+            ql, qr = self.q[l]
+            if events is not None:
+                events[l][0].record()
+            kvk.kvk_mla_decode(h, l, ql, qr, self.lens, self.sigma[l], self.out[l], self.ws)
+            if events is not None:
+                events[l][1].record()
+
+
+def run_kvk(args, rank, world, local, pg):
+    import compressed_decode_attention_kvk_b200 as pkg
+    from compressed_decode_attention_kvk_b200 import build as kb
+    if rank == 0 or not os.path.exists(kb.LIB):
+        kb.build()
+    barrier(pg)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = DecodeWorkload(args.workload, device, pkg)
+    L = wl.w.n_layers
+
+    # ---- device-timed steps (inputs resident in HBM) -----------------------------------
+    graph = None
+    if args.graph:
+        s = torch.cuda.Stream(device)
+        s.wait_stream(torch.cuda.current_stream(device))
+        with torch.cuda.stream(s):
+            for _ in range(2):
+                wl.step()
+        torch.cuda.current_stream(device).wait_stream(s)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            wl.step()
+    for _ in range(args.warmup):
+        graph.replay() if graph else wl.step()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(L)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(pg, device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(physical_gpu_index(local)) as clk:
+        start.record()
+        for k in range(args.steps):
+            if graph:
+                graph.replay()
+            else:
+                wl.step(events=ev[k])
+        stop.record()
+        torch.cuda.synchronize(device)
+    barrier(pg, device)
+    t_ms = start.elapsed_time(stop)
+    t_ms = max_over_ranks(t_ms, pg, device)
+    clocks = clk.summary()
+    ms_step = t_ms / args.steps
+
+    # dominant kernel: the decode launches (split + merge per layer), timed by CUDA events on
+    # the launching stream inside the timed region
+    dec_ms = None
+    if not graph:
+        dec_ms = sum(ev[k][l][0].elapsed_time(ev[k][l][1]) for k in range(args.steps)
+                     for l in range(L)) / (args.steps * L)
+    peak, peak_kind = measured_peaks()
+    total_bytes = wl.decode_bytes * args.steps * world
+    value = total_bytes / (t_ms * 1e-3) / 1e9
+    roof = None
+    if dec_ms:
+        ach = (wl.decode_bytes / L) / (dec_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(ach / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                "kernel": "kvk_mla_decode (split decode + merge), mean over layers",
+                "launch_ms": round(dec_ms, 5)}
+
+    # ---- end to end through the C ABI with host buffers -------------------------------
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, wl, device, pg)
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only) ---------------------------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl)
+
+    if rank == 0:
+        line = {
+            "metric": "compressed-KV MLA decode: HBM GB/s (% of peak) and decode steps/s, 14B shape",
+            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "steps_per_s": round(1000.0 / ms_step * world, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded, generated on device)",
+            "config": {"workload": args.workload, "layers": L, "heads": wl.H, "r": wl.w.r,
+                       "d_rope": wl.w.d_rope, "batch": wl.B, "tokens": wl.T,
+                       "bits_per_token": wl.lay.bits_per_token,
+                       "decode_bytes_per_step": wl.decode_bytes,
+                       "l2": "inputs larger than L2 (per-layer cache > 126 MB)",
+                       "graph": bool(graph), "parallelism": f"replicas x{world}"},
+            "roofline": roof, "e2e": e2e, "cpu_baseline": cpu,
+            "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    wl.lay.close()
+
+
+def run_e2e(args, wl, device, pg):
+    """Same metric through the public API with host buffers: every step copies the step's
+    inputs (new tokens, all layers' queries) from pinned host memory and reads every
+    layer's output back to pinned host memory."""
+    from compressed_decode_attention_kvk_b200 import kvk
+    L = wl.w.n_layers
+    h_app = {l: (c.cpu().pin_memory(), k.cpu().pin_memory()) for l, (c, k) in wl.app.items()}
+    h_q = {l: (a.cpu().pin_memory(), b.cpu().pin_memory()) for l, (a, b) in wl.q.items()}
+    h_out = {l: torch.empty(o.shape, dtype=o.dtype).pin_memory() for l, o in wl.out.items()}
+    d_app = {l: (torch.empty_like(c), torch.empty_like(k)) for l, (c, k) in wl.app.items()}
+    d_q = {l: (torch.empty_like(a), torch.empty_like(b)) for l, (a, b) in wl.q.items()}
+    h2d = sum(c.numel() * c.element_size() + k.numel() * k.element_size()
+              for c, k in h_app.values()) + sum(a.numel() * a.element_size() +
+                                                b.numel() * b.element_size()
+                                                for a, b in h_q.values())
+    d2h = sum(o.numel() * o.element_size() for o in h_out.values())
+
+    def step():
+        for l in wl.anchors:
+            dc, dk = d_app[l]
+            dc.copy_(h_app[l][0], non_blocking=True)
+            dk.copy_(h_app[l][1], non_blocking=True)
+            kvk.kvk_quant_write(wl.lay.handle, l, dc, dk, wl.app_pos)
+        for l in range(L):
+            qa, qb = d_q[l]
+            qa.copy_(h_q[l][0], non_blocking=True)
+            qb.copy_(h_q[l][1], non_blocking=True)
+            kvk.kvk_mla_decode(wl.lay.handle, l, qa, qb, wl.lens, wl.sigma[l], wl.out[l], wl.ws)
+            h_out[l].copy_(wl.out[l], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    barrier(pg, device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        step()
+    b.record()
+    torch.cuda.synchronize(device)
+    t_ms = max_over_ranks(a.elapsed_time(b), pg, device)
+    world = 1 if pg is None else pg.get_world_size()
+    v = wl.decode_bytes * args.steps * world / (t_ms * 1e-3) / 1e9
+    return {"value": round(v, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(t_ms / args.steps, 4)}
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def _oracle_sample(wl_name, n_seq, layer=0, device="cpu"):
+    """Host inputs for a bounded sample: `n_seq` sequences of one layer of the workload."""
+    w = workloads.WORKLOADS[wl_name]
+    t = workloads.table(wl_name)
+    a = t["anchor"][layer]
+    d, b = t["d"][a], t["b"][a]
+    c = workloads.latent(w, a, w.batch, w.tokens, device=device)[:n_seq].float().cpu().numpy()
+    kr = workloads.rope_key(w, a, w.batch, w.tokens, device=device)[:n_seq].float().cpu().numpy()
+    ql, qr = workloads.queries(w, layer, w.batch, device=device)
+    return (w, d, b, c, kr, ql[:n_seq].double().cpu().numpy(), qr[:n_seq].double().cpu().numpy())
+
+
+def time_oracle_decode(sample, oracle):
+    w, d, b, c, kr, ql, qr = sample
+    sigma = workloads.softmax_scale(d, w.d_rope)
+    caches = [oracle.quantize_rows(c[i], kr[i], d, b) for i in range(c.shape[0])]
+    t0 = time.perf_counter()
+    for i in range(c.shape[0]):
+        rows, s, k = caches[i]
+        oracle.decode_sequence(ql[i], qr[i], k, s, d, sigma)
+    dt = time.perf_counter() - t0
+    row_bytes = caches[0][0].shape[1]
+    nbytes = c.shape[0] * c.shape[1] * (row_bytes + 2)
+    return nbytes, dt
+
+
+def cpu_baseline(wl):
+    from oracle import oracle
+    oracle.build()
+    n_seq = 2
+    sample = _oracle_sample(wl.w.name, n_seq, device=wl.device)
+    nbytes, dt = time_oracle_decode(sample, oracle)
+    return {"value": round(nbytes / dt / 1e9, 5), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"layer 0 decode of {n_seq} of {wl.B} sequences x {wl.T} tokens "
+                      f"({dt:.1f} s, fp64, OpenMP over heads)"}
+
+
+def run_reference(args, rank, world, local, pg):
+    """Reference arm: the CPU oracle as it stands, on the host cores, each step a bounded
+    sample (layer 0 decode of 1 sequence of the workload)."""
+    if rank != 0:
+        return
+    from oracle import oracle
+    oracle.build()
+    w = workloads.WORKLOADS[args.workload]
+    sample = _oracle_sample(args.workload, 1)
+    for _ in range(args.warmup):
+        time_oracle_decode(sample, oracle)
+    tot_b, tot_t = 0, 0.0
+    for _ in range(args.steps):
+        nb, dt = time_oracle_decode(sample, oracle)
+        tot_b += nb
+        tot_t += dt
+    v = tot_b / tot_t / 1e9
+    line = {
+        "impl": "reference",
+        "metric": "compressed-KV MLA decode: HBM GB/s (% of peak) and decode steps/s, 14B shape",
+        "value": round(v, 5), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": args.workload, "layers": w.n_layers, "heads": w.n_heads,
+                   "batch": w.batch, "tokens": w.tokens},
+        "cpu_baseline": {"value": round(v, 5), "unit": "GB/s", "kind": "oracle",
+                         "cores": oracle.num_threads(),
+                         "sample": f"layer 0 decode of 1 of {w.batch} sequences x {w.tokens} "
+                                   "tokens per step"},
+        "e2e": {"value": round(v, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local, pg = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world, local, pg)
+        else:
+            run_kvk(args, rank, world, local, pg)
+    finally:
+        if pg is not None:
+            pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

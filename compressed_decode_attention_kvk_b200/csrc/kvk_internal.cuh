@@ -1,0 +1,108 @@
+// kvk_internal.cuh -- types shared by the host layer and the kernels of libkvk.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "kvk.h"
+
+namespace kvk {
+
+constexpr int kMaxRowElems = 2048;      // d + d_rope handled by the write kernel
+constexpr size_t kArenaHeader = 256;    // status flags live in the first bytes of the arena
+constexpr int kTcTileTokens = 64;       // tokens per tile of the tensor-core decode
+
+struct AnchorDesc {
+  int layer = 0;
+  int d = 0;
+  int b = 0;
+  int n = 0;             // d + d_rope
+  int row_bytes = 0;
+  int64_t codes_off = 0;
+  int64_t scales_off = 0;
+  bool tmap_ok = false;
+  CUtensorMap tmap_tile;     // 2D [rows = max_batch*max_tokens][row_bytes] uint8, 64-row box
+  CUtensorMap tmap_gather;   // same tensor, one-row box for tile::gather4
+};
+
+}  // namespace kvk
+
+struct kvk_layout {
+  int n_layers = 0;
+  int r = 0;
+  int d_rope = 0;
+  int max_batch = 0;
+  int max_tokens = 0;
+  std::vector<int> anchor, d, b;
+  std::vector<int> slot;                  // layer -> index into anchors (its anchor's)
+  std::vector<kvk::AnchorDesc> anchors;
+  uint8_t* arena = nullptr;
+  size_t arena_bytes = 0;
+  int64_t bits_per_token = 0;
+  int path = KVK_PATH_AUTO;
+  int ctas = 0;
+  int device = -1;
+  int num_sms = 0;
+};
+
+namespace kvk {
+
+// ---------------------------------------------------------------------------
+// decode parameters shared by both decode kernels and the merge
+// ---------------------------------------------------------------------------
+struct DecodeArgs {
+  const uint8_t* codes;     // anchor's codes plane
+  const __half* scales;     // anchor's scale plane
+  int row_bytes, d, d_rope, n, b;
+  int max_tokens;
+  const void* q_lat;
+  const void* q_rope;
+  int64_t ql_ss, ql_sh, qr_ss, qr_sh;  // element strides
+  int batch, H;
+  const int32_t* seq_lens;
+  const int32_t* keep_idx;   // nullable
+  const int32_t* keep_len;
+  int keep_stride;
+  float sigma;
+  float* out;
+  float* lse;
+  // workspace
+  int32_t* seq_off;          // [batch + 1] token offsets of the flattened token space
+  float* ws_ml;              // [slots][H][2]  (running max in log2 units, sum of weights)
+  float* ws_o;               // [slots][H][d]  (un-normalised weighted sums)
+  int G;                     // CTAs the flattened tokens are split over
+  uint32_t* flags;
+};
+
+// Workspace carve-up: returns total bytes; fills pointers when base != nullptr.
+size_t decode_workspace(int batch, int H, int d, int G, void* base, DecodeArgs* a);
+
+// CTA count for a decode call (depends only on the layout and batch).
+int decode_ctas(const kvk_layout* L, int batch, int path);
+
+// launchers (return cudaGetLastError())
+cudaError_t launch_quant_write(const kvk_layout* L, const AnchorDesc& A, const void* c_kv,
+                               int dtype, int64_t c_ss, int64_t c_st, const void* k_rope,
+                               int64_t kr_ss, int64_t kr_st, int batch, const int32_t* start_pos,
+                               int n_new, cudaStream_t stream);
+cudaError_t launch_decode_fma(const DecodeArgs& a, int dtype, cudaStream_t stream);
+cudaError_t launch_decode_tc(const DecodeArgs& a, const AnchorDesc& A, int dtype, int num_sms,
+                             cudaStream_t stream);
+bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H);
+cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
+
+// Position -> CTA of the balanced split: CTA c owns [c*N/G, (c+1)*N/G).
+__host__ __device__ inline int cta_of(int64_t x, int64_t N, int G) {
+  int64_t c = ((x + 1) * (int64_t)G + N - 1) / N - 1;
+  return (int)(c < 0 ? 0 : (c >= G ? G - 1 : c));
+}
+__host__ __device__ inline int64_t cta_lo(int c, int64_t N, int G) {
+  return ((int64_t)c * N) / G;
+}
+
+}  // namespace kvk

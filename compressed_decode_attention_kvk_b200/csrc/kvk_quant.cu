@@ -1,0 +1,168 @@
+// kvk_quant.cu -- quantise-on-write of one anchor layer's MLA cache (prefill and append).
+//
+// Method: KV-Kaizen, "Three Non-Eviction Compression Axes": the cached vector of a token is
+// the latent c^KV truncated to its first d coordinates plus the decoupled RoPE key k^R
+// (rank axis), stored at b bits by symmetric uniform quantisation with one scale per token
+// (precision axis).  Scale dtype, rounding and bit layout follow the library's contract in
+// include/kvk.h (fp16 scale rounded up, round-half-even codes, offset-binary fields
+// little-endian in 16-byte padded rows, separate fp16 scale plane).
+//
+// Schedule: one warp per token.  Each lane owns groups of 8 consecutive elements
+// (one 16-byte bf16 load or two 16-byte fp32 loads), keeps them in registers, the warp
+// reduces |v| with shuffles, lane 0 stores the fp16 scale, and every lane stores its
+// group's packed bytes (b bytes per group) -- consecutive lanes write consecutive bytes.
+// The kernel is HBM bound: it reads (d + d_R) * sizeof(input) and writes row + 2 bytes
+// per token.
+#include "kvk_internal.cuh"
+
+namespace kvk {
+namespace {
+
+constexpr int kWarpsPerBlock = 8;
+constexpr int kMaxRounds = kMaxRowElems / (8 * 32);  // groups of 8 per lane
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&v)[8]);
+
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
+  float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
+  uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    // a bf16 is the high half of a binary32: widening is exact
+    v[2 * k] = __uint_as_float(w[k] << 16);
+    v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+quant_write_kernel(uint8_t* __restrict__ codes, __half* __restrict__ scales, int row_bytes,
+                   int d, int d_rope, int b, int max_tokens, const T* __restrict__ c_kv,
+                   int64_t c_ss, int64_t c_st, const T* __restrict__ k_rope, int64_t kr_ss,
+                   int64_t kr_st, int batch, const int32_t* __restrict__ start_pos, int n_new,
+                   uint32_t* __restrict__ flags) {
+  const int lane = threadIdx.x & 31;
+  const int64_t tok = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  if (tok >= (int64_t)batch * n_new) return;
+  const int seq = (int)(tok / n_new);
+  const int j = (int)(tok - (int64_t)seq * n_new);
+  const int64_t pos = (int64_t)__ldg(start_pos + seq) + j;
+  if (pos < 0 || pos >= max_tokens) {
+    if (lane == 0) atomicOr(flags, KVK_FLAG_WRITE_RANGE);
+    return;
+  }
+  const int n = d + d_rope;
+  const int groups = n >> 3;            // d % 16 == 0 and d_rope % 8 == 0
+  const int d_groups = d >> 3;
+  const T* crow = c_kv + (int64_t)seq * c_ss + (int64_t)j * c_st;
+  const T* krow = k_rope + (int64_t)seq * kr_ss + (int64_t)j * kr_st;
+
+  float v[kMaxRounds][8];
+  float amax = 0.0f;
+  bool finite = true;
+#pragma unroll
+  for (int r = 0; r < kMaxRounds; ++r) {
+    const int g = r * 32 + lane;
+    if (g < groups) {
+      if (g < d_groups) load8<T>(crow + 8 * g, v[r]);
+      else load8<T>(krow + 8 * (g - d_groups), v[r]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        finite = finite && isfinite(v[r][k]);
+        amax = fmaxf(amax, fabsf(v[r][k]));
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  finite = __all_sync(0xffffffffu, finite);
+
+  const int q = (1 << (b - 1)) - 1;
+  const float s32 = __fdiv_rn(amax, (float)q);          // IEEE binary32 division
+  const __half s16 = __float2half_ru(s32);               // rounded toward +inf
+  const float s = __half2float(s16);
+  if (lane == 0) {
+    if (!finite || isinf(s)) atomicOr(flags, KVK_FLAG_NONFINITE);
+    scales[(int64_t)seq * max_tokens + pos] = s16;
+  }
+  uint8_t* row = codes + ((int64_t)seq * max_tokens + pos) * row_bytes;
+  const uint32_t off = 1u << (b - 1);
+
+#pragma unroll
+  for (int r = 0; r < kMaxRounds; ++r) {
+    const int g = r * 32 + lane;
+    if (g >= groups) continue;
+    uint32_t u[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      int c = 0;
+      if (s != 0.0f) {
+        c = __float2int_rn(__fdiv_rn(v[r][k], s));       // round half to even
+        c = min(max(c, -q), q);
+      }
+      u[k] = (uint32_t)(c + (int)off);
+    }
+    uint8_t* dst = row + (int64_t)g * b;                 // 8 elements * b bits = b bytes
+    if (b == 16) {
+      uint4 w = make_uint4(u[0] | (u[1] << 16), u[2] | (u[3] << 16), u[4] | (u[5] << 16),
+                           u[6] | (u[7] << 16));
+      *reinterpret_cast<uint4*>(dst) = w;
+    } else if (b == 8) {
+      uint2 w = make_uint2(u[0] | (u[1] << 8) | (u[2] << 16) | (u[3] << 24),
+                           u[4] | (u[5] << 8) | (u[6] << 16) | (u[7] << 24));
+      *reinterpret_cast<uint2*>(dst) = w;
+    } else if (b == 4) {
+      uint32_t w = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) w |= u[k] << (4 * k);
+      *reinterpret_cast<uint32_t*>(dst) = w;
+    } else {  // b == 2
+      uint32_t w = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) w |= u[k] << (2 * k);
+      *reinterpret_cast<uint16_t*>(dst) = (uint16_t)w;
+    }
+  }
+  // zero the row padding (fewer than 16 bytes)
+  const int used = groups * b;
+  if (lane < row_bytes - used) row[used + lane] = 0;
+}
+
+}  // namespace
+
+cudaError_t launch_quant_write(const kvk_layout* L, const AnchorDesc& A, const void* c_kv,
+                               int dtype, int64_t c_ss, int64_t c_st, const void* k_rope,
+                               int64_t kr_ss, int64_t kr_st, int batch, const int32_t* start_pos,
+                               int n_new, cudaStream_t stream) {
+  const int64_t tokens = (int64_t)batch * n_new;
+  const int64_t blocks = (tokens + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  uint8_t* codes = L->arena + A.codes_off;
+  __half* scales = reinterpret_cast<__half*>(L->arena + A.scales_off);
+  uint32_t* flags = reinterpret_cast<uint32_t*>(L->arena);
+  dim3 grid((unsigned)blocks), block(kWarpsPerBlock * 32);
+  if (dtype == KVK_BF16) {
+    quant_write_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
+        codes, scales, A.row_bytes, A.d, L->d_rope, A.b, L->max_tokens,
+        static_cast<const __nv_bfloat16*>(c_kv), c_ss, c_st,
+        static_cast<const __nv_bfloat16*>(k_rope), kr_ss, kr_st, batch, start_pos, n_new, flags);
+  } else {
+    quant_write_kernel<float><<<grid, block, 0, stream>>>(
+        codes, scales, A.row_bytes, A.d, L->d_rope, A.b, L->max_tokens,
+        static_cast<const float*>(c_kv), c_ss, c_st, static_cast<const float*>(k_rope), kr_ss,
+        kr_st, batch, start_pos, n_new, flags);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace kvk

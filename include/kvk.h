@@ -1,0 +1,214 @@
+/*
+ * kvk.h -- C ABI of libkvk, the B200 (sm_100a) library for the KV-Kaizen compressed
+ * MLA KV cache: quantise-on-write of each anchor layer's cache and the decode-step
+ * attention that reads the packed cache back.
+ *
+ * Source of the method: "KV-Kaizen: Learning Context-Adaptive Cache Compression Choices"
+ * (whiteboard summary on picx.dev), sections "Three Non-Eviction Compression Axes"
+ * (depth / rank / precision) and "Action Space and Cost Model".
+ *
+ * Conventions shared by every entry point
+ *   - Plain pointers and sizes only.  "dev_" pointers are CUDA device pointers; every
+ *     other pointer is host memory.  The caller owns all device memory (arena, inputs,
+ *     outputs, workspace); a layout owns only its host-side metadata.
+ *   - Argument and table checks are synchronous and happen before any launch; a failed
+ *     check returns its status and launches nothing.  Launches are asynchronous on the
+ *     given stream (a cudaStream_t; NULL is the legacy default stream).  A launch error
+ *     returns KVK_ERR_CUDA.
+ *   - Device-side conditions that the host cannot see (positions and lengths held in
+ *     device memory, non-finite inputs) never fault: the kernel skips or clamps the
+ *     offending item and sets a sticky flag, read with kvk_read_status().
+ *   - Every device pointer must be 16-byte aligned (the arena: 256-byte aligned), or the
+ *     call returns KVK_ERR_ALIGNMENT.
+ *   - Nothing here allocates device memory except kvk_create_layout's one synchronous
+ *     cudaMemset of the arena header; nothing falls back to the CPU.
+ */
+#ifndef KVK_H_
+#define KVK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* kvk_stream_t;
+
+/* Opaque host-side handle: per-layer table, anchor map, arena offsets, TMA descriptors. */
+typedef struct kvk_layout kvk_layout;
+
+typedef enum {
+    KVK_OK = 0,
+    KVK_ERR_INVALID_ARG = 1,      /* null / out-of-range argument, or a layout without arena */
+    KVK_ERR_BAD_TABLE = 2,        /* anchor / d / b table violates the action space          */
+    KVK_ERR_BUDGET = 3,           /* plan's bits per token exceed the given budget            */
+    KVK_ERR_INHERITING_LAYER = 4, /* quant-write addressed a layer that inherits its cache    */
+    KVK_ERR_WORKSPACE = 5,        /* arena or workspace smaller than required                 */
+    KVK_ERR_ALIGNMENT = 6,        /* device pointer or stride not aligned as required         */
+    KVK_ERR_CUDA = 7,             /* a CUDA runtime / driver call or a launch failed          */
+    KVK_ERR_UNSUPPORTED = 8       /* shape outside what the compiled kernels handle           */
+} kvk_status;
+
+typedef enum { KVK_F32 = 0, KVK_BF16 = 1, KVK_F16 = 2 } kvk_dtype;
+
+/* Sticky device flags (kvk_read_status). */
+#define KVK_FLAG_NONFINITE   0x1u /* quant-write: non-finite input, or scale above the fp16 range */
+#define KVK_FLAG_WRITE_RANGE 0x2u /* quant-write: position outside [0, max_tokens); token skipped  */
+#define KVK_FLAG_SEQ_LEN     0x4u /* decode: seq_len outside [0, max_tokens], clamped; or keep_len
+                                     outside [0, keep_stride], clamped                             */
+#define KVK_FLAG_KEEP_INDEX  0x8u /* decode: keep index outside [0, seq_len); entry skipped        */
+
+/* Decode kernel selection (kvk_set_decode_path). */
+#define KVK_PATH_AUTO      0 /* tensor-core kernel where it applies, else the CUDA-core kernel  */
+#define KVK_PATH_TENSOR    1 /* tcgen05 kernel only (KVK_ERR_UNSUPPORTED where it cannot run)   */
+#define KVK_PATH_CUDA_CORE 2 /* FFMA kernel (any shape, any dtype)                                */
+
+/*
+ * kvk_create_layout -- validate a per-layer plan and lay out its cache in an arena.
+ *
+ * Defines: the depth axis (a layer either is an anchor with its own cache or inherits the
+ * nearest anchor before it), the rank axis (an anchor keeps the first d of r latent
+ * coordinates plus the d_rope-wide RoPE key) and the precision axis (b-bit symmetric
+ * codes, one scale per token) -- "Three Non-Eviction Compression Axes"; and the budget
+ * check of "Action Space and Cost Model" with the fp16 scale counted:
+ *     bits_per_token = sum over anchors l of ((d_l + d_rope) * b_l + 16).
+ *
+ *   n_layers            L >= 1
+ *   anchor[L]           anchor[l] == l for an anchor; otherwise the largest l' < l with
+ *                       anchor[l'] == l' (the nearest preceding anchor).  anchor[0] == 0.
+ *   d[L], b[L]          for anchors: 16 <= d <= r, d % 16 == 0; b in {2, 4, 8, 16}.
+ *                       Ignored for inheriting layers.
+ *   r, d_rope           latent width (multiple of 16) and RoPE width (multiple of 8, >= 0)
+ *   max_batch, max_tokens  capacity of every anchor's cache (max_batch * max_tokens < 2^31)
+ *   budget_bits_per_token  <= 0: no check; else KVK_ERR_BUDGET when the plan costs more
+ *   dev_arena, arena_bytes caller-owned device memory (256-byte aligned), size >= needed
+ *   out                 receives the handle; NULL = query only (sizes and bits filled in)
+ *   arena_bytes_needed, bits_per_token  optional outputs (may be NULL)
+ *
+ * With out != NULL and dev_arena == NULL a planning-only layout is returned: its offsets
+ * can be inspected (kvk_get_layer_info) but it cannot write or decode.  With an arena, the
+ * arena header (status flags) is zeroed by one synchronous cudaMemset.
+ * Arena layout: 256-byte header, then per anchor (in layer order) a codes plane
+ * [max_batch][max_tokens][row_bytes] and an fp16 scale plane [max_batch][max_tokens],
+ * each 256-byte aligned.  row_bytes = ceil((d + d_rope) * b / 8) rounded up to 16.
+ * Packed row format: field u_i = code_i + 2^(b-1) (offset binary) at bit i*b of the row
+ * read as a little-endian bit stream, i over [c[0..d) || k^R[0..d_rope)], zero padding.
+ */
+kvk_status kvk_create_layout(int n_layers, const int32_t* anchor, const int32_t* d,
+                             const int32_t* b, int r, int d_rope, int max_batch, int max_tokens,
+                             int64_t budget_bits_per_token, void* dev_arena, size_t arena_bytes,
+                             kvk_layout** out, size_t* arena_bytes_needed,
+                             int64_t* bits_per_token);
+
+/* Frees the host-side handle only (never the arena).  NULL is ignored. */
+void kvk_destroy(kvk_layout* layout);
+
+/* Where a layer's cache lives.  For an inheriting layer this describes its anchor's cache
+ * (the depth axis: the cache is never duplicated).  codes / scales are device pointers
+ * into the arena (offsets from 0 for a planning-only layout). */
+typedef struct {
+    int32_t anchor;         /* anchor layer whose cache this layer reads                  */
+    int32_t d;              /* latent coordinates kept by that anchor                      */
+    int32_t b;              /* bits per stored element                                     */
+    int32_t row_bytes;      /* bytes of one packed token row                               */
+    void* codes;            /* [max_batch][max_tokens][row_bytes] uint8                    */
+    void* scales;           /* [max_batch][max_tokens] fp16                                */
+    int64_t codes_offset;   /* byte offsets of the two planes inside the arena             */
+    int64_t scales_offset;
+    int32_t max_batch;
+    int32_t max_tokens;
+    int32_t r;
+    int32_t d_rope;
+} kvk_layer_info;
+
+kvk_status kvk_get_layer_info(const kvk_layout* layout, int layer, kvk_layer_info* info);
+
+/*
+ * kvk_quant_write -- quantise and store new tokens of one anchor layer (prefill or append).
+ *
+ * Defines the precision axis ("one scale per token", symmetric uniform, b bits) applied to
+ * the rank-truncated MLA vector v = [c_kv[0..d) || k_rope[0..d_rope)] of each token:
+ *     A = max_i |v_i| (fp32);  s32 = A / (2^(b-1) - 1) (IEEE fp32 division);
+ *     s = fp16(s32) rounded toward +inf, stored in the scale plane;
+ *     code_i = clamp(round_half_even(v_i / s), -(2^(b-1)-1), 2^(b-1)-1) with the stored
+ *     scale (IEEE fp32 division); s == 0 gives all-zero codes.
+ * Token j (0 <= j < n_new) of sequence i (0 <= i < batch) goes to position
+ * dev_start_pos[i] + j of sequence i's cache.
+ *
+ *   layer        an anchor layer (an inheriting layer -> KVK_ERR_INHERITING_LAYER)
+ *   c_kv         device, element (i, j, k) at c_kv[i*c_stride_seq + j*c_stride_tok + k],
+ *                k < d read (features contiguous); dtype KVK_F32 or KVK_BF16
+ *   k_rope       device, element (i, j, k) at k_rope[i*kr_stride_seq + j*kr_stride_tok + k],
+ *                k < d_rope; same dtype.  Strides in elements, multiples of 8 (16 B).
+ *   batch        1 <= batch <= max_batch;  n_new >= 0 (0: nothing launched)
+ *   dev_start_pos  device int32 [batch]; a position outside [0, max_tokens) skips the token
+ *                and sets KVK_FLAG_WRITE_RANGE; non-finite input or a scale beyond the
+ *                fp16 range sets KVK_FLAG_NONFINITE (the stored token is then unspecified).
+ */
+kvk_status kvk_quant_write(kvk_layout* layout, int layer, const void* c_kv, int dtype,
+                           int64_t c_stride_seq, int64_t c_stride_tok, const void* k_rope,
+                           int64_t kr_stride_seq, int64_t kr_stride_tok, int batch,
+                           const int32_t* dev_start_pos, int n_new, kvk_stream_t stream);
+
+/* Bytes of device workspace kvk_mla_decode needs for (layer, batch, n_heads), covering
+ * both decode kernels. */
+kvk_status kvk_decode_workspace_bytes(const kvk_layout* layout, int layer, int batch,
+                                      int n_heads, size_t* bytes);
+
+/*
+ * kvk_mla_decode -- one decode step of attention for one layer over its anchor's cache.
+ *
+ * Defines decode attention over the compressed cache ("every decoded token reads the
+ * entire KV cache", Background; the absorbed MLA form): with a = anchor(layer), d = d_a,
+ * c_hat_t = code_t * s_t the dequantised row of token t,
+ *     z_{h,t} = softmax_scale * (q_lat[h, 0..d) . c_hat_t[0..d) + q_rope[h] . c_hat_t[d..d+d_rope))
+ *     out[h]  = sum_t softmax_t(z_{h,.}) * c_hat_t[0..d),   lse[h] = log sum_t exp(z_{h,t})
+ * over t in 0..seq_len-1, or over the keep list when one is given (composition with token
+ * eviction).  An empty token set gives out = 0 and lse = -inf.
+ *
+ *   layer        any layer; an inheriting layer reads its anchor's cache (no copy)
+ *   q_lat        device [batch][n_heads][>= d] at q_lat[i*q_lat_stride_seq + h*q_lat_stride_head + k]
+ *   q_rope       device [batch][n_heads][d_rope], strides likewise (elements, multiples of 8)
+ *   dtype        KVK_BF16 / KVK_F16 (tensor-core kernel eligible) or KVK_F32 (CUDA-core kernel)
+ *   batch        1 <= batch <= max_batch;  n_heads >= 1
+ *   dev_seq_lens device int32 [batch], clamped to [0, max_tokens] (KVK_FLAG_SEQ_LEN)
+ *   dev_keep_idx nullable device int32 [batch][keep_stride]: ascending, unique token indices;
+ *                entries >= seq_len or < 0 are skipped (KVK_FLAG_KEEP_INDEX)
+ *   dev_keep_len device int32 [batch], required iff dev_keep_idx; clamped to [0, keep_stride]
+ *   softmax_scale  sigma above
+ *   out          device fp32 [batch][n_heads][d], written completely
+ *   lse          nullable device fp32 [batch][n_heads] (natural log)
+ *   workspace    device, >= kvk_decode_workspace_bytes(); contents are scratch
+ */
+kvk_status kvk_mla_decode(kvk_layout* layout, int layer, const void* q_lat, const void* q_rope,
+                          int dtype, int64_t q_lat_stride_seq, int64_t q_lat_stride_head,
+                          int64_t q_rope_stride_seq, int64_t q_rope_stride_head, int batch,
+                          int n_heads, const int32_t* dev_seq_lens, const int32_t* dev_keep_idx,
+                          const int32_t* dev_keep_len, int keep_stride, float softmax_scale,
+                          float* out, float* lse, void* workspace, size_t workspace_bytes,
+                          kvk_stream_t stream);
+
+/* Copy the sticky device flags to *flags (synchronises the stream); clear != 0 resets them
+ * to zero afterwards. */
+kvk_status kvk_read_status(kvk_layout* layout, uint32_t* flags, int clear, kvk_stream_t stream);
+
+/* Decode kernel choice (KVK_PATH_*) and the number of CTAs the decode splits the tokens
+ * over (0 = automatic).  Both only steer the schedule: results stay within tolerance of
+ * the same definition. */
+kvk_status kvk_set_decode_path(kvk_layout* layout, int path);
+kvk_status kvk_set_decode_ctas(kvk_layout* layout, int ctas);
+
+/* Which kernel kvk_mla_decode would run for these arguments (KVK_PATH_TENSOR or
+ * KVK_PATH_CUDA_CORE), without launching anything. */
+kvk_status kvk_decode_path_for(const kvk_layout* layout, int layer, int dtype, int n_heads,
+                               int* path);
+
+/* Static description of a status code. */
+const char* kvk_status_string(kvk_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVK_H_ */
