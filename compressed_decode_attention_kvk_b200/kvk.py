@@ -31,7 +31,10 @@ _DTYPE = {torch.float32: KVK_F32, torch.bfloat16: KVK_BF16, torch.float16: KVK_F
 EXPORTED = ("kvk_create_layout", "kvk_destroy", "kvk_get_layer_info", "kvk_quant_write",
             "kvk_decode_workspace_bytes", "kvk_mla_decode", "kvk_read_status",
             "kvk_set_decode_path", "kvk_set_decode_ctas", "kvk_decode_path_for",
-            "kvk_status_string")
+            "kvk_status_string", "kvk_mla_decode_noalloc")
+
+# size of the library's built-in scratch array used by kvk_mla_decode_noalloc
+KVK_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class KvkError(RuntimeError):
@@ -68,6 +71,8 @@ def _lib_handle():
         L.kvk_decode_workspace_bytes.argtypes = [P, i32, i32, i32, P]
         L.kvk_mla_decode.argtypes = [P, i32, P, P, i32, i64, i64, i64, i64, i32, i32, P, P, P,
                                      i32, ctypes.c_float, P, P, P, sz, P]
+        L.kvk_mla_decode_noalloc.argtypes = [P, i32, P, P, i32, i64, i64, i64, i64, i32, i32,
+                                             P, P, P, i32, ctypes.c_float, P, P, P]
         L.kvk_read_status.argtypes = [P, P, i32, P]
         L.kvk_set_decode_path.argtypes = [P, i32]
         L.kvk_set_decode_ctas.argtypes = [P, i32]
@@ -194,6 +199,31 @@ def kvk_mla_decode(handle, layer, q_lat, q_rope, seq_lens, softmax_scale, out, w
         float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check("kvk_mla_decode", st)
+
+
+def kvk_mla_decode_noalloc(handle, layer, q_lat, q_rope, seq_lens, softmax_scale, out,
+                           lse=None, keep_idx=None, keep_len=None, stream=None):
+    """kvk_mla_decode with the library's built-in scratch instead of a workspace tensor,
+    for callers that cannot allocate device memory (see include/kvk.h).  Same tensor rules
+    as kvk_mla_decode."""
+    _need_cuda(q_lat, "q_lat", tuple(_DTYPE))
+    _need_cuda(q_rope, "q_rope", (q_lat.dtype,))
+    _need_cuda(seq_lens, "seq_lens", (torch.int32,))
+    _need_cuda(out, "out", (torch.float32,))
+    _need_cuda(lse, "lse", (torch.float32,))
+    _need_cuda(keep_idx, "keep_idx", (torch.int32,))
+    _need_cuda(keep_len, "keep_len", (torch.int32,))
+    if q_lat.stride(2) != 1 or q_rope.stride(2) != 1:
+        raise ValueError("q_lat / q_rope last dim must be contiguous")
+    if not out.is_contiguous() or (lse is not None and not lse.is_contiguous()):
+        raise ValueError("out / lse must be contiguous")
+    B, H = q_lat.shape[0], q_lat.shape[1]
+    st = _lib_handle().kvk_mla_decode_noalloc(
+        handle, layer, _ptr(q_lat), _ptr(q_rope), _DTYPE[q_lat.dtype], q_lat.stride(0),
+        q_lat.stride(1), q_rope.stride(0), q_rope.stride(1), B, H, _ptr(seq_lens),
+        _ptr(keep_idx), _ptr(keep_len), 0 if keep_idx is None else keep_idx.stride(0),
+        float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream))
+    _check("kvk_mla_decode_noalloc", st)
 
 
 def kvk_read_status(handle, clear=False, stream=None) -> int:

@@ -190,6 +190,40 @@ kvk_status kvk_mla_decode(kvk_layout* layout, int layer, const void* q_lat, cons
                           float* out, float* lse, void* workspace, size_t workspace_bytes,
                           kvk_stream_t stream);
 
+/*
+ * kvk_mla_decode_noalloc -- kvk_mla_decode without a caller-provided workspace.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory for the workspace: for example a host application that reserves
+ * the whole device memory budget up front and hands plugins only fixed buffers, or a
+ * latency-critical loop where an allocation (and the synchronisation it may bring) is not
+ * acceptable.  Such a caller still passes its inputs and outputs; the scratch space comes
+ * from a file-scope __device__ array of KVK_NOALLOC_SCRATCH_BYTES bytes inside libkvk,
+ * which every GPU that loads the library holds until the process exits.
+ *
+ * Arguments and results are those of kvk_mla_decode minus (workspace, workspace_bytes).
+ * A call whose workspace need (kvk_decode_workspace_bytes) exceeds
+ * KVK_NOALLOC_SCRATCH_BYTES returns KVK_ERR_WORKSPACE and launches nothing.  This entry
+ * point allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * Set-up: the first call on a device (the device current at the call) looks up the
+ * array's device address with cudaGetSymbolAddress and caches it; make that first call
+ * before any stream capture.  All calls share the one array and it keeps the previous
+ * call's contents (no part of it needs to start at zero), so calls whose executions
+ * overlap on the GPU -- on different streams, or from different host threads -- race on
+ * it and give undefined results; order them on one stream or serialise them.
+ */
+#define KVK_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+kvk_status kvk_mla_decode_noalloc(kvk_layout* layout, int layer, const void* q_lat,
+                                  const void* q_rope, int dtype, int64_t q_lat_stride_seq,
+                                  int64_t q_lat_stride_head, int64_t q_rope_stride_seq,
+                                  int64_t q_rope_stride_head, int batch, int n_heads,
+                                  const int32_t* dev_seq_lens, const int32_t* dev_keep_idx,
+                                  const int32_t* dev_keep_len, int keep_stride,
+                                  float softmax_scale, float* out, float* lse,
+                                  kvk_stream_t stream);
+
 /* Copy the sticky device flags to *flags (synchronises the stream); clear != 0 resets them
  * to zero afterwards. */
 kvk_status kvk_read_status(kvk_layout* layout, uint32_t* flags, int clear, kvk_stream_t stream);
