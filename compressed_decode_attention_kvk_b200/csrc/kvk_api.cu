@@ -257,9 +257,10 @@ kvk_status kvk_quant_write(kvk_layout* L, int layer, const void* c_kv, int dtype
   return e == cudaSuccess ? KVK_OK : KVK_ERR_CUDA;
 }
 
-static int choose_path(const kvk_layout* L, const AnchorDesc& A, int dtype, int H) {
+static int choose_path(const kvk_layout* L, const AnchorDesc& A, int dtype, int H,
+                       bool has_keep) {
   if (L->path == KVK_PATH_CUDA_CORE) return KVK_PATH_CUDA_CORE;
-  bool tc = kvk::tc_supported(L, A, dtype, H);
+  bool tc = kvk::tc_supported(L, A, dtype, H, has_keep);
   if (L->path == KVK_PATH_TENSOR) return tc ? KVK_PATH_TENSOR : -1;
   return tc ? KVK_PATH_TENSOR : KVK_PATH_CUDA_CORE;
 }
@@ -277,10 +278,10 @@ kvk_status kvk_decode_workspace_bytes(const kvk_layout* L, int layer, int batch,
 }
 
 kvk_status kvk_decode_path_for(const kvk_layout* L, int layer, int dtype, int n_heads,
-                               int* path) {
+                               int has_keep, int* path) {
   if (!L || !path || layer < 0 || layer >= L->n_layers || n_heads < 1) return KVK_ERR_INVALID_ARG;
   if (dtype != KVK_F32 && dtype != KVK_BF16 && dtype != KVK_F16) return KVK_ERR_INVALID_ARG;
-  int p = choose_path(L, L->anchors[L->slot[layer]], dtype, n_heads);
+  int p = choose_path(L, L->anchors[L->slot[layer]], dtype, n_heads, has_keep != 0);
   if (p < 0) return KVK_ERR_UNSUPPORTED;
   *path = p;
   return KVK_OK;
@@ -314,7 +315,7 @@ kvk_status kvk_mla_decode(kvk_layout* L, int layer, const void* q_lat, const voi
       q_rope_stride_head % 8)
     return KVK_ERR_ALIGNMENT;
   const AnchorDesc& A = L->anchors[L->slot[layer]];
-  int path = choose_path(L, A, dtype, n_heads);
+  int path = choose_path(L, A, dtype, n_heads, dev_keep_idx != nullptr);
   if (path < 0) return KVK_ERR_UNSUPPORTED;
 
   kvk::DecodeArgs a;

@@ -1,12 +1,926 @@
-// kvk_decode_tc.cu -- tensor-core (tcgen05) split decode; see the kernel's header comment.
+// kvk_decode_tc.cu -- tensor-core (tcgen05) split decode over the packed KV-Kaizen cache.
+//
+// Computes the same partials as the CUDA-core kernel (kvk_decode_fma.cu): for every piece of
+// a sequence that the CTA owns, the running max m (log2 units), the weight sum
+// l = sum 2^(z2 - m) and the un-normalised output o = sum 2^(z2 - m) c_hat[:d], where
+// z2 = log2(e) * sigma * s_t * (q_lat . code_t[:d] + q_rope . code_t[d:])  (absorbed MLA
+// attention over the dequantised cache; KV-Kaizen "Background": each decode step reads the
+// whole cache).
+//
+// One persistent CTA per SM walks a balanced slice of the flattened token space in tiles of
+// 64 tokens.  Warp roles (352 threads):
+//   warps 0-3  softmax: read S from TMEM, per-token scale, lazy online softmax, write P
+//              (f16) to shared memory, rescale O in TMEM when a max grows, write partials
+//   warps 4-7  convert: packed b-bit codes -> f16 operand tiles (UMMA 128-byte-swizzled,
+//              K-major), staged query (power-of-two scaled into f16 range)
+//   warp 8     TMA producer: 128-feature groups of 64 packed rows into a ring
+//   warp 9     score-MMA issuer (one thread) and TMEM owner
+//   warp 10    output-MMA issuer (one thread)
+// Per tile:  S^T[64 tok x N1 heads]  = C[64 x n] . Q^T         (M=64, TMEM, f32)
+//            O^T[128 feat x N2 heads] += C^T[128 x 64] . P    (M=128 per 128 latent features)
+// The same shared-memory tiles of C serve both products (K-major for the first, MN-major for
+// the second); heads sit on N, so 40 heads cost N = 40 / 48, never M = 128.
+// Dequantisation: codes of b <= 8 bits are exact in f16; 16-bit codes are rounded to f16
+// (relative 2^-12).  The per-token scale s_t multiplies the S row and is folded into P as
+// p * s_t / S_max, with S_max a power of two >= every scale of the CTA's slice.
+// Every wait is bounded in time; on expiry the kernel records KVK_FLAG_TIMEOUT, drains its
+// own TMA loads and MMAs, frees TMEM and exits.
+#include <string.h>
+
 #include "kvk_decode_common.cuh"
+#include "kvk_sm100.cuh"
 
 namespace kvk {
+namespace {
 
-bool tc_supported(const kvk_layout*, const AnchorDesc&, int, int) { return false; }
+using namespace sm100;
 
-cudaError_t launch_decode_tc(const DecodeArgs&, const AnchorDesc&, int, int, cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int kThreads = 352;
+constexpr int kConvWarp0 = 4;
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;    // score MMAs; owns TMEM
+constexpr int kMma2Warp = 10;  // output MMAs
+constexpr int kTile = kTcTileTokens;   // 64
+constexpr int kAtom = 8192;            // 64 rows x 128 bytes (64 f16 features)
+constexpr int kPair = 2 * kAtom;       // 128 features
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kOCol0 = 128;       // O chunks at columns 128 + 64 p; S buffers at 0, 64
+constexpr uint64_t kLimitNs = 2000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kSmemLimit = 232448;
+// barriers besides the rings: s full/empty, P full/empty (2 each), q full/empty, o empty,
+// two MMA drains, softmax group sync, convert group sync, q seen
+constexpr int kFixedBars = 8 + 8;
+
+struct TcParams {
+  DecodeArgs a;
+  int N1, N2;           // N of the score MMA (heads rounded to 8) and of the output MMA (16)
+  int NP, NPd;          // 128-feature groups per row, and those holding latent features
+  int NQA, NK16;        // 64-feature query atoms, 16-feature K steps
+  int PR, RR, raw_slot; // ring slots (f16 groups, packed groups) and packed-group bytes
+  uint32_t off_p, off_pairs, off_raw, off_bar, off_misc;
+  uint32_t idesc1, idesc2;
+  int qdtype;           // KVK_BF16 or KVK_F16
+};
+
+struct Misc {
+  uint32_t tmem_base;
+  int abort;
+  float smax;
+  float qs_inv[2];
+  int vote[2][4];
+  float qred[4];
+  float m_ref[64];
+  float alpha[64];
+  float red[4][64];
+  int32_t scan_tmp[32];
+};
+
+struct Cursor {
+  int seq, pos, p0, p1, cnt, tile, piece;
+  bool valid, first, last;
+};
+
+__device__ __forceinline__ bool find_piece(Cursor& c, const int32_t* off, int batch, int64_t lo,
+                                           int64_t hi) {
+  while (c.seq < batch && off[c.seq] < hi) {
+    const int64_t s0 = max(lo, (int64_t)off[c.seq]), s1 = min(hi, (int64_t)off[c.seq + 1]);
+    if (s0 < s1) {
+      c.p0 = (int)(s0 - off[c.seq]);
+      c.p1 = (int)(s1 - off[c.seq]);
+      c.pos = c.p0;
+      return true;
+    }
+    ++c.seq;
+  }
+  return false;
+}
+__device__ __forceinline__ void set_tile(Cursor& c) {
+  c.cnt = min(kTile, c.p1 - c.pos);
+  c.first = (c.pos == c.p0);
+  c.last = (c.pos + kTile >= c.p1);
+}
+__device__ __forceinline__ void cursor_start(Cursor& c, int seq0, const int32_t* off, int batch,
+                                             int64_t lo, int64_t hi) {
+  c.seq = seq0;
+  c.tile = 0;
+  c.piece = 0;
+  c.valid = find_piece(c, off, batch, lo, hi);
+  if (c.valid) set_tile(c);
+}
+__device__ __forceinline__ void cursor_next(Cursor& c, const int32_t* off, int batch, int64_t lo,
+                                            int64_t hi) {
+  ++c.tile;
+  c.pos += kTile;
+  if (c.pos >= c.p1) {
+    ++c.seq;
+    ++c.piece;
+    c.valid = find_piece(c, off, batch, lo, hi);
+  }
+  if (c.valid) set_tile(c);
+}
+
+__device__ __forceinline__ bool wait_noabort(uint64_t* b, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try(b, parity)) {
+    if (globaltimer() - t0 > kLimitNs) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// two 16-bit offset-binary codes -> f16x2 of (u - 32768), rounded once:
+// code = (hi - 128) * 256 + lo with both parts exact in f16, fused multiply-add
+__device__ __forceinline__ uint32_t cvt_code16(uint32_t w) {
+  const __half2 hs = __hsub2(bits_h2(__byte_perm(w, 0x64u, 0x4341u)), __float2half2_rn(1152.f));
+  const __half2 ls = __hsub2(bits_h2(__byte_perm(w, 0x64u, 0x4240u)), __float2half2_rn(1024.f));
+  return h2_bits(__hfma2(hs, __float2half2_rn(256.f), ls));
+}
+// bytes of w selected by `sel` (each a field u < 1024) -> f16x2 of (u - bias), exact
+__device__ __forceinline__ uint32_t cvt_small(uint32_t w, uint32_t sel, __half2 bias) {
+  return h2_bits(__hsub2(bits_h2(__byte_perm(w, 0x64u, sel)), bias));
+}
+__device__ __forceinline__ uint32_t spread2(uint32_t x) {  // 4 x 2-bit fields -> 4 bytes
+  x = (x | (x << 12)) & 0x000F000Fu;
+  x = (x | (x << 6)) & 0x03030303u;
+  return x;
+}
+
+template <int BITS>
+__device__ __forceinline__ void convert_group(const uint8_t* rawslot, uint8_t* pair, int ct) {
+  if constexpr (BITS == 8) {
+    const __half2 bias = __float2half2_rn(1152.f);
+#pragma unroll 4
+    for (int i = ct; i < 1024; i += 128) {
+      const int r = i >> 4, g = i & 15;
+      const uint2 w = *reinterpret_cast<const uint2*>(rawslot + r * 128 +
+                                                      ((((g >> 1) ^ (r & 7))) << 4) + ((g & 1) << 3));
+      uint4 o;
+      o.x = cvt_small(w.x, 0x4140u, bias);
+      o.y = cvt_small(w.x, 0x4342u, bias);
+      o.z = cvt_small(w.y, 0x4140u, bias);
+      o.w = cvt_small(w.y, 0x4342u, bias);
+      *reinterpret_cast<uint4*>(pair + (g >> 3) * kAtom + r * 128 + (((g & 7) ^ (r & 7)) << 4)) = o;
+    }
+  } else if constexpr (BITS == 4) {
+    const __half2 bias = __float2half2_rn(1032.f);
+#pragma unroll 4
+    for (int i = ct; i < 1024; i += 128) {
+      const int r = i >> 4, g = i & 15;
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(
+          rawslot + r * 64 + (((g >> 2) ^ ((r >> 1) & 3)) << 4) + ((g & 3) << 2));
+      const uint32_t x = w & 0x0F0F0F0Fu, y = (w >> 4) & 0x0F0F0F0Fu;
+      const uint32_t u01 = __byte_perm(x, y, 0x5140u), u45 = __byte_perm(x, y, 0x7362u);
+      uint4 o;
+      o.x = cvt_small(u01, 0x4140u, bias);
+      o.y = cvt_small(u01, 0x4342u, bias);
+      o.z = cvt_small(u45, 0x4140u, bias);
+      o.w = cvt_small(u45, 0x4342u, bias);
+      *reinterpret_cast<uint4*>(pair + (g >> 3) * kAtom + r * 128 + (((g & 7) ^ (r & 7)) << 4)) = o;
+    }
+  } else if constexpr (BITS == 2) {
+    const __half2 bias = __float2half2_rn(1026.f);
+#pragma unroll 4
+    for (int i = ct; i < 1024; i += 128) {
+      const int r = i >> 4, g = i & 15;
+      const uint32_t w = *reinterpret_cast<const uint16_t*>(
+          rawslot + r * 32 + (((g >> 3) ^ ((r >> 2) & 1)) << 4) + ((g & 7) << 1));
+      const uint32_t u0 = spread2(w & 0xFFu), u1 = spread2(w >> 8);
+      uint4 o;
+      o.x = cvt_small(u0, 0x4140u, bias);
+      o.y = cvt_small(u0, 0x4342u, bias);
+      o.z = cvt_small(u1, 0x4140u, bias);
+      o.w = cvt_small(u1, 0x4342u, bias);
+      *reinterpret_cast<uint4*>(pair + (g >> 3) * kAtom + r * 128 + (((g & 7) ^ (r & 7)) << 4)) = o;
+    }
+  }
+}
+
+__device__ __forceinline__ void load8_bits(const uint4 u, int dtype, float (&v)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (dtype == KVK_BF16) {
+      v[2 * k] = __uint_as_float(w[k] << 16);
+      v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    } else {
+      const float2 f = __half22float2(bits_h2(w[k]));
+      v[2 * k] = f.x;
+      v[2 * k + 1] = f.y;
+    }
+  }
+}
+
+template <int BITS, int NH>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUtensorMap tmap) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const DecodeArgs& a = P.a;
+  uint8_t* q_s = smem;
+  uint8_t* p_s = smem + P.off_p;
+  uint8_t* pairs = smem + P.off_pairs;
+  uint8_t* raw = smem + P.off_raw;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.off_bar);
+  uint64_t* b_pfull = bars;               // [PR] group converted, visible to the tensor core
+  uint64_t* b_pempty = b_pfull + P.PR;    // [PR] group released by the MMAs
+  uint64_t* b_tfull = b_pempty + P.PR;    // [PR] 16-bit: TMA landed in the group slot
+  uint64_t* b_rfull = b_tfull + P.PR;     // [RR] packed group landed
+  uint64_t* b_rempty = b_rfull + P.RR;    // [RR] packed group consumed
+  uint64_t* b_sfull = b_rempty + P.RR;    // [2] scores ready in TMEM
+  uint64_t* b_sempty = b_sfull + 2;       // [2] scores read
+  uint64_t* b_Pfull = b_sempty + 2;       // [2] P written
+  uint64_t* b_Pempty = b_Pfull + 2;       // [2] output MMA of that P done
+  uint64_t* b_qfull = b_Pempty + 2;       // query staged
+  uint64_t* b_qempty = b_qfull + 1;       // query no longer read
+  uint64_t* b_oempty = b_qempty + 1;      // O read out by the epilogue
+  uint64_t* b_final = b_oempty + 1;       // MMA drain
+  uint64_t* b_ssync = b_final + 1;        // softmax group sync
+  uint64_t* b_csync = b_ssync + 1;        // convert group sync
+  uint64_t* b_qseen = b_csync + 1;        // softmax has taken the piece's query scale
+  uint64_t* b_final2 = b_qseen + 1;       // output-MMA drain (last of kFixedBars)
+  Misc* m = reinterpret_cast<Misc*>(smem + P.off_misc);
+  int32_t* off = reinterpret_cast<int32_t*>(m + 1);
+  volatile int* abort = &m->abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    for (int i = 0; i < P.PR; ++i) {
+      mbar_init(&b_pfull[i], 4);
+      mbar_init(&b_pempty[i], 1);
+      mbar_init(&b_tfull[i], 1);
+    }
+    for (int i = 0; i < P.RR; ++i) {
+      mbar_init(&b_rfull[i], 1);
+      mbar_init(&b_rempty[i], 4);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&b_sfull[i], 1);
+      mbar_init(&b_sempty[i], 4);
+      mbar_init(&b_Pfull[i], 4);
+      mbar_init(&b_Pempty[i], 1);
+    }
+    mbar_init(b_qfull, 4);
+    mbar_init(b_qempty, 1);
+    mbar_init(b_oempty, 4);
+    mbar_init(b_final, 1);
+    mbar_init(b_ssync, 128);
+    mbar_init(b_csync, 128);
+    mbar_init(b_qseen, 4);
+    mbar_init(b_final2, 1);
+    m->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&m->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kTmaWarp && lane == 0) tma_prefetch_desc(&tmap);
+  block_seq_offsets(a, off, m->scan_tmp);   // contains __syncthreads
+  if (blockIdx.x == 0)
+    for (int i = tid; i <= a.batch; i += kThreads) a.seq_off[i] = off[i];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = m->tmem_base;
+
+  const int64_t N = off[a.batch];
+  const int64_t lo = cta_lo(blockIdx.x, N, a.G), hi = cta_lo(blockIdx.x + 1, N, a.G);
+  int seq0 = 0;
+  {
+    int L = 0, H = a.batch;
+    while (L < H) {
+      const int mid = (L + H + 1) >> 1;
+      if (off[mid] <= lo) L = mid; else H = mid - 1;
+    }
+    seq0 = L;
+  }
+  const bool has_work = lo < hi;
+
+  if (has_work && warp == kTmaWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      Cursor c;
+      cursor_start(c, seq0, off, a.batch, lo, hi);
+      uint32_t cnt = 0;
+      const int slots = (BITS == 16) ? P.PR : P.RR;
+      while (c.valid && !*abort) {
+        const int row0 = c.seq * a.max_tokens + c.pos;
+        bool ok = true;
+        for (int p = 0; p < P.NP && ok; ++p) {
+          const uint32_t s = cnt % slots, ph = (cnt / slots) & 1u;
+          if (BITS == 16) {
+            if (!(ok = mbar_wait(&b_pempty[s], ph ^ 1u, abort, kLimitNs))) break;
+            const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
+            mbar_arrive_expect_tx(&b_tfull[s], nat * kAtom);
+            for (int t = 0; t < nat; ++t)
+              tma_load_2d(pairs + s * kPair + t * kAtom, &tmap, (2 * p + t) * 128, row0,
+                          &b_tfull[s]);
+          } else {
+            if (!(ok = mbar_wait(&b_rempty[s], ph ^ 1u, abort, kLimitNs))) break;
+            mbar_arrive_expect_tx(&b_rfull[s], P.raw_slot);
+            tma_load_2d(raw + s * P.raw_slot, &tmap, p * 16 * BITS, row0, &b_rfull[s]);
+          }
+          ++cnt;
+        }
+        if (!ok) break;
+        cursor_next(c, off, a.batch, lo, hi);
+      }
+      if (*abort) {  // let the loads already issued land before the block exits
+        const uint32_t first = cnt > (uint32_t)slots ? cnt - slots : 0u;
+        for (uint32_t k = first; k < cnt; ++k) {
+          const uint32_t s = k % slots, ph = (k / slots) & 1u;
+          wait_noabort(BITS == 16 ? &b_tfull[s] : &b_rfull[s], ph);
+        }
+      }
+    }
+  } else if (has_work && warp == kMmaWarp) {
+    // ------------------------------------------------------------------ score MMAs
+    // The whole warp runs the schedule (warp-uniform waits); one elected lane issues the
+    // MMAs in groups of four, and commits them.
+    Cursor g;
+    cursor_start(g, seq0, off, a.batch, lo, hi);
+    uint32_t pc = 0;
+    // descriptors of slot 0 / atom 0; every other operand differs only in its start address
+    // (bits 0-13, address >> 4), so each operand adds its byte offset >> 4
+    const uint64_t a0 = sdesc(smem_u32(pairs), 16u, 1024u, kLayoutSw128);
+    const uint64_t b0 = sdesc(smem_u32(q_s), 16u, 1024u, kLayoutSw128);
+    const uint32_t q_atom = (uint32_t)P.N1 * 128u;
+    bool ok = true;
+    while (g.valid && ok) {
+      const int sb = g.tile & 1;
+      ok = mbar_wait(&b_sempty[sb], ((uint32_t)(g.tile >> 1) & 1u) ^ 1u, abort, kLimitNs);
+      if (ok && g.first) ok = mbar_wait(b_qfull, (uint32_t)g.piece & 1u, abort, kLimitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      for (int p = 0; p < P.NP && ok; ++p) {
+        const uint32_t u = pc + p, s = u % P.PR;
+        ok = __all_sync(0xffffffffu, mbar_wait(&b_pfull[s], (u / P.PR) & 1u, abort, kLimitNs));
+        if (!ok) break;
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t) {
+          const int atom = 2 * p + t;
+          if (atom * 64 >= a.n) break;
+          const uint64_t ad = a0 + ((s * kPair + t * kAtom) >> 4);
+          const uint64_t bd = b0 + ((atom * q_atom) >> 4);
+          const int k0 = atom * 4;
+          if (k0 + 4 <= P.NK16) {
+            mma4_elect(tmem + 64u * sb, ad, 2u, bd, 2u, P.idesc1, k0 > 0 ? 1u : 0u);
+          } else {
+            for (int ks = 0; k0 + ks < P.NK16; ++ks)
+              mma1_elect(tmem + 64u * sb, ad + 2u * ks, bd + 2u * ks, P.idesc1, (k0 + ks) > 0);
+          }
+        }
+        if (p >= P.NPd) commit_elect(&b_pempty[s]);   // rope-only group: free after scores
+      }
+      if (!ok) break;
+      commit_elect(&b_sfull[sb]);
+      if (g.last) commit_elect(b_qempty);
+      pc += P.NP;
+      cursor_next(g, off, a.batch, lo, hi);
+    }
+    commit_elect(b_final);          // every MMA issued above has completed after this
+    if (lane == 0) wait_noabort(b_final, 0);
+    __syncwarp();
+  } else if (has_work && warp == kMma2Warp) {
+    // ------------------------------------------------------------------ output MMAs
+    Cursor g;
+    cursor_start(g, seq0, off, a.batch, lo, hi);
+    uint32_t pc = 0;
+    const uint32_t p_bytes = (uint32_t)kTile * P.N2 * 2u;
+    const uint32_t lbo_p = (uint32_t)P.N2 * 16u;
+    const uint64_t a0 = sdesc(smem_u32(pairs), kAtom, 1024u, kLayoutSw128);
+    const uint64_t b0 = sdesc(smem_u32(p_s), lbo_p, 128u, kLayoutNone);
+    bool ok = true;
+    while (g.valid && ok) {
+      const int sb = g.tile & 1;
+      ok = mbar_wait(&b_Pfull[sb], (uint32_t)(g.tile >> 1) & 1u, abort, kLimitNs);
+      if (ok && g.first && g.piece > 0)
+        ok = mbar_wait(b_oempty, (uint32_t)(g.piece - 1) & 1u, abort, kLimitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint64_t bd = b0 + ((sb * p_bytes) >> 4);
+      for (int p = 0; p < P.NPd; ++p) {
+        const uint32_t s = (pc + p) % P.PR;
+        // K = 64 tokens in four steps of 16: A advances 2048 bytes (two 8-row groups),
+        // B two core-matrix rows of P
+        mma4_elect(tmem + kOCol0 + 64u * p, a0 + ((s * kPair) >> 4), 2048u >> 4, bd,
+                   (2u * lbo_p) >> 4, P.idesc2, g.first ? 0u : 1u);
+        commit_elect(&b_pempty[s]);
+      }
+      commit_elect(&b_Pempty[sb]);
+      pc += P.NP;
+      cursor_next(g, off, a.batch, lo, hi);
+    }
+    commit_elect(b_final2);
+    if (lane == 0) wait_noabort(b_final2, 0);
+    __syncwarp();
+  } else if (has_work && warp >= kConvWarp0) {
+    // ------------------------------------------------------------------ convert
+    // The four convert warps leave their loop only together (named_or agreement at the top
+    // of every tile), so their named barriers never wait for a warp that has gone.
+    const int ct = tid - kConvWarp0 * 32, cw = warp - kConvWarp0;
+    uint32_t pc = 0, rc = 0;
+    int last_piece = -1;
+    bool fail = false;
+    const int cpr = P.NQA * 8;   // 16-byte chunks per staged query row
+    {  // warm L2 with the queries of every sequence this CTA touches
+      Cursor c;
+      cursor_start(c, seq0, off, a.batch, lo, hi);
+      while (c.valid) {
+        const uint8_t* ql = static_cast<const uint8_t*>(a.q_lat) + 2 * ((int64_t)c.seq * a.ql_ss);
+        const uint8_t* qr = static_cast<const uint8_t*>(a.q_rope) + 2 * ((int64_t)c.seq * a.qr_ss);
+        const int lat_lines = (2 * a.d + 127) / 128, rope_lines = (2 * a.d_rope + 127) / 128;
+        for (int i = ct; i < a.H * (lat_lines + rope_lines); i += 128) {
+          const int h = i / (lat_lines + rope_lines), k = i - h * (lat_lines + rope_lines);
+          if (k < lat_lines) prefetch_l2(ql + 2 * ((int64_t)h * a.ql_sh) + 128 * k);
+          else prefetch_l2(qr + 2 * ((int64_t)h * a.qr_sh) + 128 * (k - lat_lines));
+        }
+        ++c.seq;
+        c.valid = find_piece(c, off, a.batch, lo, hi);
+      }
+    }
+    Cursor c;
+    cursor_start(c, seq0, off, a.batch, lo, hi);
+    while (c.valid) {
+      if (named_or(2, 128, fail || *abort)) break;
+      if (c.piece != last_piece) {
+        // Stage this sequence's query as f16 rows [N1][n], scaled by 2^e so that max |q|
+        // lands in [2^14, 2^15) (exact for bf16 inputs in range); rows >= H and features
+        // >= n are zero.  Wait until the previous piece's scores no longer read it and the
+        // softmax warps have taken the previous piece's scale (bounds q_full to one phase
+        // ahead of its slowest waiter).
+        fail = fail || !mbar_wait(b_qempty, ((uint32_t)c.piece & 1u) ^ 1u, abort, kLimitNs);
+        if (c.piece > 0)
+          fail = fail || !mbar_wait(b_qseen, ((uint32_t)c.piece - 1u) & 1u, abort, kLimitNs);
+        const uint8_t* qlat = static_cast<const uint8_t*>(a.q_lat) + 2 * ((int64_t)c.seq * a.ql_ss);
+        const uint8_t* qrope =
+            static_cast<const uint8_t*>(a.q_rope) + 2 * ((int64_t)c.seq * a.qr_ss);
+        auto src = [&](int h, int f0) -> const uint4* {
+          return reinterpret_cast<const uint4*>(
+              (f0 < a.d) ? qlat + 2 * ((int64_t)h * a.ql_sh + f0)
+                         : qrope + 2 * ((int64_t)h * a.qr_sh + (f0 - a.d)));
+        };
+        float mx = 0.f;
+        const int nch = a.H * cpr;
+        for (int base = ct; base < nch; base += 128 * 8) {
+          uint4 v[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {   // eight independent loads in flight
+            const int i = base + 128 * k;
+            const int h = i / cpr, f0 = (i - h * cpr) * 8;
+            v[k] = (i < nch && f0 < a.n) ? *src(h, f0) : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            float f[8];
+            load8_bits(v[k], P.qdtype, f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) m->qred[cw] = mx;
+        named_sync(2, 128);
+        mx = fmaxf(fmaxf(m->qred[0], m->qred[1]), fmaxf(m->qred[2], m->qred[3]));
+        const int e = (mx > 0.f && isfinite(mx)) ? 14 - ilogbf(mx) : 0;
+        const float qscale = ldexpf(1.f, e);
+        if (ct == 0) m->qs_inv[c.piece & 1] = ldexpf(1.f, -e);
+        const int nst = P.N1 * cpr;
+        for (int base = ct; base < nst; base += 128 * 8) {
+          uint4 v[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int i = base + 128 * k;
+            const int h = i / cpr, f0 = (i - h * cpr) * 8;
+            v[k] = (i < nst && h < a.H && f0 < a.n) ? *src(h, f0) : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int i = base + 128 * k;
+            if (i >= nst) continue;
+            const int h = i / cpr, fc = i - h * cpr;
+            float f[8];
+            load8_bits(v[k], P.qdtype, f);
+            uint4 o;
+            o.x = h2_bits(__floats2half2_rn(f[0] * qscale, f[1] * qscale));
+            o.y = h2_bits(__floats2half2_rn(f[2] * qscale, f[3] * qscale));
+            o.z = h2_bits(__floats2half2_rn(f[4] * qscale, f[5] * qscale));
+            o.w = h2_bits(__floats2half2_rn(f[6] * qscale, f[7] * qscale));
+            const int at = fc >> 3, j = fc & 7;
+            *reinterpret_cast<uint4*>(q_s + at * (P.N1 * 128) + h * 128 + ((j ^ (h & 7)) << 4)) = o;
+          }
+        }
+        fence_proxy_async_smem();
+        named_sync(2, 128);   // every warp's rows written (and qred read) before q_full
+        if (lane == 0) mbar_arrive(b_qfull);
+        last_piece = c.piece;
+      }
+      for (int p = 0; p < P.NP; ++p) {
+        const uint32_t s = pc % P.PR, ph = (pc / P.PR) & 1u;
+        uint8_t* pair = pairs + s * kPair;
+        if constexpr (BITS == 16) {
+          fail = fail || !mbar_wait(&b_tfull[s], ph, abort, kLimitNs);
+          const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
+          if (!fail) {
+#pragma unroll 4
+            for (int i = ct; i < nat * 512; i += 128) {   // in place: 16-bit codes -> f16
+              uint4* q4 = reinterpret_cast<uint4*>(pair + i * 16);
+              uint4 v = *q4;
+              v.x = cvt_code16(v.x);
+              v.y = cvt_code16(v.y);
+              v.z = cvt_code16(v.z);
+              v.w = cvt_code16(v.w);
+              *q4 = v;
+            }
+          }
+        } else {
+          const uint32_t rs = rc % P.RR, rph = (rc / P.RR) & 1u;
+          fail = fail || !mbar_wait(&b_rfull[rs], rph, abort, kLimitNs);
+          fail = fail || !mbar_wait(&b_pempty[s], ph ^ 1u, abort, kLimitNs);
+          if (!fail) convert_group<BITS>(raw + rs * P.raw_slot, pair, ct);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b_rempty[rs]);
+          ++rc;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b_pfull[s]);
+        ++pc;
+      }
+      cursor_next(c, off, a.batch, lo, hi);
+    }
+  } else if (has_work) {
+    // ------------------------------------------------------------------ softmax
+    // TMEM holds S^T with tokens on lanes: the M = 64 layout puts rows 16q .. 16q+15 in
+    // lanes 32q .. 32q+15.  Loaded with the 16x256b shape, thread t of warp q holds rows
+    // ra = 16q + t/4 and rb = ra + 8, heads 8j + 2(t%4) + {0, 1} of every 8-head block j.
+    // The four warps leave the loop only together (named_or agreement every tile).
+    constexpr int NB = NH / 8;
+    const int q = warp;
+    const uint32_t lb = tmem + ((uint32_t)(32 * q) << 16);
+    const int ra = 16 * q + (lane >> 2), rb = ra + 8;
+    const int hc = 2 * (lane & 3);
+    bool fail = false;
+
+    // S_max: power of two >= every scale in the CTA's slice (keeps p * s / S_max <= 2^8)
+    float smx = 0.f;
+    {
+      Cursor c;
+      cursor_start(c, seq0, off, a.batch, lo, hi);
+      while (c.valid) {
+        const __half* sp = a.scales + (int64_t)c.seq * a.max_tokens;
+        for (int base = c.p0 + tid; base < c.p1; base += 128 * 8) {
+          __half hv[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int pp = base + 128 * k;
+            hv[k] = pp < c.p1 ? sp[pp] : __float2half(0.f);
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) smx = fmaxf(smx, __half2float(hv[k]));
+        }
+        ++c.seq;
+        c.valid = find_piece(c, off, a.batch, lo, hi);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) smx = fmaxf(smx, __shfl_xor_sync(0xffffffffu, smx, o));
+    if (lane == 0) m->red[q][0] = smx;
+    named_sync(1, 128);
+    smx = fmaxf(fmaxf(m->red[0][0], m->red[1][0]), fmaxf(m->red[2][0], m->red[3][0]));
+    float smax = 1.f;
+    if (smx > 0.f && isfinite(smx)) {
+      int ex;
+      const float fr = frexpf(smx, &ex);             // smx = fr * 2^ex, fr in [0.5, 1)
+      smax = (fr == 0.5f) ? smx : ldexpf(1.f, ex);
+    }
+    const float inv_smax = 1.f / smax;
+
+    float l[2 * NB];    // partial weight sums of this thread's heads
+    float mr[2 * NB];   // reference max of this thread's heads (log2 units)
+    float qs_inv = 1.f;
+    int pt = 0;
+    Cursor c;
+    cursor_start(c, seq0, off, a.batch, lo, hi);
+    const float coef0 = a.sigma * kLog2e;
+    const uint32_t p_bytes = (uint32_t)kTile * P.N2 * 2u;
+    while (c.valid) {
+      const int t = c.tile, sb = t & 1;
+      if (c.first) {
+        fail = fail || !mbar_wait(b_qfull, (uint32_t)c.piece & 1u, abort, kLimitNs);
+        qs_inv = m->qs_inv[c.piece & 1];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b_qseen);
+#pragma unroll
+        for (int i = 0; i < 2 * NB; ++i) {
+          l[i] = 0.f;
+          mr[i] = -INFINITY;
+        }
+        pt = 0;
+      }
+      const bool va = ra < c.cnt, vb = rb < c.cnt;
+      const __half* sp = a.scales + (int64_t)c.seq * a.max_tokens + c.pos;
+      const float s_a = va ? __half2float(sp[ra]) : 0.f;
+      const float s_b = vb ? __half2float(sp[rb]) : 0.f;
+      const float ca = coef0 * s_a * qs_inv, cbf = coef0 * s_b * qs_inv;
+      fail = fail || !mbar_wait(&b_sfull[sb], (uint32_t)(t >> 1) & 1u, abort, kLimitNs);
+      tc_fence_after();
+      float x[4 * NB];
+      if constexpr (NB >= 6) {
+        float v[32];
+        tmem_ld16x256b_x8(lb + 64u * sb, v);
+#pragma unroll
+        for (int i = 0; i < 4 * NB; ++i) x[i] = v[i];
+      } else if constexpr (NB == 4) {
+        float v[16];
+        tmem_ld16x256b_x4(lb + 64u * sb, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = v[i];
+      } else {
+        float v[8];
+        tmem_ld16x256b_x2(lb + 64u * sb, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = v[i];
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b_sempty[sb]);
+      bool mine = (pt == 0);
+#pragma unroll
+      for (int j = 0; j < NB; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const bool hv = (8 * j + hc + e) < a.H;
+          x[4 * j + e] = (va && hv) ? x[4 * j + e] * ca : -INFINITY;
+          x[4 * j + 2 + e] = (vb && hv) ? x[4 * j + 2 + e] * cbf : -INFINITY;
+          mine = mine || (x[4 * j + e] > mr[2 * j + e] + 8.f) ||
+                 (x[4 * j + 2 + e] > mr[2 * j + e] + 8.f);
+        }
+      }
+      // lazy running max: recompute (and rescale) only when a score exceeds the reference
+      // by more than 2^8, so P stays within f16 range without touching O every tile
+      if (named_or(1, 128, mine || fail || *abort)) {
+        if (named_or(1, 128, fail || *abort)) break;
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            float v = fmaxf(x[4 * j + e], x[4 * j + 2 + e]);
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+            if (lane < 4) m->red[q][8 * j + 2 * lane + e] = v;
+          }
+        }
+        named_sync(1, 128);
+        if (tid < NH) {   // one thread per head: new reference and the factor for old sums
+          const float tm = fmaxf(fmaxf(m->red[0][tid], m->red[1][tid]),
+                                 fmaxf(m->red[2][tid], m->red[3][tid]));
+          const float mo = (pt == 0) ? -INFINITY : m->m_ref[tid];
+          const float mn = fmaxf(mo, tm);
+          m->alpha[tid] = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+          m->m_ref[tid] = mn;
+        }
+        named_sync(1, 128);
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) mr[2 * j + e] = m->m_ref[8 * j + hc + e];
+        }
+        if (pt > 0) {
+#pragma unroll
+          for (int j = 0; j < NB; ++j) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) l[2 * j + e] *= m->alpha[8 * j + hc + e];
+          }
+          // rescale O once the previous tile's output MMAs are done
+          const int tp = t - 1;
+          fail = fail ||
+                 !mbar_wait(&b_Pempty[tp & 1], (uint32_t)(tp >> 1) & 1u, abort, kLimitNs);
+          tc_fence_after();
+          for (int p = 0; p < P.NPd; ++p) {
+#pragma unroll
+            for (int cb = 0; cb < NH; cb += 8) {
+              float v[8];
+              const uint32_t ta = lb + kOCol0 + 64u * p + cb;
+              tmem_ld8(ta, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int k = 0; k < 8; ++k) v[k] *= m->alpha[cb + k];
+              tmem_st8(ta, v);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+        }
+      }
+
+      // P tile (MN-major core matrices): row r, heads 8j..8j+7 at (r/8)*16*N2 + 128j +
+      // (r%8)*16; this thread's word for heads 8j + hc + {0, 1} of row ra is at
+      // 32 q N2 + 128 j + 4 lane, of row rb 16 N2 further
+      fail = fail || !mbar_wait(&b_Pempty[sb], ((uint32_t)(t >> 1) & 1u) ^ 1u, abort, kLimitNs);
+      {
+        const float wa = s_a * inv_smax, wb = s_b * inv_smax;
+        uint8_t* pa = p_s + sb * p_bytes + 32 * q * P.N2 + 4 * lane;
+        uint8_t* pbp = pa + 16 * P.N2;
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          float ea[2], eb[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float m0 = mr[2 * j + e];
+            const float xa = x[4 * j + e], xb = x[4 * j + 2 + e];
+            ea[e] = (xa == -INFINITY || m0 == -INFINITY) ? 0.f : exp2f(xa - m0);
+            eb[e] = (xb == -INFINITY || m0 == -INFINITY) ? 0.f : exp2f(xb - m0);
+            l[2 * j + e] += ea[e] + eb[e];
+          }
+          *reinterpret_cast<uint32_t*>(pa + 128 * j) = h2_bits(__floats2half2_rn(ea[0] * wa, ea[1] * wa));
+          *reinterpret_cast<uint32_t*>(pbp + 128 * j) = h2_bits(__floats2half2_rn(eb[0] * wb, eb[1] * wb));
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b_Pfull[sb]);
+      ++pt;
+
+      if (c.last) {
+        // -------- epilogue of the piece: partials to the workspace slot blockIdx.x + seq
+        fail = fail || !mbar_wait(&b_Pempty[sb], (uint32_t)(t >> 1) & 1u, abort, kLimitNs);
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            float v = l[2 * j + e];
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            v += __shfl_xor_sync(0xffffffffu, v, 8);
+            v += __shfl_xor_sync(0xffffffffu, v, 16);
+            if (lane < 4) m->red[q][8 * j + 2 * lane + e] = v;
+          }
+        }
+        named_sync(1, 128);
+        const int64_t slot = (int64_t)blockIdx.x + c.seq;
+        for (int h = tid; h < a.H; h += 128) {
+          const float L = (m->red[0][h] + m->red[1][h]) + (m->red[2][h] + m->red[3][h]);
+          a.ws_ml[2 * (slot * a.H + h)] = m->m_ref[h];
+          a.ws_ml[2 * (slot * a.H + h) + 1] = L;
+        }
+        if (!fail) {
+          for (int p = 0; p < P.NPd; ++p) {
+            const int f = 128 * p + 32 * q + lane;
+#pragma unroll
+            for (int cb = 0; cb < NH; cb += 8) {
+              float v[8];
+              tmem_ld8(lb + kOCol0 + 64u * p + cb, v);
+              tmem_wait_ld();
+              if (f < a.d) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                  const int h = cb + k;
+                  if (h < a.H) a.ws_o[(slot * a.H + h) * a.d + f] = v[k] * smax;
+                }
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b_oempty);
+        named_sync(1, 128);   // red / m_ref reads done before the next piece writes them
+      }
+      cursor_next(c, off, a.batch, lo, hi);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && *abort) atomicOr(a.flags, KVK_FLAG_TIMEOUT);
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------
+
+struct Plan {
+  TcParams p;
+  size_t smem;
+  bool ok;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+Plan make_plan(int d, int d_rope, int b, int H, int batch) {
+  Plan pl;
+  memset(&pl, 0, sizeof(pl));
+  TcParams& P = pl.p;
+  const int n = d + d_rope;
+  P.N1 = (H + 7) / 8 * 8;
+  P.N2 = (H + 15) / 16 * 16;
+  P.NP = (n + 127) / 128;
+  P.NPd = (d + 127) / 128;
+  P.NQA = (n + 63) / 64;
+  P.NK16 = (n + 15) / 16;
+  if (H < 1 || P.N2 > 64 || P.NPd > 6) return pl;
+  const size_t q_bytes = (size_t)P.NQA * P.N1 * 128;
+  const size_t p_bytes = 2 * (size_t)kTile * P.N2 * 2;
+  const size_t misc_bytes = sizeof(Misc) + sizeof(int32_t) * (size_t)(batch + 1);
+  const int raw_slot = (b == 16) ? 0 : 64 * 16 * b;
+  P.raw_slot = raw_slot;
+  // try the largest rings that fit
+  const size_t fixed = align_up(q_bytes, 1024) + align_up(p_bytes, 1024);
+  auto total_for = [&](int PR, int RR) {
+    size_t off = fixed;
+    off += (size_t)PR * kPair;
+    off = align_up(off + (size_t)RR * raw_slot, 1024);
+    off = align_up(off + (size_t)(3 * PR + 2 * RR + kFixedBars) * 8, 16);
+    off += misc_bytes;
+    return off + 1024;   // runtime alignment slack of the dynamic shared memory base
+  };
+  int PR = 0, RR = 0;
+  if (b == 16) {
+    for (PR = 3 * P.NP; PR >= P.NP; --PR)
+      if (total_for(PR, 0) <= (size_t)kSmemLimit) break;
+  } else {
+    const int want = P.NP + (P.NP + 1) / 2;
+    for (PR = want; PR >= P.NP; --PR) {
+      for (RR = 4 * P.NP; RR >= 2; --RR)
+        if (total_for(PR, RR) <= (size_t)kSmemLimit) break;
+      if (RR >= 2 && total_for(PR, RR) <= (size_t)kSmemLimit) break;
+    }
+  }
+  if (PR < P.NP || (b != 16 && RR < 2)) return pl;
+  P.PR = PR;
+  P.RR = RR;
+  size_t off = fixed;
+  P.off_p = (uint32_t)align_up(q_bytes, 1024);
+  P.off_pairs = (uint32_t)fixed;
+  off += (size_t)PR * kPair;
+  P.off_raw = (uint32_t)off;
+  off = align_up(off + (size_t)RR * raw_slot, 1024);
+  P.off_bar = (uint32_t)off;
+  off = align_up(off + (size_t)(3 * PR + 2 * RR + kFixedBars) * 8, 16);
+  P.off_misc = (uint32_t)off;
+  pl.smem = off + misc_bytes + 1024;
+  P.idesc1 = sm100::idesc_f16(64, P.N1, false, false);
+  P.idesc2 = sm100::idesc_f16(128, P.N2, true, true);
+  pl.ok = pl.smem <= (size_t)kSmemLimit;
+  return pl;
+}
+
+template <int BITS, int NH>
+cudaError_t launch_bits_nh(const TcParams& P, const CUtensorMap& tmap, size_t smem, int grid,
+                           cudaStream_t st) {
+  auto k = decode_tc_kernel<BITS, NH>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, kThreads, smem, st>>>(P, tmap);
+  return cudaGetLastError();
+}
+
+template <int BITS>
+cudaError_t launch_bits(const TcParams& P, const CUtensorMap& tmap, size_t smem, int grid,
+                        cudaStream_t st) {
+  switch (P.N2) {
+    case 16: return launch_bits_nh<BITS, 16>(P, tmap, smem, grid, st);
+    case 32: return launch_bits_nh<BITS, 32>(P, tmap, smem, grid, st);
+    case 48: return launch_bits_nh<BITS, 48>(P, tmap, smem, grid, st);
+    case 64: return launch_bits_nh<BITS, 64>(P, tmap, smem, grid, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H, bool has_keep) {
+  if (dtype != KVK_BF16 && dtype != KVK_F16) return false;
+  if (has_keep || !A.tmap_ok) return false;
+  return make_plan(A.d, L->d_rope, A.b, H, L->max_batch).ok;
+}
+
+cudaError_t launch_decode_tc(const DecodeArgs& a, const AnchorDesc& A, int dtype, int,
+                             cudaStream_t st) {
+  Plan pl = make_plan(a.d, a.d_rope, a.b, a.H, a.batch);
+  if (!pl.ok) return cudaErrorInvalidValue;
+  pl.p.a = a;
+  pl.p.qdtype = dtype;
+  switch (a.b) {
+    case 16: return launch_bits<16>(pl.p, A.tmap_tile, pl.smem, a.G, st);
+    case 8: return launch_bits<8>(pl.p, A.tmap_tile, pl.smem, a.G, st);
+    case 4: return launch_bits<4>(pl.p, A.tmap_tile, pl.smem, a.G, st);
+    case 2: return launch_bits<2>(pl.p, A.tmap_tile, pl.smem, a.G, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace kvk

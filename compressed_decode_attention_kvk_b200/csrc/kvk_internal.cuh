@@ -93,7 +93,7 @@ cudaError_t launch_quant_write(const kvk_layout* L, const AnchorDesc& A, const v
 cudaError_t launch_decode_fma(const DecodeArgs& a, int dtype, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeArgs& a, const AnchorDesc& A, int dtype, int num_sms,
                              cudaStream_t stream);
-bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H);
+bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H, bool has_keep);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
 
 // Position -> CTA of the balanced split: CTA c owns [c*N/G, (c+1)*N/G).

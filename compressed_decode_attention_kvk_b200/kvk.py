@@ -24,6 +24,7 @@ STATUS_NAMES = {0: "KVK_OK", 1: "KVK_ERR_INVALID_ARG", 2: "KVK_ERR_BAD_TABLE",
 KVK_F32, KVK_BF16, KVK_F16 = 0, 1, 2
 KVK_PATH_AUTO, KVK_PATH_TENSOR, KVK_PATH_CUDA_CORE = 0, 1, 2
 KVK_FLAG_NONFINITE, KVK_FLAG_WRITE_RANGE, KVK_FLAG_SEQ_LEN, KVK_FLAG_KEEP_INDEX = 1, 2, 4, 8
+KVK_FLAG_TIMEOUT = 16
 
 _DTYPE = {torch.float32: KVK_F32, torch.bfloat16: KVK_BF16, torch.float16: KVK_F16}
 
@@ -76,7 +77,7 @@ def _lib_handle():
         L.kvk_read_status.argtypes = [P, P, i32, P]
         L.kvk_set_decode_path.argtypes = [P, i32]
         L.kvk_set_decode_ctas.argtypes = [P, i32]
-        L.kvk_decode_path_for.argtypes = [P, i32, i32, i32, P]
+        L.kvk_decode_path_for.argtypes = [P, i32, i32, i32, i32, P]
         L.kvk_status_string.argtypes = [i32]
         L.kvk_status_string.restype = ctypes.c_char_p
         for name in EXPORTED:
@@ -241,10 +242,10 @@ def kvk_set_decode_ctas(handle, ctas):
     _check("kvk_set_decode_ctas", _lib_handle().kvk_set_decode_ctas(handle, ctas))
 
 
-def kvk_decode_path_for(handle, layer, dtype, n_heads) -> int:
+def kvk_decode_path_for(handle, layer, dtype, n_heads, has_keep=False) -> int:
     p = ctypes.c_int(0)
     _check("kvk_decode_path_for", _lib_handle().kvk_decode_path_for(
-        handle, layer, _DTYPE.get(dtype, dtype), n_heads, ctypes.byref(p)))
+        handle, layer, _DTYPE.get(dtype, dtype), n_heads, 1 if has_keep else 0, ctypes.byref(p)))
     return p.value
 
 
@@ -330,8 +331,8 @@ class Layout:
     def set_decode_ctas(self, ctas):
         kvk_set_decode_ctas(self.handle, ctas)
 
-    def decode_path_for(self, layer, dtype, n_heads):
-        return kvk_decode_path_for(self.handle, layer, dtype, n_heads)
+    def decode_path_for(self, layer, dtype, n_heads, has_keep=False):
+        return kvk_decode_path_for(self.handle, layer, dtype, n_heads, has_keep)
 
     def close(self):
         if getattr(self, "handle", None):

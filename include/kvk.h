@@ -59,6 +59,8 @@ typedef enum { KVK_F32 = 0, KVK_BF16 = 1, KVK_F16 = 2 } kvk_dtype;
 #define KVK_FLAG_SEQ_LEN     0x4u /* decode: seq_len outside [0, max_tokens], clamped; or keep_len
                                      outside [0, keep_stride], clamped                             */
 #define KVK_FLAG_KEEP_INDEX  0x8u /* decode: keep index outside [0, seq_len); entry skipped        */
+#define KVK_FLAG_TIMEOUT     0x10u /* decode: a tensor-core kernel wait exceeded its time limit and
+                                      the kernel stopped early; that call's outputs are unspecified */
 
 /* Decode kernel selection (kvk_set_decode_path). */
 #define KVK_PATH_AUTO      0 /* tensor-core kernel where it applies, else the CUDA-core kernel  */
@@ -81,7 +83,8 @@ typedef enum { KVK_F32 = 0, KVK_BF16 = 1, KVK_F16 = 2 } kvk_dtype;
  *   d[L], b[L]          for anchors: 16 <= d <= r, d % 16 == 0; b in {2, 4, 8, 16}.
  *                       Ignored for inheriting layers.
  *   r, d_rope           latent width (multiple of 16) and RoPE width (multiple of 8, >= 0)
- *   max_batch, max_tokens  capacity of every anchor's cache (max_batch * max_tokens < 2^31)
+ *   max_batch, max_tokens  capacity of every anchor's cache (max_batch <= 4096,
+ *                       max_batch * max_tokens < 2^31)
  *   budget_bits_per_token  <= 0: no check; else KVK_ERR_BUDGET when the plan costs more
  *   dev_arena, arena_bytes caller-owned device memory (256-byte aligned), size >= needed
  *   out                 receives the handle; NULL = query only (sizes and bits filled in)
@@ -235,9 +238,9 @@ kvk_status kvk_set_decode_path(kvk_layout* layout, int path);
 kvk_status kvk_set_decode_ctas(kvk_layout* layout, int ctas);
 
 /* Which kernel kvk_mla_decode would run for these arguments (KVK_PATH_TENSOR or
- * KVK_PATH_CUDA_CORE), without launching anything. */
+ * KVK_PATH_CUDA_CORE), without launching anything.  has_keep != 0: a keep list is given. */
 kvk_status kvk_decode_path_for(const kvk_layout* layout, int layer, int dtype, int n_heads,
-                               int* path);
+                               int has_keep, int* path);
 
 /* Static description of a status code. */
 const char* kvk_status_string(kvk_status status);

@@ -136,7 +136,7 @@ def test_planning_layout_cannot_launch(kvk):
         assert ws.value > 0
         assert lib.kvk_decode_workspace_bytes(handle, 1, 2, 8, ctypes.byref(ws)) == 1  # batch > max
         path = ctypes.c_int(-1)
-        assert lib.kvk_decode_path_for(handle, 0, 0, 8, ctypes.byref(path)) == 0
+        assert lib.kvk_decode_path_for(handle, 0, 0, 8, 0, ctypes.byref(path)) == 0
         assert path.value == kvk.KVK_PATH_CUDA_CORE            # fp32 queries
         assert lib.kvk_set_decode_path(handle, 7) == 1
         assert lib.kvk_set_decode_ctas(handle, -1) == 1

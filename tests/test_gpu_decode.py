@@ -40,12 +40,12 @@ def _decode(case, layer, ql, qr, lens, sigma, path, ctas=0, keep=None, keep_len=
     return out.cpu().numpy(), lse.cpu().numpy()
 
 
-def _paths(pkg, case, dtype, H):
+def _paths(pkg, case, dtype, H, has_keep=False):
     """Decode kernels that run this shape: always the CUDA-core one, plus the tensor one."""
     ps = [2]
     case.lay.set_decode_path(1)
     try:
-        if case.lay.decode_path_for(0, dtype, H) == 1:
+        if case.lay.decode_path_for(0, dtype, H, has_keep) == 1:
             ps.append(1)
     except pkg.KvkError:
         pass
@@ -187,7 +187,7 @@ def test_keep_list_equals_compacted_cache(pkg, oracle_mod):
         sigma = 1 / math.sqrt(d + dR)
         ref_cache = oracle_cache(oracle_mod, c, kr, d, 8)
         keep_t = torch.from_numpy(keep)
-        for path in _paths(pkg, case, torch.bfloat16, H):
+        for path in _paths(pkg, case, torch.bfloat16, H, has_keep=True):
             out, lse = _decode(case, 0, ql, qr, torch.tensor(lens, dtype=torch.int32), sigma,
                                path, keep=keep_t, keep_len=torch.tensor(klen, dtype=torch.int32))
             for i in range(B):
