@@ -12,14 +12,19 @@
 //   warps 0-3  softmax: read S from TMEM, per-token scale, lazy online softmax, write P
 //              (f16) to shared memory, rescale O in TMEM when a max grows, write partials
 //   warps 4-7  convert: packed b-bit codes -> f16 operand tiles (UMMA 128-byte-swizzled,
-//              K-major), staged query (power-of-two scaled into f16 range)
+//              K-major) and their transpose into TMEM; staged query (power-of-two scaled)
 //   warp 8     TMA producer: 128-feature groups of 64 packed rows into a ring
 //   warp 9     score-MMA issuer (one thread) and TMEM owner
 //   warp 10    output-MMA issuer (one thread)
-// Per tile:  S^T[64 tok x N1 heads]  = C[64 x n] . Q^T         (M=64, TMEM, f32)
-//            O^T[128 feat x N2 heads] += C^T[128 x 64] . P    (M=128 per 128 latent features)
-// The same shared-memory tiles of C serve both products (K-major for the first, MN-major for
-// the second); heads sit on N, so 40 heads cost N = 40 / 48, never M = 128.
+// Per tile:  S^T[64 tok x N1 heads]  = C[64 x n] . Q^T         (M=64, A in smem, TMEM f32)
+//            O^T[128 feat x N2 heads] += C^T[128 x 64] . P    (M=128 per 128 latent features,
+//                                                               A = C^T in TMEM)
+// Heads sit on N, so 40 heads cost N = 40 / 48, never M = 128.  After the convert warps have
+// turned a 128-feature group into f16 (UMMA 128-byte swizzled, K-major: the score MMA's A),
+// each of them transposes its 32 features of it into TMEM (ldmatrix.trans -> tcgen05.st),
+// so a ring slot is free as soon as the score MMA has read it; the output MMA reads TMEM.
+// The transpose fragment orders the 16 tokens of each K step as 0,1,8,9,2,3,10,11,4,5,12,13,
+// 6,7,14,15; the softmax warps write P's K rows in that same order.
 // Dequantisation: codes of b <= 8 bits are exact in f16; 16-bit codes are rounded to f16
 // (relative 2^-12).  The per-token scale s_t multiplies the S row and is folded into P as
 // p * s_t / S_max, with S_max a power of two >= every scale of the CTA's slice.
@@ -44,13 +49,17 @@ constexpr int kTile = kTcTileTokens;   // 64
 constexpr int kAtom = 8192;            // 64 rows x 128 bytes (64 f16 features)
 constexpr int kPair = 2 * kAtom;       // 128 features
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kOCol0 = 128;       // O chunks at columns 128 + 64 p; S buffers at 0, 64
+constexpr uint32_t kSCol = 0;          // scores S^T, one buffer (N1 <= 64 columns)
+constexpr uint32_t kCtCol0 = 64;       // C^T double buffer: 64 + 128 b, latent group p at + 32 p
+constexpr uint32_t kOCol0 = 320;       // O^T group p at 320 + N2 p
 constexpr uint64_t kLimitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kSmemLimit = 232448;
-// barriers besides the rings: s full/empty, P full/empty (2 each), q full/empty, o empty,
-// two MMA drains, softmax group sync, convert group sync, q seen
-constexpr int kFixedBars = 8 + 8;
+constexpr int kQH = 5;   // query rows a convert warp loads per round
+constexpr int kQC = 4;   // 16-byte chunks per lane per query row (rows of up to 1024 features)
+// barriers besides the rings: s full/empty, P full/empty (2), C^T full/empty (2), q full/empty,
+// o empty, two MMA drains, q seen
+constexpr int kFixedBars = 2 + 4 + 4 + 6;
 
 struct TcParams {
   DecodeArgs a;
@@ -58,6 +67,8 @@ struct TcParams {
   int NP, NPd;          // 128-feature groups per row, and those holding latent features
   int NQA, NK16;        // 64-feature query atoms, 16-feature K steps
   int PR, RR, raw_slot; // ring slots (f16 groups, packed groups) and packed-group bytes
+  uint32_t lbo_p;       // bytes between the 8-token core-matrix rows of P (16 N2 + 32)
+  uint32_t p_bytes;     // one P buffer: 8 lbo_p
   uint32_t off_p, off_pairs, off_raw, off_bar, off_misc;
   uint32_t idesc1, idesc2;
   int qdtype;           // KVK_BF16 or KVK_F16
@@ -66,13 +77,12 @@ struct TcParams {
 struct Misc {
   uint32_t tmem_base;
   int abort;
-  float smax;
-  float qs_inv[2];
+  float qs_inv[2][64];   // per piece parity and head: 2^-e of the staged query row
   int vote[2][4];
-  float qred[4];
   float m_ref[64];
   float alpha[64];
   float red[4][64];
+  float sred[4];
   int32_t scan_tmp[32];
 };
 
@@ -148,53 +158,66 @@ __device__ __forceinline__ uint32_t spread2(uint32_t x) {  // 4 x 2-bit fields -
   return x;
 }
 
+// Row handled by `lane` in pass k of a convert warp (four lanes per row): rows 8k + rev3(lane/4)
+// put rows that differ in bit 2 (opposite halves of the 128-byte swizzle) in every 8-lane
+// phase and rows 0, 4, 2, 6 in every 16-lane phase, so no access of the convert loops has a
+// shared-memory bank conflict.
+__device__ __forceinline__ int conv_row(int lane, int k) {
+  const int u = lane >> 2;
+  return 8 * k + (((u & 1) << 2) | (u & 2) | ((u >> 2) & 1));
+}
+
+// Packed b-bit group (64 rows x 128 features, TMA-swizzled) -> f16 pair slot, for the 32
+// features 32cw .. 32cw+31 (eight-feature groups g = 4cw .. 4cw+3 of every row).  All eight
+// packed words of a lane are loaded before the first store.
 template <int BITS>
-__device__ __forceinline__ void convert_group(const uint8_t* rawslot, uint8_t* pair, int ct) {
-  if constexpr (BITS == 8) {
-    const __half2 bias = __float2half2_rn(1152.f);
-#pragma unroll 4
-    for (int i = ct; i < 1024; i += 128) {
-      const int r = i >> 4, g = i & 15;
-      const uint2 w = *reinterpret_cast<const uint2*>(rawslot + r * 128 +
-                                                      ((((g >> 1) ^ (r & 7))) << 4) + ((g & 1) << 3));
-      uint4 o;
-      o.x = cvt_small(w.x, 0x4140u, bias);
-      o.y = cvt_small(w.x, 0x4342u, bias);
-      o.z = cvt_small(w.y, 0x4140u, bias);
-      o.w = cvt_small(w.y, 0x4342u, bias);
-      *reinterpret_cast<uint4*>(pair + (g >> 3) * kAtom + r * 128 + (((g & 7) ^ (r & 7)) << 4)) = o;
-    }
-  } else if constexpr (BITS == 4) {
-    const __half2 bias = __float2half2_rn(1032.f);
-#pragma unroll 4
-    for (int i = ct; i < 1024; i += 128) {
-      const int r = i >> 4, g = i & 15;
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(
+__device__ __forceinline__ void convert_group(const uint8_t* rawslot, uint8_t* pair, int lane,
+                                              int cw) {
+  const int g = 4 * cw + (lane & 3);
+  uint32_t w[8][BITS == 8 ? 2 : 1];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = conv_row(lane, k);
+    if constexpr (BITS == 8) {
+      const uint2 u = *reinterpret_cast<const uint2*>(rawslot + r * 128 +
+                                                      (((g >> 1) ^ (r & 7)) << 4) + ((g & 1) << 3));
+      w[k][0] = u.x;
+      w[k][BITS == 8 ? 1 : 0] = u.y;
+    } else if constexpr (BITS == 4) {
+      w[k][0] = *reinterpret_cast<const uint32_t*>(
           rawslot + r * 64 + (((g >> 2) ^ ((r >> 1) & 3)) << 4) + ((g & 3) << 2));
-      const uint32_t x = w & 0x0F0F0F0Fu, y = (w >> 4) & 0x0F0F0F0Fu;
+    } else {   // BITS == 2
+      w[k][0] = *reinterpret_cast<const uint16_t*>(
+          rawslot + r * 32 + (((g >> 3) ^ ((r >> 2) & 1)) << 4) + ((g & 7) << 1));
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = conv_row(lane, k);
+    uint4 o;
+    if constexpr (BITS == 8) {
+      const __half2 bias = __float2half2_rn(1152.f);
+      o.x = cvt_small(w[k][0], 0x4140u, bias);
+      o.y = cvt_small(w[k][0], 0x4342u, bias);
+      o.z = cvt_small(w[k][BITS == 8 ? 1 : 0], 0x4140u, bias);
+      o.w = cvt_small(w[k][BITS == 8 ? 1 : 0], 0x4342u, bias);
+    } else if constexpr (BITS == 4) {
+      const __half2 bias = __float2half2_rn(1032.f);
+      const uint32_t x = w[k][0] & 0x0F0F0F0Fu, y = (w[k][0] >> 4) & 0x0F0F0F0Fu;
       const uint32_t u01 = __byte_perm(x, y, 0x5140u), u45 = __byte_perm(x, y, 0x7362u);
-      uint4 o;
       o.x = cvt_small(u01, 0x4140u, bias);
       o.y = cvt_small(u01, 0x4342u, bias);
       o.z = cvt_small(u45, 0x4140u, bias);
       o.w = cvt_small(u45, 0x4342u, bias);
-      *reinterpret_cast<uint4*>(pair + (g >> 3) * kAtom + r * 128 + (((g & 7) ^ (r & 7)) << 4)) = o;
-    }
-  } else if constexpr (BITS == 2) {
-    const __half2 bias = __float2half2_rn(1026.f);
-#pragma unroll 4
-    for (int i = ct; i < 1024; i += 128) {
-      const int r = i >> 4, g = i & 15;
-      const uint32_t w = *reinterpret_cast<const uint16_t*>(
-          rawslot + r * 32 + (((g >> 3) ^ ((r >> 2) & 1)) << 4) + ((g & 7) << 1));
-      const uint32_t u0 = spread2(w & 0xFFu), u1 = spread2(w >> 8);
-      uint4 o;
+    } else {   // BITS == 2
+      const __half2 bias = __float2half2_rn(1026.f);
+      const uint32_t u0 = spread2(w[k][0] & 0xFFu), u1 = spread2(w[k][0] >> 8);
       o.x = cvt_small(u0, 0x4140u, bias);
       o.y = cvt_small(u0, 0x4342u, bias);
       o.z = cvt_small(u1, 0x4140u, bias);
       o.w = cvt_small(u1, 0x4342u, bias);
-      *reinterpret_cast<uint4*>(pair + (g >> 3) * kAtom + r * 128 + (((g & 7) ^ (r & 7)) << 4)) = o;
     }
+    *reinterpret_cast<uint4*>(pair + (g >> 3) * kAtom + r * 128 + (((g & 7) ^ (r & 7)) << 4)) = o;
   }
 }
 
@@ -230,18 +253,18 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   uint64_t* b_tfull = b_pempty + P.PR;    // [PR] 16-bit: TMA landed in the group slot
   uint64_t* b_rfull = b_tfull + P.PR;     // [RR] packed group landed
   uint64_t* b_rempty = b_rfull + P.RR;    // [RR] packed group consumed
-  uint64_t* b_sfull = b_rempty + P.RR;    // [2] scores ready in TMEM
-  uint64_t* b_sempty = b_sfull + 2;       // [2] scores read
-  uint64_t* b_Pfull = b_sempty + 2;       // [2] P written
+  uint64_t* b_sfull = b_rempty + P.RR;    // scores ready in TMEM
+  uint64_t* b_sempty = b_sfull + 1;       // scores read
+  uint64_t* b_Pfull = b_sempty + 1;       // [2] P written
   uint64_t* b_Pempty = b_Pfull + 2;       // [2] output MMA of that P done
-  uint64_t* b_qfull = b_Pempty + 2;       // query staged
+  uint64_t* b_ctfull = b_Pempty + 2;      // [2] C^T of a tile in TMEM
+  uint64_t* b_ctempty = b_ctfull + 2;     // [2] output MMA of that C^T done
+  uint64_t* b_qfull = b_ctempty + 2;      // query staged
   uint64_t* b_qempty = b_qfull + 1;       // query no longer read
   uint64_t* b_oempty = b_qempty + 1;      // O read out by the epilogue
-  uint64_t* b_final = b_oempty + 1;       // MMA drain
-  uint64_t* b_ssync = b_final + 1;        // softmax group sync
-  uint64_t* b_csync = b_ssync + 1;        // convert group sync
-  uint64_t* b_qseen = b_csync + 1;        // softmax has taken the piece's query scale
-  uint64_t* b_final2 = b_qseen + 1;       // output-MMA drain (last of kFixedBars)
+  uint64_t* b_final = b_oempty + 1;       // score-MMA drain
+  uint64_t* b_final2 = b_final + 1;       // output-MMA drain
+  uint64_t* b_qseen = b_final2 + 1;       // softmax has taken the piece's query scale (last)
   Misc* m = reinterpret_cast<Misc*>(smem + P.off_misc);
   int32_t* off = reinterpret_cast<int32_t*>(m + 1);
   volatile int* abort = &m->abort;
@@ -251,27 +274,27 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   if (tid == 0) {
     for (int i = 0; i < P.PR; ++i) {
       mbar_init(&b_pfull[i], 4);
-      mbar_init(&b_pempty[i], 1);
+      mbar_init(&b_pempty[i], 5);   // score MMAs (commit) + the four convert warps
       mbar_init(&b_tfull[i], 1);
     }
     for (int i = 0; i < P.RR; ++i) {
       mbar_init(&b_rfull[i], 1);
       mbar_init(&b_rempty[i], 4);
     }
+    mbar_init(b_sfull, 1);
+    mbar_init(b_sempty, 4);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&b_sfull[i], 1);
-      mbar_init(&b_sempty[i], 4);
       mbar_init(&b_Pfull[i], 4);
       mbar_init(&b_Pempty[i], 1);
+      mbar_init(&b_ctfull[i], 4);
+      mbar_init(&b_ctempty[i], 1);
     }
     mbar_init(b_qfull, 4);
     mbar_init(b_qempty, 1);
     mbar_init(b_oempty, 4);
     mbar_init(b_final, 1);
-    mbar_init(b_ssync, 128);
-    mbar_init(b_csync, 128);
-    mbar_init(b_qseen, 4);
     mbar_init(b_final2, 1);
+    mbar_init(b_qseen, 4);
     m->abort = 0;
     fence_mbar_init();
   }
@@ -352,8 +375,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     const uint32_t q_atom = (uint32_t)P.N1 * 128u;
     bool ok = true;
     while (g.valid && ok) {
-      const int sb = g.tile & 1;
-      ok = mbar_wait(&b_sempty[sb], ((uint32_t)(g.tile >> 1) & 1u) ^ 1u, abort, kLimitNs);
+      ok = mbar_wait(b_sempty, ((uint32_t)g.tile & 1u) ^ 1u, abort, kLimitNs);
       if (ok && g.first) ok = mbar_wait(b_qfull, (uint32_t)g.piece & 1u, abort, kLimitNs);
       ok = __all_sync(0xffffffffu, ok);
       for (int p = 0; p < P.NP && ok; ++p) {
@@ -368,16 +390,16 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           const uint64_t bd = b0 + ((atom * q_atom) >> 4);
           const int k0 = atom * 4;
           if (k0 + 4 <= P.NK16) {
-            mma4_elect(tmem + 64u * sb, ad, 2u, bd, 2u, P.idesc1, k0 > 0 ? 1u : 0u);
+            mma4_elect(tmem + kSCol, ad, 2u, bd, 2u, P.idesc1, k0 > 0 ? 1u : 0u);
           } else {
             for (int ks = 0; k0 + ks < P.NK16; ++ks)
-              mma1_elect(tmem + 64u * sb, ad + 2u * ks, bd + 2u * ks, P.idesc1, (k0 + ks) > 0);
+              mma1_elect(tmem + kSCol, ad + 2u * ks, bd + 2u * ks, P.idesc1, (k0 + ks) > 0);
           }
         }
-        if (p >= P.NPd) commit_elect(&b_pempty[s]);   // rope-only group: free after scores
+        commit_elect(&b_pempty[s]);   // this group's share of the slot release
       }
       if (!ok) break;
-      commit_elect(&b_sfull[sb]);
+      commit_elect(b_sfull);
       if (g.last) commit_elect(b_qempty);
       pc += P.NP;
       cursor_next(g, off, a.batch, lo, hi);
@@ -389,31 +411,27 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     // ------------------------------------------------------------------ output MMAs
     Cursor g;
     cursor_start(g, seq0, off, a.batch, lo, hi);
-    uint32_t pc = 0;
-    const uint32_t p_bytes = (uint32_t)kTile * P.N2 * 2u;
-    const uint32_t lbo_p = (uint32_t)P.N2 * 16u;
-    const uint64_t a0 = sdesc(smem_u32(pairs), kAtom, 1024u, kLayoutSw128);
+    const uint32_t lbo_p = P.lbo_p;
     const uint64_t b0 = sdesc(smem_u32(p_s), lbo_p, 128u, kLayoutNone);
     bool ok = true;
     while (g.valid && ok) {
       const int sb = g.tile & 1;
       ok = mbar_wait(&b_Pfull[sb], (uint32_t)(g.tile >> 1) & 1u, abort, kLimitNs);
+      if (ok) ok = mbar_wait(&b_ctfull[sb], (uint32_t)(g.tile >> 1) & 1u, abort, kLimitNs);
       if (ok && g.first && g.piece > 0)
         ok = mbar_wait(b_oempty, (uint32_t)(g.piece - 1) & 1u, abort, kLimitNs);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const uint64_t bd = b0 + ((sb * p_bytes) >> 4);
+      const uint64_t bd = b0 + ((sb * P.p_bytes) >> 4);
       for (int p = 0; p < P.NPd; ++p) {
-        const uint32_t s = (pc + p) % P.PR;
-        // K = 64 tokens in four steps of 16: A advances 2048 bytes (two 8-row groups),
-        // B two core-matrix rows of P
-        mma4_elect(tmem + kOCol0 + 64u * p, a0 + ((s * kPair) >> 4), 2048u >> 4, bd,
-                   (2u * lbo_p) >> 4, P.idesc2, g.first ? 0u : 1u);
-        commit_elect(&b_pempty[s]);
+        // K = 64 tokens in four steps of 16: A advances 8 TMEM columns, B two core-matrix
+        // rows of P
+        mma4_ts_elect(tmem + kOCol0 + (uint32_t)P.N2 * p, tmem + kCtCol0 + 128u * sb + 32u * p,
+                      8u, bd, (2u * lbo_p) >> 4, P.idesc2, g.first ? 0u : 1u);
       }
+      commit_elect(&b_ctempty[sb]);
       commit_elect(&b_Pempty[sb]);
-      pc += P.NP;
       cursor_next(g, off, a.batch, lo, hi);
     }
     commit_elect(b_final2);
@@ -460,90 +478,96 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         const uint8_t* qlat = static_cast<const uint8_t*>(a.q_lat) + 2 * ((int64_t)c.seq * a.ql_ss);
         const uint8_t* qrope =
             static_cast<const uint8_t*>(a.q_rope) + 2 * ((int64_t)c.seq * a.qr_ss);
-        auto src = [&](int h, int f0) -> const uint4* {
-          return reinterpret_cast<const uint4*>(
-              (f0 < a.d) ? qlat + 2 * ((int64_t)h * a.ql_sh + f0)
-                         : qrope + 2 * ((int64_t)h * a.qr_sh + (f0 - a.d)));
-        };
-        float mx = 0.f;
-        const int nch = a.H * cpr;
-        for (int base = ct; base < nch; base += 128 * 8) {
-          uint4 v[8];
+        // one pass: warp cw stages heads cw, cw + 4, ..., kQH at a time with every load in
+        // flight; lane l holds chunks l, l + 32, ... of each row, the warp reduces the row's
+        // max |q|, and the row is written scaled by 2^e_h (max |q_h| in [2^14, 2^15), exact
+        // for bf16 inputs in range).  Rows >= H and chunks >= n are zero.
+        for (int h0 = cw; h0 < P.N1; h0 += 4 * kQH) {
+          uint4 v[kQH][kQC];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {   // eight independent loads in flight
-            const int i = base + 128 * k;
-            const int h = i / cpr, f0 = (i - h * cpr) * 8;
-            v[k] = (i < nch && f0 < a.n) ? *src(h, f0) : make_uint4(0u, 0u, 0u, 0u);
+          for (int k = 0; k < kQH; ++k) {
+            const int h = h0 + 4 * k;
+#pragma unroll
+            for (int j = 0; j < kQC; ++j) {
+              const int f0 = 8 * (lane + 32 * j);
+              v[k][j] = make_uint4(0u, 0u, 0u, 0u);
+              if (h < a.H && f0 < a.n)
+                v[k][j] = *reinterpret_cast<const uint4*>(
+                    (f0 < a.d) ? qlat + 2 * ((int64_t)h * a.ql_sh + f0)
+                               : qrope + 2 * ((int64_t)h * a.qr_sh + (f0 - a.d)));
+            }
           }
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            float f[8];
-            load8_bits(v[k], P.qdtype, f);
+          for (int k = 0; k < kQH; ++k) {
+            const int h = h0 + 4 * k;
+            if (h >= P.N1) break;
+            float f[kQC][8];
+            float mx = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
-          }
-        }
+            for (int j = 0; j < kQC; ++j) {
+              load8_bits(v[k][j], P.qdtype, f[j]);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) m->qred[cw] = mx;
-        named_sync(2, 128);
-        mx = fmaxf(fmaxf(m->qred[0], m->qred[1]), fmaxf(m->qred[2], m->qred[3]));
-        const int e = (mx > 0.f && isfinite(mx)) ? 14 - ilogbf(mx) : 0;
-        const float qscale = ldexpf(1.f, e);
-        if (ct == 0) m->qs_inv[c.piece & 1] = ldexpf(1.f, -e);
-        const int nst = P.N1 * cpr;
-        for (int base = ct; base < nst; base += 128 * 8) {
-          uint4 v[8];
+              for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[j][e]));
+            }
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int i = base + 128 * k;
-            const int h = i / cpr, f0 = (i - h * cpr) * 8;
-            v[k] = (i < nst && h < a.H && f0 < a.n) ? *src(h, f0) : make_uint4(0u, 0u, 0u, 0u);
-          }
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const int e = (mx > 0.f && isfinite(mx)) ? 14 - ilogbf(mx) : 0;
+            const float qscale = ldexpf(1.f, e);
+            if (lane == 0) m->qs_inv[c.piece & 1][h] = ldexpf(1.f, -e);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int i = base + 128 * k;
-            if (i >= nst) continue;
-            const int h = i / cpr, fc = i - h * cpr;
-            float f[8];
-            load8_bits(v[k], P.qdtype, f);
-            uint4 o;
-            o.x = h2_bits(__floats2half2_rn(f[0] * qscale, f[1] * qscale));
-            o.y = h2_bits(__floats2half2_rn(f[2] * qscale, f[3] * qscale));
-            o.z = h2_bits(__floats2half2_rn(f[4] * qscale, f[5] * qscale));
-            o.w = h2_bits(__floats2half2_rn(f[6] * qscale, f[7] * qscale));
-            const int at = fc >> 3, j = fc & 7;
-            *reinterpret_cast<uint4*>(q_s + at * (P.N1 * 128) + h * 128 + ((j ^ (h & 7)) << 4)) = o;
+            for (int j = 0; j < kQC; ++j) {
+              const int fc = lane + 32 * j;
+              if (fc >= cpr) break;
+              uint4 o;
+              o.x = h2_bits(__floats2half2_rn(f[j][0] * qscale, f[j][1] * qscale));
+              o.y = h2_bits(__floats2half2_rn(f[j][2] * qscale, f[j][3] * qscale));
+              o.z = h2_bits(__floats2half2_rn(f[j][4] * qscale, f[j][5] * qscale));
+              o.w = h2_bits(__floats2half2_rn(f[j][6] * qscale, f[j][7] * qscale));
+              const int at = fc >> 3, jj = fc & 7;
+              *reinterpret_cast<uint4*>(q_s + at * (P.N1 * 128) + h * 128 + ((jj ^ (h & 7)) << 4)) = o;
+            }
           }
         }
         fence_proxy_async_smem();
-        named_sync(2, 128);   // every warp's rows written (and qred read) before q_full
+        named_sync(2, 128);   // every warp's rows written before q_full
         if (lane == 0) mbar_arrive(b_qfull);
         last_piece = c.piece;
       }
+      const int ctb = c.tile & 1;   // C^T buffer of this tile
       for (int p = 0; p < P.NP; ++p) {
         const uint32_t s = pc % P.PR, ph = (pc / P.PR) & 1u;
         uint8_t* pair = pairs + s * kPair;
+        const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
+        // this warp owns features 32cw .. 32cw+31 of the group: atom cw/2, chunks
+        // 4(cw%2) .. 4(cw%2)+3 of every token row; it converts them and later transposes them
+        const bool owns = (cw >> 1) < nat;
         if constexpr (BITS == 16) {
           fail = fail || !mbar_wait(&b_tfull[s], ph, abort, kLimitNs);
-          const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
-          if (!fail) {
-#pragma unroll 4
-            for (int i = ct; i < nat * 512; i += 128) {   // in place: 16-bit codes -> f16
-              uint4* q4 = reinterpret_cast<uint4*>(pair + i * 16);
-              uint4 v = *q4;
-              v.x = cvt_code16(v.x);
-              v.y = cvt_code16(v.y);
-              v.z = cvt_code16(v.z);
-              v.w = cvt_code16(v.w);
-              *q4 = v;
+          if (!fail && owns) {
+            uint8_t* atom = pair + (cw >> 1) * kAtom;
+            // in place: 16-bit codes -> f16; every load issued before the first store
+            uint4* q4[8];
+            uint4 v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int r = conv_row(lane, k), cc = 4 * (cw & 1) + (lane & 3);
+              q4[k] = reinterpret_cast<uint4*>(atom + r * 128 + ((cc ^ (r & 7)) << 4));
+              v[k] = *q4[k];
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              v[k].x = cvt_code16(v[k].x);
+              v[k].y = cvt_code16(v[k].y);
+              v[k].z = cvt_code16(v[k].z);
+              v[k].w = cvt_code16(v[k].w);
+              *q4[k] = v[k];
             }
           }
         } else {
           const uint32_t rs = rc % P.RR, rph = (rc / P.RR) & 1u;
           fail = fail || !mbar_wait(&b_rfull[rs], rph, abort, kLimitNs);
           fail = fail || !mbar_wait(&b_pempty[s], ph ^ 1u, abort, kLimitNs);
-          if (!fail) convert_group<BITS>(raw + rs * P.raw_slot, pair, ct);
+          if (!fail) convert_group<BITS>(raw + rs * P.raw_slot, pair, lane, cw);
           __syncwarp();
           if (lane == 0) mbar_arrive(&b_rempty[rs]);
           ++rc;
@@ -551,8 +575,43 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&b_pfull[s]);
+        if (p < P.NPd) {
+          // transpose this warp's 32 features x 64 tokens into C^T (TMEM lanes 32cw ..
+          // 32cw+31 of latent group p): per 16 features, four 16-token blocks
+          if (p == 0) {   // the output MMAs of tile - 2 have finished reading this buffer
+            fail = fail || !mbar_wait(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u, abort,
+                                      kLimitNs);
+            tc_fence_after();
+          }
+          if (!fail && owns) {
+            const uint32_t abase = smem_u32(pair + (cw >> 1) * kAtom);
+            const int mi = lane >> 3, r8 = lane & 7;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              uint32_t rr[16];
+              const int cc = 4 * (cw & 1) + 2 * h + (mi >> 1);
+#pragma unroll
+              for (int tg = 0; tg < 4; ++tg) {
+                const int tok = 16 * tg + 8 * (mi & 1) + r8;
+                uint32_t d4[4];
+                ldsm_x4_trans(abase + tok * 128 + ((cc ^ (tok & 7)) << 4), d4);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) rr[4 * tg + i] = d4[i];
+              }
+              tmem_st16x256b_x4(tmem + ((uint32_t)(32 * cw + 16 * h) << 16) + kCtCol0 +
+                                    128u * ctb + 32u * p,
+                                rr);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b_pempty[s]);   // this warp is done reading the slot
         ++pc;
       }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b_ctfull[ctb]);
       cursor_next(c, off, a.batch, lo, hi);
     }
   } else if (has_work) {
@@ -568,53 +627,45 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     const int hc = 2 * (lane & 3);
     bool fail = false;
 
-    // S_max: power of two >= every scale in the CTA's slice (keeps p * s / S_max <= 2^8)
-    float smx = 0.f;
-    {
-      Cursor c;
-      cursor_start(c, seq0, off, a.batch, lo, hi);
-      while (c.valid) {
-        const __half* sp = a.scales + (int64_t)c.seq * a.max_tokens;
-        for (int base = c.p0 + tid; base < c.p1; base += 128 * 8) {
-          __half hv[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int pp = base + 128 * k;
-            hv[k] = pp < c.p1 ? sp[pp] : __float2half(0.f);
-          }
-#pragma unroll
-          for (int k = 0; k < 8; ++k) smx = fmaxf(smx, __half2float(hv[k]));
-        }
-        ++c.seq;
-        c.valid = find_piece(c, off, a.batch, lo, hi);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) smx = fmaxf(smx, __shfl_xor_sync(0xffffffffu, smx, o));
-    if (lane == 0) m->red[q][0] = smx;
-    named_sync(1, 128);
-    smx = fmaxf(fmaxf(m->red[0][0], m->red[1][0]), fmaxf(m->red[2][0], m->red[3][0]));
-    float smax = 1.f;
-    if (smx > 0.f && isfinite(smx)) {
-      int ex;
-      const float fr = frexpf(smx, &ex);             // smx = fr * 2^ex, fr in [0.5, 1)
-      smax = (fr == 0.5f) ? smx : ldexpf(1.f, ex);
-    }
-    const float inv_smax = 1.f / smax;
+    // S_run: running power of two >= every token scale seen so far (P = p * s / S_run keeps
+    // P <= 2^8 in f16).  It only grows; when a tile brings a larger scale the slow path
+    // rescales O by S_old / S_new, exactly (powers of two), together with any max update.
+    float srun = 0.f, inv_srun = 0.f;
 
     float l[2 * NB];    // partial weight sums of this thread's heads
     float mr[2 * NB];   // reference max of this thread's heads (log2 units)
-    float qs_inv = 1.f;
+    float qsi[2 * NB];   // 2^-e_h of this thread's heads for the current piece
     int pt = 0;
     Cursor c;
     cursor_start(c, seq0, off, a.batch, lo, hi);
     const float coef0 = a.sigma * kLog2e;
-    const uint32_t p_bytes = (uint32_t)kTile * P.N2 * 2u;
+    // K slot of this thread's rows in P: the transposed C^T holds, in the 16 K slots of each
+    // step, tokens 0,1,8,9,2,3,10,11,4,5,12,13,6,7,14,15 of the step's 16 tokens
+    const int ka = 16 * q + 4 * (lane >> 3) + ((lane >> 2) & 1), kb = ka + 2;
+    // token scales of rows ra / rb, loaded one tile ahead so the load latency overlaps the
+    // current tile
+    auto load_scales = [&](const Cursor& cc, float& sa, float& sbv) {
+      const __half* sp = a.scales + (int64_t)cc.seq * a.max_tokens + cc.pos;
+      sa = (ra < cc.cnt) ? __half2float(sp[ra]) : 0.f;
+      sbv = (rb < cc.cnt) ? __half2float(sp[rb]) : 0.f;
+    };
+    float s_a_next = 0.f, s_b_next = 0.f;
+    if (c.valid) load_scales(c, s_a_next, s_b_next);
     while (c.valid) {
       const int t = c.tile, sb = t & 1;
+      const float s_a = s_a_next, s_b = s_b_next;
+      {
+        Cursor cn = c;
+        cursor_next(cn, off, a.batch, lo, hi);
+        if (cn.valid) load_scales(cn, s_a_next, s_b_next);
+      }
       if (c.first) {
         fail = fail || !mbar_wait(b_qfull, (uint32_t)c.piece & 1u, abort, kLimitNs);
-        qs_inv = m->qs_inv[c.piece & 1];
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) qsi[2 * j + e] = m->qs_inv[c.piece & 1][8 * j + hc + e];
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(b_qseen);
 #pragma unroll
@@ -625,41 +676,38 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         pt = 0;
       }
       const bool va = ra < c.cnt, vb = rb < c.cnt;
-      const __half* sp = a.scales + (int64_t)c.seq * a.max_tokens + c.pos;
-      const float s_a = va ? __half2float(sp[ra]) : 0.f;
-      const float s_b = vb ? __half2float(sp[rb]) : 0.f;
-      const float ca = coef0 * s_a * qs_inv, cbf = coef0 * s_b * qs_inv;
-      fail = fail || !mbar_wait(&b_sfull[sb], (uint32_t)(t >> 1) & 1u, abort, kLimitNs);
+      const float ca = coef0 * s_a, cbf = coef0 * s_b;
+      fail = fail || !mbar_wait(b_sfull, (uint32_t)t & 1u, abort, kLimitNs);
       tc_fence_after();
       float x[4 * NB];
       if constexpr (NB >= 6) {
         float v[32];
-        tmem_ld16x256b_x8(lb + 64u * sb, v);
+        tmem_ld16x256b_x8(lb + kSCol, v);
 #pragma unroll
         for (int i = 0; i < 4 * NB; ++i) x[i] = v[i];
       } else if constexpr (NB == 4) {
         float v[16];
-        tmem_ld16x256b_x4(lb + 64u * sb, v);
+        tmem_ld16x256b_x4(lb + kSCol, v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) x[i] = v[i];
       } else {
         float v[8];
-        tmem_ld16x256b_x2(lb + 64u * sb, v);
+        tmem_ld16x256b_x2(lb + kSCol, v);
 #pragma unroll
         for (int i = 0; i < 8; ++i) x[i] = v[i];
       }
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&b_sempty[sb]);
-      bool mine = (pt == 0);
+      if (lane == 0) mbar_arrive(b_sempty);
+      bool mine = (pt == 0) || s_a > srun || s_b > srun;
 #pragma unroll
       for (int j = 0; j < NB; ++j) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const bool hv = (8 * j + hc + e) < a.H;
-          x[4 * j + e] = (va && hv) ? x[4 * j + e] * ca : -INFINITY;
-          x[4 * j + 2 + e] = (vb && hv) ? x[4 * j + 2 + e] * cbf : -INFINITY;
+          x[4 * j + e] = (va && hv) ? x[4 * j + e] * qsi[2 * j + e] * ca : -INFINITY;
+          x[4 * j + 2 + e] = (vb && hv) ? x[4 * j + 2 + e] * qsi[2 * j + e] * cbf : -INFINITY;
           mine = mine || (x[4 * j + e] > mr[2 * j + e] + 8.f) ||
                  (x[4 * j + 2 + e] > mr[2 * j + e] + 8.f);
         }
@@ -679,7 +727,25 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
             if (lane < 4) m->red[q][8 * j + 2 * lane + e] = v;
           }
         }
+        {
+          float sm = fmaxf(s_a, s_b);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, o));
+          if (lane == 0) m->sred[q] = sm;
+        }
         named_sync(1, 128);
+        float ratio = 1.f;   // S_old / S_new, applied to O only (l sums p, not p * s)
+        {
+          const float sm = fmaxf(fmaxf(m->sred[0], m->sred[1]), fmaxf(m->sred[2], m->sred[3]));
+          if (sm > srun && isfinite(sm)) {
+            int ex;
+            const float fr = frexpf(sm, &ex);   // sm = fr * 2^ex, fr in [0.5, 1)
+            const float sn = (fr == 0.5f) ? sm : ldexpf(1.f, ex);
+            ratio = srun / sn;
+            srun = sn;
+            inv_srun = 1.f / sn;
+          }
+        }
         if (tid < NH) {   // one thread per head: new reference and the factor for old sums
           const float tm = fmaxf(fmaxf(m->red[0][tid], m->red[1][tid]),
                                  fmaxf(m->red[2][tid], m->red[3][tid]));
@@ -709,11 +775,11 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
 #pragma unroll
             for (int cb = 0; cb < NH; cb += 8) {
               float v[8];
-              const uint32_t ta = lb + kOCol0 + 64u * p + cb;
+              const uint32_t ta = lb + kOCol0 + (uint32_t)P.N2 * p + cb;
               tmem_ld8(ta, v);
               tmem_wait_ld();
 #pragma unroll
-              for (int k = 0; k < 8; ++k) v[k] *= m->alpha[cb + k];
+              for (int k = 0; k < 8; ++k) v[k] *= m->alpha[cb + k] * ratio;
               tmem_st8(ta, v);
             }
           }
@@ -722,14 +788,16 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         }
       }
 
-      // P tile (MN-major core matrices): row r, heads 8j..8j+7 at (r/8)*16*N2 + 128j +
-      // (r%8)*16; this thread's word for heads 8j + hc + {0, 1} of row ra is at
-      // 32 q N2 + 128 j + 4 lane, of row rb 16 N2 further
+      // P tile (MN-major core matrices, no swizzle): K slot k, heads 8j..8j+7 at
+      // (k/8) lbo_p + 128 j + (k%8) 16; this thread's word for heads 8j + hc + {0, 1} is at
+      // + 4 (lane % 4).  lbo_p = 16 N2 + 32 puts the two core rows a warp writes in
+      // disjoint banks.
       fail = fail || !mbar_wait(&b_Pempty[sb], ((uint32_t)(t >> 1) & 1u) ^ 1u, abort, kLimitNs);
       {
-        const float wa = s_a * inv_smax, wb = s_b * inv_smax;
-        uint8_t* pa = p_s + sb * p_bytes + 32 * q * P.N2 + 4 * lane;
-        uint8_t* pbp = pa + 16 * P.N2;
+        const float wa = s_a * inv_srun, wb = s_b * inv_srun;
+        uint8_t* pbuf = p_s + sb * P.p_bytes + 4 * (lane & 3);
+        uint8_t* pa = pbuf + (ka >> 3) * P.lbo_p + (ka & 7) * 16;
+        uint8_t* pbp = pbuf + (kb >> 3) * P.lbo_p + (kb & 7) * 16;
 #pragma unroll
         for (int j = 0; j < NB; ++j) {
           float ea[2], eb[2];
@@ -778,13 +846,13 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
 #pragma unroll
             for (int cb = 0; cb < NH; cb += 8) {
               float v[8];
-              tmem_ld8(lb + kOCol0 + 64u * p + cb, v);
+              tmem_ld8(lb + kOCol0 + (uint32_t)P.N2 * p + cb, v);
               tmem_wait_ld();
               if (f < a.d) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                   const int h = cb + k;
-                  if (h < a.H) a.ws_o[(slot * a.H + h) * a.d + f] = v[k] * smax;
+                  if (h < a.H) a.ws_o[(slot * a.H + h) * a.d + f] = v[k] * srun;
                 }
               }
             }
@@ -831,9 +899,13 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
   P.NPd = (d + 127) / 128;
   P.NQA = (n + 63) / 64;
   P.NK16 = (n + 15) / 16;
-  if (H < 1 || P.N2 > 64 || P.NPd > 6) return pl;
+  // TMEM: S^T (N1 <= 64 columns), two C^T buffers of 4 x 32 columns, O^T NPd x N2 columns
+  if (H < 1 || P.N2 > 64 || P.NPd > 4 || kOCol0 + (uint32_t)(P.NPd * P.N2) > kTmemCols) return pl;
+  if (P.NQA * 8 > 32 * kQC) return pl;   // staged query rows of up to 1024 features
   const size_t q_bytes = (size_t)P.NQA * P.N1 * 128;
-  const size_t p_bytes = 2 * (size_t)kTile * P.N2 * 2;
+  P.lbo_p = (uint32_t)P.N2 * 16u + 32u;
+  P.p_bytes = 8u * P.lbo_p;
+  const size_t p_bytes = 2 * (size_t)P.p_bytes;
   const size_t misc_bytes = sizeof(Misc) + sizeof(int32_t) * (size_t)(batch + 1);
   const int raw_slot = (b == 16) ? 0 : 64 * 16 * b;
   P.raw_slot = raw_slot;
@@ -873,7 +945,7 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
   P.off_misc = (uint32_t)off;
   pl.smem = off + misc_bytes + 1024;
   P.idesc1 = sm100::idesc_f16(64, P.N1, false, false);
-  P.idesc2 = sm100::idesc_f16(128, P.N2, true, true);
+  P.idesc2 = sm100::idesc_f16(128, P.N2, false, true);   // A = C^T from TMEM, B = P MN-major
   pl.ok = pl.smem <= (size_t)kSmemLimit;
   return pl;
 }

@@ -14,45 +14,97 @@ namespace kvk {
 namespace {
 
 constexpr int kMergeThreads = 128;
+constexpr int kChunk = 256;   // pieces whose weights are staged in shared memory at once
 constexpr float kLn2 = 0.6931471805599453f;
 
-__global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
-  const int i = blockIdx.x, h = blockIdx.y;
+template <bool kMax>
+__device__ __forceinline__ float block_reduce(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float u = __shfl_xor_sync(0xffffffffu, v, o);
+    v = kMax ? fmaxf(v, u) : v + u;
+  }
+  const int w = threadIdx.x >> 5;
+  __syncthreads();   // red[] free from any earlier use
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  v = red[0];
+  for (int k = 1; k < kMergeThreads / 32; ++k) v = kMax ? fmaxf(v, red[k]) : v + red[k];
+  return v;
+}
+
+// One CTA per (sequence, head).  The pieces' (m, l) are reduced by the whole block; the
+// outputs are then accumulated four features per thread, the pieces' loads independent of
+// one another (weights staged in shared memory), so the kernel streams the partials instead
+// of waiting on one load per piece.
+__global__ void __launch_bounds__(kMergeThreads, 4) merge_kernel(DecodeArgs a) {
+  __shared__ float w_s[kChunk];
+  __shared__ float red[kMergeThreads / 32];
+  const int i = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
   const int64_t N = a.seq_off[a.batch];
   const int64_t s0 = a.seq_off[i], s1 = a.seq_off[i + 1];
   float* out = a.out + ((int64_t)i * a.H + h) * a.d;
-  float M = -INFINITY;
-  int c0 = 0, c1 = -1;
+  int c0 = 0, np = 0;
   if (s1 > s0) {
     c0 = cta_of(s0, N, a.G);
-    c1 = cta_of(s1 - 1, N, a.G);
-    for (int c = c0; c <= c1; ++c) {
-      const int64_t sh = (int64_t)(c + i) * a.H + h;
-      if (a.ws_ml[2 * sh + 1] > 0.0f) M = fmaxf(M, a.ws_ml[2 * sh]);
-    }
+    np = cta_of(s1 - 1, N, a.G) - c0 + 1;
   }
+  auto ml = [&](int k) -> float2 {   // (m, l) of piece k of this sequence and head
+    const int64_t sh = (int64_t)(c0 + k + i) * a.H + h;
+    return *reinterpret_cast<const float2*>(a.ws_ml + 2 * sh);
+  };
+  float M = -INFINITY;
+  for (int k = tid; k < np; k += kMergeThreads) {
+    const float2 v = ml(k);
+    if (v.y > 0.0f) M = fmaxf(M, v.x);
+  }
+  M = block_reduce<true>(M, red);
   if (M == -INFINITY) {
-    for (int j = threadIdx.x; j < a.d; j += blockDim.x) out[j] = 0.0f;
-    if (a.lse && threadIdx.x == 0) a.lse[(int64_t)i * a.H + h] = -INFINITY;
+    for (int j = tid; j < a.d; j += kMergeThreads) out[j] = 0.0f;
+    if (a.lse && tid == 0) a.lse[(int64_t)i * a.H + h] = -INFINITY;
     return;
   }
-  float lsum = 0.0f;
-  for (int c = c0; c <= c1; ++c) {
-    const int64_t sh = (int64_t)(c + i) * a.H + h;
-    const float l = a.ws_ml[2 * sh + 1];
-    if (l > 0.0f) lsum += exp2f(a.ws_ml[2 * sh] - M) * l;
+  float ls = 0.0f;
+  for (int k = tid; k < np; k += kMergeThreads) {
+    const float2 v = ml(k);
+    if (v.y > 0.0f) ls += exp2f(v.x - M) * v.y;
   }
+  const float lsum = block_reduce<false>(ls, red);
   const float inv = 1.0f / lsum;
-  for (int j = threadIdx.x; j < a.d; j += blockDim.x) {
-    float acc = 0.0f;
-    for (int c = c0; c <= c1; ++c) {
-      const int64_t sh = (int64_t)(c + i) * a.H + h;
-      const float l = a.ws_ml[2 * sh + 1];
-      if (l > 0.0f) acc = fmaf(exp2f(a.ws_ml[2 * sh] - M), a.ws_o[sh * a.d + j], acc);
+  const int d4 = a.d >> 2;   // d is a multiple of 16
+  for (int j0 = 0; j0 < d4; j0 += kMergeThreads) {
+    const int j = j0 + tid;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k0 = 0; k0 < np; k0 += kChunk) {
+      const int nk = min(kChunk, np - k0);
+      __syncthreads();   // previous chunk's weights consumed
+      for (int k = tid; k < nk; k += kMergeThreads) {
+        const float2 v = ml(k0 + k);
+        w_s[k] = (v.y > 0.0f) ? exp2f(v.x - M) : 0.0f;
+      }
+      __syncthreads();
+      if (j < d4) {
+        const float4* src = reinterpret_cast<const float4*>(
+            a.ws_o + ((int64_t)(c0 + k0 + i) * a.H + h) * a.d) + j;
+        const int64_t stride = (int64_t)a.H * d4;   // float4s between consecutive pieces
+#pragma unroll 4
+        for (int k = 0; k < nk; ++k) {
+          const float w = w_s[k];
+          if (w != 0.0f) {
+            const float4 v = src[k * stride];
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+          }
+        }
+      }
     }
-    out[j] = acc * inv;
+    if (j < d4)
+      reinterpret_cast<float4*>(out)[j] =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   }
-  if (a.lse && threadIdx.x == 0) a.lse[(int64_t)i * a.H + h] = kLn2 * (M + log2f(lsum));
+  if (a.lse && tid == 0) a.lse[(int64_t)i * a.H + h] = kLn2 * (M + log2f(lsum));
 }
 
 }  // namespace

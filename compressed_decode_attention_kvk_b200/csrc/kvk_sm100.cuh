@@ -161,6 +161,48 @@ __device__ __forceinline__ void mma1_elect(uint32_t d_tmem, uint64_t a, uint64_t
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
+// Four MMAs with A read from tensor memory: D (+)= A_k * B_k, A_k at column a_tmem + k*a_cols
+// (M = 128 lanes, two 16-bit K elements per 32-bit column), B_k by descriptor.
+__device__ __forceinline__ void mma4_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint32_t a_cols,
+                                              uint64_t b, uint32_t b_step, uint32_t idesc,
+                                              uint32_t acc) {
+  const uint32_t a1 = a_tmem + a_cols, a2 = a_tmem + 2u * a_cols, a3 = a_tmem + 3u * a_cols;
+  const uint64_t b1 = b + b_step, b2 = b + 2u * b_step, b3 = b + 3u * b_step;
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %10, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %9, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %9, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %9, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %9, 1;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(a1), "r"(a2), "r"(a3), "l"(b), "l"(b1), "l"(b2), "l"(b3), "r"(idesc),
+      "r"(acc)
+      : "memory");
+}
+
+// ldmatrix, four 8x8 16-bit matrices, transposed: thread t supplies the row address of row
+// t%8 of matrix t/8 and receives, from matrix i, elements (rows 2(t%4), 2(t%4)+1; column t/4)
+// packed low / high in d[i].
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t saddr, uint32_t (&d)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+               : "r"(saddr)
+               : "memory");
+}
+
+// 16 lanes x 256 bits, repeated 4 times (32 columns): the register layout of
+// tmem_ld16x256b_*, i.e. r[4k], r[4k+1] -> lane base + t/4, columns 8k + 2(t%4) + {0,1};
+// r[4k+2], r[4k+3] -> lane base + 8 + t/4, the same columns.
+__device__ __forceinline__ void tmem_st16x256b_x4(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 // Commit by the same elected lane that issued the MMAs (elect.sync picks the lowest lane).
 __device__ __forceinline__ void commit_elect(uint64_t* bar) {
   asm volatile(
