@@ -86,6 +86,17 @@ struct Misc {
   int32_t scan_tmp[32];
 };
 
+// Position in a ring of n slots: slot index and the phase parity of its mbarriers.
+struct Ring {
+  uint32_t slot = 0, phase = 0;
+  __device__ __forceinline__ void next(int n) {
+    if (++slot == (uint32_t)n) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
 struct Cursor {
   int seq, pos, p0, p1, cnt, tile, piece;
   bool valid, first, last;
@@ -240,8 +251,9 @@ template <int BITS, int NH>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUtensorMap tmap) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base, derived from the shared array by an offset so that every
+  // pointer below stays in the shared state space (plain LDS / STS, not generic accesses)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const DecodeArgs& a = P.a;
   uint8_t* q_s = smem;
   uint8_t* p_s = smem + P.off_p;
@@ -267,7 +279,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   uint64_t* b_qseen = b_final2 + 1;       // softmax has taken the piece's query scale (last)
   Misc* m = reinterpret_cast<Misc*>(smem + P.off_misc);
   int32_t* off = reinterpret_cast<int32_t*>(m + 1);
-  volatile int* abort = &m->abort;
+  const uint32_t abort = smem_u32(&m->abort);   // shared abort word (abort_read / abort_set)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -330,12 +342,13 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       Cursor c;
       cursor_start(c, seq0, off, a.batch, lo, hi);
       uint32_t cnt = 0;
+      Ring rg;
       const int slots = (BITS == 16) ? P.PR : P.RR;
-      while (c.valid && !*abort) {
+      while (c.valid && !abort_read(abort)) {
         const int row0 = c.seq * a.max_tokens + c.pos;
         bool ok = true;
         for (int p = 0; p < P.NP && ok; ++p) {
-          const uint32_t s = cnt % slots, ph = (cnt / slots) & 1u;
+          const uint32_t s = rg.slot, ph = rg.phase;
           if (BITS == 16) {
             if (!(ok = mbar_wait(&b_pempty[s], ph ^ 1u, abort, kLimitNs))) break;
             const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
@@ -349,11 +362,12 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
             tma_load_2d(raw + s * P.raw_slot, &tmap, p * 16 * BITS, row0, &b_rfull[s]);
           }
           ++cnt;
+          rg.next(slots);
         }
         if (!ok) break;
         cursor_next(c, off, a.batch, lo, hi);
       }
-      if (*abort) {  // let the loads already issued land before the block exits
+      if (abort_read(abort)) {  // let the loads already issued land before the block exits
         const uint32_t first = cnt > (uint32_t)slots ? cnt - slots : 0u;
         for (uint32_t k = first; k < cnt; ++k) {
           const uint32_t s = k % slots, ph = (k / slots) & 1u;
@@ -367,7 +381,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     // MMAs in groups of four, and commits them.
     Cursor g;
     cursor_start(g, seq0, off, a.batch, lo, hi);
-    uint32_t pc = 0;
+    Ring rg;
     // descriptors of slot 0 / atom 0; every other operand differs only in its start address
     // (bits 0-13, address >> 4), so each operand adds its byte offset >> 4
     const uint64_t a0 = sdesc(smem_u32(pairs), 16u, 1024u, kLayoutSw128);
@@ -379,8 +393,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       if (ok && g.first) ok = mbar_wait(b_qfull, (uint32_t)g.piece & 1u, abort, kLimitNs);
       ok = __all_sync(0xffffffffu, ok);
       for (int p = 0; p < P.NP && ok; ++p) {
-        const uint32_t u = pc + p, s = u % P.PR;
-        ok = __all_sync(0xffffffffu, mbar_wait(&b_pfull[s], (u / P.PR) & 1u, abort, kLimitNs));
+        const uint32_t s = rg.slot;
+        ok = __all_sync(0xffffffffu, mbar_wait(&b_pfull[s], rg.phase, abort, kLimitNs));
         if (!ok) break;
         tc_fence_after();
         for (int t = 0; t < 2; ++t) {
@@ -397,11 +411,11 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           }
         }
         commit_elect(&b_pempty[s]);   // this group's share of the slot release
+        rg.next(P.PR);
       }
       if (!ok) break;
       commit_elect(b_sfull);
       if (g.last) commit_elect(b_qempty);
-      pc += P.NP;
       cursor_next(g, off, a.batch, lo, hi);
     }
     commit_elect(b_final);          // every MMA issued above has completed after this
@@ -442,7 +456,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     // The four convert warps leave their loop only together (named_or agreement at the top
     // of every tile), so their named barriers never wait for a warp that has gone.
     const int ct = tid - kConvWarp0 * 32, cw = warp - kConvWarp0;
-    uint32_t pc = 0, rc = 0;
+    Ring pr, rr;   // f16 group ring, packed group ring
     int last_piece = -1;
     bool fail = false;
     const int cpr = P.NQA * 8;   // 16-byte chunks per staged query row
@@ -465,7 +479,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     Cursor c;
     cursor_start(c, seq0, off, a.batch, lo, hi);
     while (c.valid) {
-      if (named_or(2, 128, fail || *abort)) break;
+      if (named_or(2, 128, fail || abort_read(abort))) break;
       if (c.piece != last_piece) {
         // Stage this sequence's query as f16 rows [N1][n], scaled by 2^e so that max |q|
         // lands in [2^14, 2^15) (exact for bf16 inputs in range); rows >= H and features
@@ -535,7 +549,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       }
       const int ctb = c.tile & 1;   // C^T buffer of this tile
       for (int p = 0; p < P.NP; ++p) {
-        const uint32_t s = pc % P.PR, ph = (pc / P.PR) & 1u;
+        const uint32_t s = pr.slot, ph = pr.phase;
         uint8_t* pair = pairs + s * kPair;
         const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
         // this warp owns features 32cw .. 32cw+31 of the group: atom cw/2, chunks
@@ -564,13 +578,13 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
             }
           }
         } else {
-          const uint32_t rs = rc % P.RR, rph = (rc / P.RR) & 1u;
+          const uint32_t rs = rr.slot, rph = rr.phase;
           fail = fail || !mbar_wait(&b_rfull[rs], rph, abort, kLimitNs);
           fail = fail || !mbar_wait(&b_pempty[s], ph ^ 1u, abort, kLimitNs);
           if (!fail) convert_group<BITS>(raw + rs * P.raw_slot, pair, lane, cw);
           __syncwarp();
           if (lane == 0) mbar_arrive(&b_rempty[rs]);
-          ++rc;
+          rr.next(P.RR);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -606,7 +620,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&b_pempty[s]);   // this warp is done reading the slot
-        ++pc;
+        pr.next(P.PR);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -714,8 +728,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       }
       // lazy running max: recompute (and rescale) only when a score exceeds the reference
       // by more than 2^8, so P stays within f16 range without touching O every tile
-      if (named_or(1, 128, mine || fail || *abort)) {
-        if (named_or(1, 128, fail || *abort)) break;
+      if (named_or(1, 128, mine || fail || abort_read(abort))) {
+        if (named_or(1, 128, fail || abort_read(abort))) break;
 #pragma unroll
         for (int j = 0; j < NB; ++j) {
 #pragma unroll
@@ -869,7 +883,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
 
   tc_fence_before();
   __syncthreads();
-  if (tid == 0 && *abort) atomicOr(a.flags, KVK_FLAG_TIMEOUT);
+  if (tid == 0 && abort_read(abort)) atomicOr(a.flags, KVK_FLAG_TIMEOUT);
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

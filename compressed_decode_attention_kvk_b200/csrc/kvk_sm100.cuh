@@ -59,17 +59,32 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: returns false (after setting *abort) if the phase did not complete within
-// `limit_ns`, or at once if another thread already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort,
+// Shared-memory abort word (one per CTA), read and written with volatile shared-space
+// accesses so that polling it never leaves the SM.
+__device__ __forceinline__ uint32_t abort_read(uint32_t saddr) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void abort_set(uint32_t saddr) {
+  asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(saddr), "r"(1u) : "memory");
+}
+
+// Bounded wait: returns false (after setting the abort word) if the phase did not complete
+// within limit_ns, or at once (false) if another role has set the abort word.  The loop
+// spins on try_wait (which suspends the thread in hardware for a while) and looks at the
+// abort word and the clock only every 32 tries, so waiting warps take few issue slots.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, uint32_t abort_saddr,
                                           uint64_t limit_ns) {
   if (mbar_try(b, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try(b, parity)) return true;
-    if (*abort) return false;
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try(b, parity)) return true;
+    if (abort_read(abort_saddr)) return false;
     if (globaltimer() - t0 > limit_ns) {
-      *abort = 1;
+      abort_set(abort_saddr);
       return false;
     }
   }
