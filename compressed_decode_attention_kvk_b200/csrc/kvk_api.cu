@@ -177,7 +177,9 @@ kvk_status kvk_create_layout(int n_layers, const int32_t* anchor, const int32_t*
     }
     tmp.slot[l] = (int)tmp.anchors.size() - 1;
   }
-  off = align_up(off, kAlign);
+  // tail slack: the tensor-core decode reads each tile's token scales as a 144-byte window
+  // from the 16-byte boundary at or below the first one, up to 16 bytes past a scale plane
+  off = align_up(off, kAlign) + kAlign;
   if (arena_bytes_needed) *arena_bytes_needed = off;
   if (budget_bits_per_token > 0 && bits > budget_bits_per_token) return KVK_ERR_BUDGET;
   if (!out) return KVK_OK;  // query mode

@@ -8,20 +8,24 @@
 // whole cache).
 //
 // One persistent CTA per SM walks a balanced slice of the flattened token space in tiles of
-// 64 tokens.  Warp roles (352 threads):
+// 64 tokens.  Warp roles (512 threads, four warpgroups with their own register budgets):
 //   warps 0-3  softmax: read S from TMEM, per-token scale, lazy online softmax, write P
 //              (f16) to shared memory, rescale O in TMEM when a max grows, write partials
-//   warps 4-7  convert: packed b-bit codes -> f16 operand tiles (UMMA 128-byte-swizzled,
-//              K-major) and their transpose into TMEM; staged query (power-of-two scaled)
-//   warp 8     TMA producer: 128-feature groups of 64 packed rows into a ring
-//   warp 9     score-MMA issuer (one thread) and TMEM owner
-//   warp 10    output-MMA issuer (one thread)
+//   warps 4-11 convert: packed b-bit codes -> f16 operand tiles (UMMA 128-byte-swizzled,
+//              K-major) and their transpose into TMEM; staged query (power-of-two scaled).
+//              Two warps per SM sub-partition, 16 features of every 128-feature group each.
+//   warp 12    TMA producer: 128-feature groups of 64 packed rows into a ring
+//   warp 13    score-MMA issuer (one thread) and TMEM owner
+//   warp 14    output-MMA issuer (one thread); warp 15 idle
+// Launched with 128 registers per thread; the softmax warpgroup raises its budget to
+// kRegsSoftmax, the conversion warpgroups lower theirs to kRegsConvert and the last
+// warpgroup to kRegsIssue (4 x 32 x (192 + 2 x 120 + 56) = 62464 <= 65536).
 // Per tile:  S^T[64 tok x N1 heads]  = C[64 x n] . Q^T         (M=64, A in smem, TMEM f32)
 //            O^T[128 feat x N2 heads] += C^T[128 x 64] . P    (M=128 per 128 latent features,
 //                                                               A = C^T in TMEM)
 // Heads sit on N, so 40 heads cost N = 40 / 48, never M = 128.  After the convert warps have
 // turned a 128-feature group into f16 (UMMA 128-byte swizzled, K-major: the score MMA's A),
-// each of them transposes its 32 features of it into TMEM (ldmatrix.trans -> tcgen05.st),
+// each of them transposes its 16 features of it into TMEM (ldmatrix.trans -> tcgen05.st),
 // so a ring slot is free as soon as the score MMA has read it; the output MMA reads TMEM.
 // The transpose fragment orders the 16 tokens of each K step as 0,1,8,9,2,3,10,11,4,5,12,13,
 // 6,7,14,15; the softmax warps write P's K rows in that same order.
@@ -40,11 +44,15 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 352;
+constexpr int kThreads = 512;   // 16 warps = 4 warpgroups (warp 15 has no role)
 constexpr int kConvWarp0 = 4;
-constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;    // score MMAs; owns TMEM
-constexpr int kMma2Warp = 10;  // output MMAs
+constexpr int kConvWarps = 8;
+constexpr int kConvThreads = 32 * kConvWarps;
+constexpr int kTmaWarp = 12;
+constexpr int kMmaWarp = 13;   // score MMAs; owns TMEM
+constexpr int kMma2Warp = 14;  // output MMAs
+constexpr uint32_t kRegsSoftmax = 192, kRegsConvert = 120, kRegsIssue = 56;
+static_assert(128 * (kRegsSoftmax + 2 * kRegsConvert + kRegsIssue) <= 65536, "register split");
 constexpr int kTile = kTcTileTokens;   // 64
 constexpr int kAtom = 8192;            // 64 rows x 128 bytes (64 f16 features)
 constexpr int kPair = 2 * kAtom;       // 128 features
@@ -55,11 +63,15 @@ constexpr uint32_t kOCol0 = 320;       // O^T group p at 320 + N2 p
 constexpr uint64_t kLimitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kSmemLimit = 232448;
-constexpr int kQH = 5;   // query rows a convert warp loads per round
-constexpr int kQC = 4;   // 16-byte chunks per lane per query row (rows of up to 1024 features)
+constexpr int kQH = 6;   // query rows a convert warp loads per round (one round for 48 heads)
+constexpr int kQC = 3;   // 16-byte chunks per lane per query row (rows of up to 768 features)
+// Token-scale ring: per tile a 144-byte window (the tile's 64 fp16 scales from the 16-byte
+// boundary at or below the first), loaded by the TMA warp with a plain bulk copy.
+constexpr int kScSlots = 4;
+constexpr uint32_t kScBytes = 144;
 // barriers besides the rings: s full/empty, P full/empty (2), C^T full/empty (2), q full/empty,
-// o empty, two MMA drains, q seen
-constexpr int kFixedBars = 2 + 4 + 4 + 6;
+// o empty, two MMA drains, q seen, scale full/empty (kScSlots each)
+constexpr int kFixedBars = 2 + 4 + 4 + 6 + 2 * kScSlots;
 
 struct TcParams {
   DecodeArgs a;
@@ -75,6 +87,7 @@ struct TcParams {
 };
 
 struct Misc {
+  alignas(16) uint8_t sc[kScSlots][kScBytes];   // token-scale windows
   uint32_t tmem_base;
   int abort;
   float qs_inv[2][64];   // per piece parity and head: 2^-e of the staged query row
@@ -169,25 +182,26 @@ __device__ __forceinline__ uint32_t spread2(uint32_t x) {  // 4 x 2-bit fields -
   return x;
 }
 
-// Row handled by `lane` in pass k of a convert warp (four lanes per row): rows 8k + rev3(lane/4)
-// put rows that differ in bit 2 (opposite halves of the 128-byte swizzle) in every 8-lane
-// phase and rows 0, 4, 2, 6 in every 16-lane phase, so no access of the convert loops has a
-// shared-memory bank conflict.
+// Row handled by `lane` in pass k of a convert warp (two lanes per row, one 16-byte chunk
+// each): rows 16k + 8(u/8) + (0,2,4,6,1,3,5,7)[u%8], u = lane/2.  Every 8-lane phase then
+// touches rows that differ in bits 1 and 2 (distinct chunks of the 128-byte swizzle) and
+// every 16-lane phase eight rows with distinct (row % 8), so the convert loops are free of
+// shared-memory bank conflicts for 16- and 8-byte accesses.
 __device__ __forceinline__ int conv_row(int lane, int k) {
-  const int u = lane >> 2;
-  return 8 * k + (((u & 1) << 2) | (u & 2) | ((u >> 2) & 1));
+  const int u = lane >> 1, x = u & 7;
+  return 16 * k + 8 * (u >> 3) + (((x & 3) << 1) | (x >> 2));
 }
 
-// Packed b-bit group (64 rows x 128 features, TMA-swizzled) -> f16 pair slot, for the 32
-// features 32cw .. 32cw+31 (eight-feature groups g = 4cw .. 4cw+3 of every row).  All eight
+// Packed b-bit group (64 rows x 128 features, TMA-swizzled) -> f16 pair slot, for the 16
+// features fb .. fb+15 (eight-feature groups g = fb/8 + {0, 1} of every row).  All four
 // packed words of a lane are loaded before the first store.
 template <int BITS>
 __device__ __forceinline__ void convert_group(const uint8_t* rawslot, uint8_t* pair, int lane,
-                                              int cw) {
-  const int g = 4 * cw + (lane & 3);
-  uint32_t w[8][BITS == 8 ? 2 : 1];
+                                              int fb) {
+  const int g = (fb >> 3) + (lane & 1);
+  uint32_t w[4][BITS == 8 ? 2 : 1];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
+  for (int k = 0; k < 4; ++k) {
     const int r = conv_row(lane, k);
     if constexpr (BITS == 8) {
       const uint2 u = *reinterpret_cast<const uint2*>(rawslot + r * 128 +
@@ -203,7 +217,7 @@ __device__ __forceinline__ void convert_group(const uint8_t* rawslot, uint8_t* p
     }
   }
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
+  for (int k = 0; k < 4; ++k) {
     const int r = conv_row(lane, k);
     uint4 o;
     if constexpr (BITS == 8) {
@@ -276,7 +290,9 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   uint64_t* b_oempty = b_qempty + 1;      // O read out by the epilogue
   uint64_t* b_final = b_oempty + 1;       // score-MMA drain
   uint64_t* b_final2 = b_final + 1;       // output-MMA drain
-  uint64_t* b_qseen = b_final2 + 1;       // softmax has taken the piece's query scale (last)
+  uint64_t* b_qseen = b_final2 + 1;       // softmax has taken the piece's query scale
+  uint64_t* b_scfull = b_qseen + 1;       // [kScSlots] scale window landed
+  uint64_t* b_scempty = b_scfull + kScSlots;   // [kScSlots] scale window read (last)
   Misc* m = reinterpret_cast<Misc*>(smem + P.off_misc);
   int32_t* off = reinterpret_cast<int32_t*>(m + 1);
   const uint32_t abort = smem_u32(&m->abort);   // shared abort word (abort_read / abort_set)
@@ -285,28 +301,32 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
 
   if (tid == 0) {
     for (int i = 0; i < P.PR; ++i) {
-      mbar_init(&b_pfull[i], 4);
-      mbar_init(&b_pempty[i], 5);   // score MMAs (commit) + the four convert warps
+      mbar_init(&b_pfull[i], kConvWarps);
+      mbar_init(&b_pempty[i], 1 + kConvWarps);   // score MMAs (commit) + the convert warps
       mbar_init(&b_tfull[i], 1);
     }
     for (int i = 0; i < P.RR; ++i) {
       mbar_init(&b_rfull[i], 1);
-      mbar_init(&b_rempty[i], 4);
+      mbar_init(&b_rempty[i], kConvWarps);
     }
     mbar_init(b_sfull, 1);
     mbar_init(b_sempty, 4);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b_Pfull[i], 4);
       mbar_init(&b_Pempty[i], 1);
-      mbar_init(&b_ctfull[i], 4);
+      mbar_init(&b_ctfull[i], kConvWarps);
       mbar_init(&b_ctempty[i], 1);
     }
-    mbar_init(b_qfull, 4);
+    mbar_init(b_qfull, kConvWarps);
     mbar_init(b_qempty, 1);
     mbar_init(b_oempty, 4);
     mbar_init(b_final, 1);
     mbar_init(b_final2, 1);
     mbar_init(b_qseen, 4);
+    for (int i = 0; i < kScSlots; ++i) {
+      mbar_init(&b_scfull[i], 1);
+      mbar_init(&b_scempty[i], 4);
+    }
     m->abort = 0;
     fence_mbar_init();
   }
@@ -336,126 +356,151 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   }
   const bool has_work = lo < hi;
 
-  if (has_work && warp == kTmaWarp) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      Cursor c;
-      cursor_start(c, seq0, off, a.batch, lo, hi);
-      uint32_t cnt = 0;
-      Ring rg;
-      const int slots = (BITS == 16) ? P.PR : P.RR;
-      while (c.valid && !abort_read(abort)) {
-        const int row0 = c.seq * a.max_tokens + c.pos;
-        bool ok = true;
-        for (int p = 0; p < P.NP && ok; ++p) {
-          const uint32_t s = rg.slot, ph = rg.phase;
-          if (BITS == 16) {
-            if (!(ok = mbar_wait(&b_pempty[s], ph ^ 1u, abort, kLimitNs))) break;
-            const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
-            mbar_arrive_expect_tx(&b_tfull[s], nat * kAtom);
-            for (int t = 0; t < nat; ++t)
-              tma_load_2d(pairs + s * kPair + t * kAtom, &tmap, (2 * p + t) * 128, row0,
-                          &b_tfull[s]);
-          } else {
-            if (!(ok = mbar_wait(&b_rempty[s], ph ^ 1u, abort, kLimitNs))) break;
-            mbar_arrive_expect_tx(&b_rfull[s], P.raw_slot);
-            tma_load_2d(raw + s * P.raw_slot, &tmap, p * 16 * BITS, row0, &b_rfull[s]);
+  // Roles by warpgroup; each warpgroup first sets its register budget (one call site per
+  // warpgroup, executed by all four of its warps).
+  if (has_work && warp >= kTmaWarp) {
+    regs_dec<kRegsIssue>();
+    if (warp == kTmaWarp) {
+      // ------------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        Cursor c;
+        cursor_start(c, seq0, off, a.batch, lo, hi);
+        uint32_t cnt = 0;
+        Ring rg;
+        const int slots = (BITS == 16) ? P.PR : P.RR;
+        // hold the first cache loads until the first query is staged: its loads then do not
+        // queue behind every CTA's ring fill
+        mbar_wait(b_qfull, 0u, abort, kLimitNs);
+        Ring sr;   // scale ring
+        uint32_t nsc = 0;
+        while (c.valid && !abort_read(abort)) {
+          const int row0 = c.seq * a.max_tokens + c.pos;
+          bool ok = true;
+          {   // this tile's scale window (the arena has tail slack for the last one)
+            const uintptr_t sp = reinterpret_cast<uintptr_t>(a.scales + row0);
+            if (!(ok = mbar_wait(&b_scempty[sr.slot], sr.phase ^ 1u, abort, kLimitNs))) break;
+            mbar_arrive_expect_tx(&b_scfull[sr.slot], kScBytes);
+            bulk_load(m->sc[sr.slot], reinterpret_cast<const void*>(sp & ~uintptr_t(15)),
+                      kScBytes, &b_scfull[sr.slot]);
+            sr.next(kScSlots);
+            ++nsc;
           }
-          ++cnt;
-          rg.next(slots);
+          for (int p = 0; p < P.NP && ok; ++p) {
+            const uint32_t s = rg.slot, ph = rg.phase;
+            if (BITS == 16) {
+              if (!(ok = mbar_wait(&b_pempty[s], ph ^ 1u, abort, kLimitNs))) break;
+              const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
+              mbar_arrive_expect_tx(&b_tfull[s], nat * kAtom);
+              for (int t = 0; t < nat; ++t)
+                tma_load_2d(pairs + s * kPair + t * kAtom, &tmap, (2 * p + t) * 128, row0,
+                            &b_tfull[s]);
+            } else {
+              if (!(ok = mbar_wait(&b_rempty[s], ph ^ 1u, abort, kLimitNs))) break;
+              mbar_arrive_expect_tx(&b_rfull[s], P.raw_slot);
+              tma_load_2d(raw + s * P.raw_slot, &tmap, p * 16 * BITS, row0, &b_rfull[s]);
+            }
+            ++cnt;
+            rg.next(slots);
+          }
+          if (!ok) break;
+          cursor_next(c, off, a.batch, lo, hi);
+        }
+        if (abort_read(abort)) {  // let the loads already issued land before the block exits
+          for (uint32_t k = nsc > (uint32_t)kScSlots ? nsc - kScSlots : 0u; k < nsc; ++k)
+            wait_noabort(&b_scfull[k % kScSlots], (k / kScSlots) & 1u);
+          const uint32_t first = cnt > (uint32_t)slots ? cnt - slots : 0u;
+          for (uint32_t k = first; k < cnt; ++k) {
+            const uint32_t s = k % slots, ph = (k / slots) & 1u;
+            wait_noabort(BITS == 16 ? &b_tfull[s] : &b_rfull[s], ph);
+          }
+        }
+      }
+    } else if (warp == kMmaWarp) {
+      // ------------------------------------------------------------------ score MMAs
+      // The whole warp runs the schedule (warp-uniform waits); one elected lane issues the
+      // MMAs in groups of four, and commits them.
+      Cursor g;
+      cursor_start(g, seq0, off, a.batch, lo, hi);
+      Ring rg;
+      // descriptors of slot 0 / atom 0; every other operand differs only in its start address
+      // (bits 0-13, address >> 4), so each operand adds its byte offset >> 4
+      const uint64_t a0 = sdesc(smem_u32(pairs), 16u, 1024u, kLayoutSw128);
+      const uint64_t b0 = sdesc(smem_u32(q_s), 16u, 1024u, kLayoutSw128);
+      const uint32_t q_atom = (uint32_t)P.N1 * 128u;
+      bool ok = true;
+      while (g.valid && ok) {
+        ok = mbar_wait(b_sempty, ((uint32_t)g.tile & 1u) ^ 1u, abort, kLimitNs);
+        if (ok && g.first) ok = mbar_wait(b_qfull, (uint32_t)g.piece & 1u, abort, kLimitNs);
+        ok = __all_sync(0xffffffffu, ok);
+        for (int p = 0; p < P.NP && ok; ++p) {
+          const uint32_t s = rg.slot;
+          ok = __all_sync(0xffffffffu, mbar_wait(&b_pfull[s], rg.phase, abort, kLimitNs));
+          if (!ok) break;
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t) {
+            const int atom = 2 * p + t;
+            if (atom * 64 >= a.n) break;
+            const uint64_t ad = a0 + ((s * kPair + t * kAtom) >> 4);
+            const uint64_t bd = b0 + ((atom * q_atom) >> 4);
+            const int k0 = atom * 4;
+            if (k0 + 4 <= P.NK16) {
+              mma4_elect(tmem + kSCol, ad, 2u, bd, 2u, P.idesc1, k0 > 0 ? 1u : 0u);
+            } else {
+              for (int ks = 0; k0 + ks < P.NK16; ++ks)
+                mma1_elect(tmem + kSCol, ad + 2u * ks, bd + 2u * ks, P.idesc1, (k0 + ks) > 0);
+            }
+          }
+          commit_elect(&b_pempty[s]);   // this group's share of the slot release
+          rg.next(P.PR);
         }
         if (!ok) break;
-        cursor_next(c, off, a.batch, lo, hi);
+        commit_elect(b_sfull);
+        if (g.last) commit_elect(b_qempty);
+        cursor_next(g, off, a.batch, lo, hi);
       }
-      if (abort_read(abort)) {  // let the loads already issued land before the block exits
-        const uint32_t first = cnt > (uint32_t)slots ? cnt - slots : 0u;
-        for (uint32_t k = first; k < cnt; ++k) {
-          const uint32_t s = k % slots, ph = (k / slots) & 1u;
-          wait_noabort(BITS == 16 ? &b_tfull[s] : &b_rfull[s], ph);
-        }
-      }
-    }
-  } else if (has_work && warp == kMmaWarp) {
-    // ------------------------------------------------------------------ score MMAs
-    // The whole warp runs the schedule (warp-uniform waits); one elected lane issues the
-    // MMAs in groups of four, and commits them.
-    Cursor g;
-    cursor_start(g, seq0, off, a.batch, lo, hi);
-    Ring rg;
-    // descriptors of slot 0 / atom 0; every other operand differs only in its start address
-    // (bits 0-13, address >> 4), so each operand adds its byte offset >> 4
-    const uint64_t a0 = sdesc(smem_u32(pairs), 16u, 1024u, kLayoutSw128);
-    const uint64_t b0 = sdesc(smem_u32(q_s), 16u, 1024u, kLayoutSw128);
-    const uint32_t q_atom = (uint32_t)P.N1 * 128u;
-    bool ok = true;
-    while (g.valid && ok) {
-      ok = mbar_wait(b_sempty, ((uint32_t)g.tile & 1u) ^ 1u, abort, kLimitNs);
-      if (ok && g.first) ok = mbar_wait(b_qfull, (uint32_t)g.piece & 1u, abort, kLimitNs);
-      ok = __all_sync(0xffffffffu, ok);
-      for (int p = 0; p < P.NP && ok; ++p) {
-        const uint32_t s = rg.slot;
-        ok = __all_sync(0xffffffffu, mbar_wait(&b_pfull[s], rg.phase, abort, kLimitNs));
+      commit_elect(b_final);          // every MMA issued above has completed after this
+      if (lane == 0) wait_noabort(b_final, 0);
+      __syncwarp();
+    } else if (warp == kMma2Warp) {
+      // ------------------------------------------------------------------ output MMAs
+      Cursor g;
+      cursor_start(g, seq0, off, a.batch, lo, hi);
+      const uint32_t lbo_p = P.lbo_p;
+      const uint64_t b0 = sdesc(smem_u32(p_s), lbo_p, 128u, kLayoutNone);
+      bool ok = true;
+      while (g.valid && ok) {
+        const int sb = g.tile & 1;
+        ok = mbar_wait(&b_Pfull[sb], (uint32_t)(g.tile >> 1) & 1u, abort, kLimitNs);
+        if (ok) ok = mbar_wait(&b_ctfull[sb], (uint32_t)(g.tile >> 1) & 1u, abort, kLimitNs);
+        if (ok && g.first && g.piece > 0)
+          ok = mbar_wait(b_oempty, (uint32_t)(g.piece - 1) & 1u, abort, kLimitNs);
+        ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        for (int t = 0; t < 2; ++t) {
-          const int atom = 2 * p + t;
-          if (atom * 64 >= a.n) break;
-          const uint64_t ad = a0 + ((s * kPair + t * kAtom) >> 4);
-          const uint64_t bd = b0 + ((atom * q_atom) >> 4);
-          const int k0 = atom * 4;
-          if (k0 + 4 <= P.NK16) {
-            mma4_elect(tmem + kSCol, ad, 2u, bd, 2u, P.idesc1, k0 > 0 ? 1u : 0u);
-          } else {
-            for (int ks = 0; k0 + ks < P.NK16; ++ks)
-              mma1_elect(tmem + kSCol, ad + 2u * ks, bd + 2u * ks, P.idesc1, (k0 + ks) > 0);
-          }
+        const uint64_t bd = b0 + ((sb * P.p_bytes) >> 4);
+        for (int p = 0; p < P.NPd; ++p) {
+          // K = 64 tokens in four steps of 16: A advances 8 TMEM columns, B two core-matrix
+          // rows of P
+          mma4_ts_elect(tmem + kOCol0 + (uint32_t)P.N2 * p, tmem + kCtCol0 + 128u * sb + 32u * p,
+                        8u, bd, (2u * lbo_p) >> 4, P.idesc2, g.first ? 0u : 1u);
         }
-        commit_elect(&b_pempty[s]);   // this group's share of the slot release
-        rg.next(P.PR);
+        commit_elect(&b_ctempty[sb]);
+        commit_elect(&b_Pempty[sb]);
+        cursor_next(g, off, a.batch, lo, hi);
       }
-      if (!ok) break;
-      commit_elect(b_sfull);
-      if (g.last) commit_elect(b_qempty);
-      cursor_next(g, off, a.batch, lo, hi);
+      commit_elect(b_final2);
+      if (lane == 0) wait_noabort(b_final2, 0);
+      __syncwarp();
     }
-    commit_elect(b_final);          // every MMA issued above has completed after this
-    if (lane == 0) wait_noabort(b_final, 0);
-    __syncwarp();
-  } else if (has_work && warp == kMma2Warp) {
-    // ------------------------------------------------------------------ output MMAs
-    Cursor g;
-    cursor_start(g, seq0, off, a.batch, lo, hi);
-    const uint32_t lbo_p = P.lbo_p;
-    const uint64_t b0 = sdesc(smem_u32(p_s), lbo_p, 128u, kLayoutNone);
-    bool ok = true;
-    while (g.valid && ok) {
-      const int sb = g.tile & 1;
-      ok = mbar_wait(&b_Pfull[sb], (uint32_t)(g.tile >> 1) & 1u, abort, kLimitNs);
-      if (ok) ok = mbar_wait(&b_ctfull[sb], (uint32_t)(g.tile >> 1) & 1u, abort, kLimitNs);
-      if (ok && g.first && g.piece > 0)
-        ok = mbar_wait(b_oempty, (uint32_t)(g.piece - 1) & 1u, abort, kLimitNs);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      const uint64_t bd = b0 + ((sb * P.p_bytes) >> 4);
-      for (int p = 0; p < P.NPd; ++p) {
-        // K = 64 tokens in four steps of 16: A advances 8 TMEM columns, B two core-matrix
-        // rows of P
-        mma4_ts_elect(tmem + kOCol0 + (uint32_t)P.N2 * p, tmem + kCtCol0 + 128u * sb + 32u * p,
-                      8u, bd, (2u * lbo_p) >> 4, P.idesc2, g.first ? 0u : 1u);
-      }
-      commit_elect(&b_ctempty[sb]);
-      commit_elect(&b_Pempty[sb]);
-      cursor_next(g, off, a.batch, lo, hi);
-    }
-    commit_elect(b_final2);
-    if (lane == 0) wait_noabort(b_final2, 0);
-    __syncwarp();
   } else if (has_work && warp >= kConvWarp0) {
+    regs_dec<kRegsConvert>();
     // ------------------------------------------------------------------ convert
-    // The four convert warps leave their loop only together (named_or agreement at the top
-    // of every tile), so their named barriers never wait for a warp that has gone.
+    // The convert warps leave their loop only together (named_or agreement at the top of
+    // every tile), so their named barriers never wait for a warp that has gone.  Warp cw
+    // sits in TMEM lane quarter cq = cw % 4 and owns features fb .. fb+15 of every group,
+    // fb = 32 cq + 16 ch (ch = cw / 4): TMEM lanes fb .. fb+15 of C^T.
     const int ct = tid - kConvWarp0 * 32, cw = warp - kConvWarp0;
+    const int cq = cw & 3, ch = cw >> 2, fb = 32 * cq + 16 * ch;
     Ring pr, rr;   // f16 group ring, packed group ring
     int last_piece = -1;
     bool fail = false;
@@ -467,7 +512,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         const uint8_t* ql = static_cast<const uint8_t*>(a.q_lat) + 2 * ((int64_t)c.seq * a.ql_ss);
         const uint8_t* qr = static_cast<const uint8_t*>(a.q_rope) + 2 * ((int64_t)c.seq * a.qr_ss);
         const int lat_lines = (2 * a.d + 127) / 128, rope_lines = (2 * a.d_rope + 127) / 128;
-        for (int i = ct; i < a.H * (lat_lines + rope_lines); i += 128) {
+        for (int i = ct; i < a.H * (lat_lines + rope_lines); i += kConvThreads) {
           const int h = i / (lat_lines + rope_lines), k = i - h * (lat_lines + rope_lines);
           if (k < lat_lines) prefetch_l2(ql + 2 * ((int64_t)h * a.ql_sh) + 128 * k);
           else prefetch_l2(qr + 2 * ((int64_t)h * a.qr_sh) + 128 * (k - lat_lines));
@@ -479,7 +524,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     Cursor c;
     cursor_start(c, seq0, off, a.batch, lo, hi);
     while (c.valid) {
-      if (named_or(2, 128, fail || abort_read(abort))) break;
+      if (named_or(2, kConvThreads, fail || abort_read(abort))) break;
       if (c.piece != last_piece) {
         // Stage this sequence's query as f16 rows [N1][n], scaled by 2^e so that max |q|
         // lands in [2^14, 2^15) (exact for bf16 inputs in range); rows >= H and features
@@ -492,15 +537,15 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         const uint8_t* qlat = static_cast<const uint8_t*>(a.q_lat) + 2 * ((int64_t)c.seq * a.ql_ss);
         const uint8_t* qrope =
             static_cast<const uint8_t*>(a.q_rope) + 2 * ((int64_t)c.seq * a.qr_ss);
-        // one pass: warp cw stages heads cw, cw + 4, ..., kQH at a time with every load in
+        // one pass: warp cw stages heads cw, cw + 8, ..., kQH at a time with every load in
         // flight; lane l holds chunks l, l + 32, ... of each row, the warp reduces the row's
         // max |q|, and the row is written scaled by 2^e_h (max |q_h| in [2^14, 2^15), exact
         // for bf16 inputs in range).  Rows >= H and chunks >= n are zero.
-        for (int h0 = cw; h0 < P.N1; h0 += 4 * kQH) {
+        for (int h0 = cw; h0 < P.N1; h0 += kConvWarps * kQH) {
           uint4 v[kQH][kQC];
 #pragma unroll
           for (int k = 0; k < kQH; ++k) {
-            const int h = h0 + 4 * k;
+            const int h = h0 + kConvWarps * k;
 #pragma unroll
             for (int j = 0; j < kQC; ++j) {
               const int f0 = 8 * (lane + 32 * j);
@@ -513,7 +558,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           }
 #pragma unroll
           for (int k = 0; k < kQH; ++k) {
-            const int h = h0 + 4 * k;
+            const int h = h0 + kConvWarps * k;
             if (h >= P.N1) break;
             float f[kQC][8];
             float mx = 0.f;
@@ -543,7 +588,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           }
         }
         fence_proxy_async_smem();
-        named_sync(2, 128);   // every warp's rows written before q_full
+        named_sync(2, kConvThreads);   // every warp's rows written before q_full
         if (lane == 0) mbar_arrive(b_qfull);
         last_piece = c.piece;
       }
@@ -552,24 +597,24 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         const uint32_t s = pr.slot, ph = pr.phase;
         uint8_t* pair = pairs + s * kPair;
         const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
-        // this warp owns features 32cw .. 32cw+31 of the group: atom cw/2, chunks
-        // 4(cw%2) .. 4(cw%2)+3 of every token row; it converts them and later transposes them
-        const bool owns = (cw >> 1) < nat;
+        // this warp owns features fb .. fb+15 of the group: atom cq/2, chunks
+        // 4(cq%2) + 2ch + {0, 1} of every token row; it converts them and later transposes them
+        const bool owns = (cq >> 1) < nat;
         if constexpr (BITS == 16) {
           fail = fail || !mbar_wait(&b_tfull[s], ph, abort, kLimitNs);
           if (!fail && owns) {
-            uint8_t* atom = pair + (cw >> 1) * kAtom;
+            uint8_t* atom = pair + (cq >> 1) * kAtom;
             // in place: 16-bit codes -> f16; every load issued before the first store
-            uint4* q4[8];
-            uint4 v[8];
+            uint4* q4[4];
+            uint4 v[4];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int r = conv_row(lane, k), cc = 4 * (cw & 1) + (lane & 3);
+            for (int k = 0; k < 4; ++k) {
+              const int r = conv_row(lane, k), cc = 4 * (cq & 1) + 2 * ch + (lane & 1);
               q4[k] = reinterpret_cast<uint4*>(atom + r * 128 + ((cc ^ (r & 7)) << 4));
               v[k] = *q4[k];
             }
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < 4; ++k) {
               v[k].x = cvt_code16(v[k].x);
               v[k].y = cvt_code16(v[k].y);
               v[k].z = cvt_code16(v[k].z);
@@ -581,7 +626,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           const uint32_t rs = rr.slot, rph = rr.phase;
           fail = fail || !mbar_wait(&b_rfull[rs], rph, abort, kLimitNs);
           fail = fail || !mbar_wait(&b_pempty[s], ph ^ 1u, abort, kLimitNs);
-          if (!fail) convert_group<BITS>(raw + rs * P.raw_slot, pair, lane, cw);
+          if (!fail) convert_group<BITS>(raw + rs * P.raw_slot, pair, lane, fb);
           __syncwarp();
           if (lane == 0) mbar_arrive(&b_rempty[rs]);
           rr.next(P.RR);
@@ -590,32 +635,27 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         __syncwarp();
         if (lane == 0) mbar_arrive(&b_pfull[s]);
         if (p < P.NPd) {
-          // transpose this warp's 32 features x 64 tokens into C^T (TMEM lanes 32cw ..
-          // 32cw+31 of latent group p): per 16 features, four 16-token blocks
+          // transpose this warp's 16 features x 64 tokens into C^T (TMEM lanes fb .. fb+15
+          // of latent group p): four 16-token blocks
           if (p == 0) {   // the output MMAs of tile - 2 have finished reading this buffer
             fail = fail || !mbar_wait(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u, abort,
                                       kLimitNs);
             tc_fence_after();
           }
           if (!fail && owns) {
-            const uint32_t abase = smem_u32(pair + (cw >> 1) * kAtom);
+            const uint32_t abase = smem_u32(pair + (cq >> 1) * kAtom);
             const int mi = lane >> 3, r8 = lane & 7;
+            const int cc = 4 * (cq & 1) + 2 * ch + (mi >> 1);
+            uint32_t rr[16];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              uint32_t rr[16];
-              const int cc = 4 * (cw & 1) + 2 * h + (mi >> 1);
+            for (int tg = 0; tg < 4; ++tg) {
+              const int tok = 16 * tg + 8 * (mi & 1) + r8;
+              uint32_t d4[4];
+              ldsm_x4_trans(abase + tok * 128 + ((cc ^ (tok & 7)) << 4), d4);
 #pragma unroll
-              for (int tg = 0; tg < 4; ++tg) {
-                const int tok = 16 * tg + 8 * (mi & 1) + r8;
-                uint32_t d4[4];
-                ldsm_x4_trans(abase + tok * 128 + ((cc ^ (tok & 7)) << 4), d4);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) rr[4 * tg + i] = d4[i];
-              }
-              tmem_st16x256b_x4(tmem + ((uint32_t)(32 * cw + 16 * h) << 16) + kCtCol0 +
-                                    128u * ctb + 32u * p,
-                                rr);
+              for (int i = 0; i < 4; ++i) rr[4 * tg + i] = d4[i];
             }
+            tmem_st16x256b_x4(tmem + ((uint32_t)fb << 16) + kCtCol0 + 128u * ctb + 32u * p, rr);
           }
         }
         __syncwarp();
@@ -629,6 +669,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       cursor_next(c, off, a.batch, lo, hi);
     }
   } else if (has_work) {
+    regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax
     // TMEM holds S^T with tokens on lanes: the M = 64 layout puts rows 16q .. 16q+15 in
     // lanes 32q .. 32q+15.  Loaded with the 16x256b shape, thread t of warp q holds rows
@@ -648,7 +689,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
 
     float l[2 * NB];    // partial weight sums of this thread's heads
     float mr[2 * NB];   // reference max of this thread's heads (log2 units)
-    float qsi[2 * NB];   // 2^-e_h of this thread's heads for the current piece
+    const float* qsi = nullptr;   // 2^-e_h of the current piece's heads (shared memory)
     int pt = 0;
     Cursor c;
     cursor_start(c, seq0, off, a.batch, lo, hi);
@@ -656,30 +697,27 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     // K slot of this thread's rows in P: the transposed C^T holds, in the 16 K slots of each
     // step, tokens 0,1,8,9,2,3,10,11,4,5,12,13,6,7,14,15 of the step's 16 tokens
     const int ka = 16 * q + 4 * (lane >> 3) + ((lane >> 2) & 1), kb = ka + 2;
-    // token scales of rows ra / rb, loaded one tile ahead so the load latency overlaps the
-    // current tile
-    auto load_scales = [&](const Cursor& cc, float& sa, float& sbv) {
-      const __half* sp = a.scales + (int64_t)cc.seq * a.max_tokens + cc.pos;
-      sa = (ra < cc.cnt) ? __half2float(sp[ra]) : 0.f;
-      sbv = (rb < cc.cnt) ? __half2float(sp[rb]) : 0.f;
-    };
-    float s_a_next = 0.f, s_b_next = 0.f;
-    if (c.valid) load_scales(c, s_a_next, s_b_next);
+    // Token scales of rows ra / rb come from the tile's scale window in shared memory
+    // (bulk-copied by the TMA warp at least a tile ahead): no global loads in this role, so
+    // the proxy fence after each P write has nothing outstanding to wait for.
+    Ring sr;
     while (c.valid) {
       const int t = c.tile, sb = t & 1;
-      const float s_a = s_a_next, s_b = s_b_next;
+      float s_a = 0.f, s_b = 0.f;
       {
-        Cursor cn = c;
-        cursor_next(cn, off, a.batch, lo, hi);
-        if (cn.valid) load_scales(cn, s_a_next, s_b_next);
+        fail = fail || !mbar_wait(&b_scfull[sr.slot], sr.phase, abort, kLimitNs);
+        const __half* w = reinterpret_cast<const __half*>(m->sc[sr.slot]) +
+                          ((reinterpret_cast<uintptr_t>(a.scales + (int64_t)c.seq * a.max_tokens +
+                                                        c.pos) & 15u) >> 1);
+        if (ra < c.cnt) s_a = __half2float(w[ra]);
+        if (rb < c.cnt) s_b = __half2float(w[rb]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b_scempty[sr.slot]);
+        sr.next(kScSlots);
       }
       if (c.first) {
         fail = fail || !mbar_wait(b_qfull, (uint32_t)c.piece & 1u, abort, kLimitNs);
-#pragma unroll
-        for (int j = 0; j < NB; ++j) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) qsi[2 * j + e] = m->qs_inv[c.piece & 1][8 * j + hc + e];
-        }
+        qsi = m->qs_inv[c.piece & 1] + hc;
         __syncwarp();
         if (lane == 0) mbar_arrive(b_qseen);
 #pragma unroll
@@ -694,11 +732,19 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       fail = fail || !mbar_wait(b_sfull, (uint32_t)t & 1u, abort, kLimitNs);
       tc_fence_after();
       float x[4 * NB];
-      if constexpr (NB >= 6) {
+      if constexpr (NB == 8) {
         float v[32];
         tmem_ld16x256b_x8(lb + kSCol, v);
 #pragma unroll
-        for (int i = 0; i < 4 * NB; ++i) x[i] = v[i];
+        for (int i = 0; i < 32; ++i) x[i] = v[i];
+      } else if constexpr (NB == 6) {   // columns 0-31 and 32-47
+        float v[16], w[8];
+        tmem_ld16x256b_x4(lb + kSCol, v);
+        tmem_ld16x256b_x2(lb + kSCol + 32u, w);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = v[i];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[16 + i] = w[i];
       } else if constexpr (NB == 4) {
         float v[16];
         tmem_ld16x256b_x4(lb + kSCol, v);
@@ -720,8 +766,9 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const bool hv = (8 * j + hc + e) < a.H;
-          x[4 * j + e] = (va && hv) ? x[4 * j + e] * qsi[2 * j + e] * ca : -INFINITY;
-          x[4 * j + 2 + e] = (vb && hv) ? x[4 * j + 2 + e] * qsi[2 * j + e] * cbf : -INFINITY;
+          const float qh = qsi[8 * j + e];
+          x[4 * j + e] = (va && hv) ? x[4 * j + e] * qh * ca : -INFINITY;
+          x[4 * j + 2 + e] = (vb && hv) ? x[4 * j + 2 + e] * qh * cbf : -INFINITY;
           mine = mine || (x[4 * j + e] > mr[2 * j + e] + 8.f) ||
                  (x[4 * j + 2 + e] > mr[2 * j + e] + 8.f);
         }
@@ -855,19 +902,19 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           a.ws_ml[2 * (slot * a.H + h) + 1] = L;
         }
         if (!fail) {
+          float* wo = a.ws_o + slot * a.H * a.d + 32 * q + lane;   // feature 32q + lane, head 0
+#pragma unroll 1
           for (int p = 0; p < P.NPd; ++p) {
-            const int f = 128 * p + 32 * q + lane;
-#pragma unroll
+            const bool fv = 128 * p + 32 * q + lane < a.d;
+#pragma unroll 1
             for (int cb = 0; cb < NH; cb += 8) {
               float v[8];
               tmem_ld8(lb + kOCol0 + (uint32_t)P.N2 * p + cb, v);
               tmem_wait_ld();
-              if (f < a.d) {
+              if (fv) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                  const int h = cb + k;
-                  if (h < a.H) a.ws_o[(slot * a.H + h) * a.d + f] = v[k] * srun;
-                }
+                for (int k = 0; k < 8; ++k)
+                  if (cb + k < a.H) wo[(int64_t)(cb + k) * a.d + 128 * p] = v[k] * srun;
               }
             }
           }
@@ -915,7 +962,7 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
   P.NK16 = (n + 15) / 16;
   // TMEM: S^T (N1 <= 64 columns), two C^T buffers of 4 x 32 columns, O^T NPd x N2 columns
   if (H < 1 || P.N2 > 64 || P.NPd > 4 || kOCol0 + (uint32_t)(P.NPd * P.N2) > kTmemCols) return pl;
-  if (P.NQA * 8 > 32 * kQC) return pl;   // staged query rows of up to 1024 features
+  if (P.NQA * 8 > 32 * kQC) return pl;   // staged query rows of up to 768 features
   const size_t q_bytes = (size_t)P.NQA * P.N1 * 128;
   P.lbo_p = (uint32_t)P.N2 * 16u + 32u;
   P.p_bytes = 8u * P.lbo_p;

@@ -95,7 +95,8 @@ typedef enum { KVK_F32 = 0, KVK_BF16 = 1, KVK_F16 = 2 } kvk_dtype;
  * arena header (status flags) is zeroed by one synchronous cudaMemset.
  * Arena layout: 256-byte header, then per anchor (in layer order) a codes plane
  * [max_batch][max_tokens][row_bytes] and an fp16 scale plane [max_batch][max_tokens],
- * each 256-byte aligned.  row_bytes = ceil((d + d_rope) * b / 8) rounded up to 16.
+ * each 256-byte aligned, and 256 bytes of tail slack (read, never written, by the decode).
+ * row_bytes = ceil((d + d_rope) * b / 8) rounded up to 16.
  * Packed row format: field u_i = code_i + 2^(b-1) (offset binary) at bit i*b of the row
  * read as a little-endian bit stream, i over [c[0..d) || k^R[0..d_rope)], zero padding.
  */
