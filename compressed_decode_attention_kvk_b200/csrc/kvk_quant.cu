@@ -56,11 +56,8 @@ quant_write_kernel(uint8_t* __restrict__ codes, __half* __restrict__ scales, int
   if (tok >= (int64_t)batch * n_new) return;
   const int seq = (int)(tok / n_new);
   const int j = (int)(tok - (int64_t)seq * n_new);
+  // the write position is loaded alongside the token's values (neither depends on the other)
   const int64_t pos = (int64_t)__ldg(start_pos + seq) + j;
-  if (pos < 0 || pos >= max_tokens) {
-    if (lane == 0) atomicOr(flags, KVK_FLAG_WRITE_RANGE);
-    return;
-  }
   const int n = d + d_rope;
   const int groups = n >> 3;            // d % 16 == 0 and d_rope % 8 == 0
   const int d_groups = d >> 3;
@@ -86,6 +83,10 @@ quant_write_kernel(uint8_t* __restrict__ codes, __half* __restrict__ scales, int
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   finite = __all_sync(0xffffffffu, finite);
+  if (pos < 0 || pos >= max_tokens) {
+    if (lane == 0) atomicOr(flags, KVK_FLAG_WRITE_RANGE);
+    return;
+  }
 
   const int q = (1 << (b - 1)) - 1;
   const float s32 = __fdiv_rn(amax, (float)q);          // IEEE binary32 division
