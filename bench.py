@@ -82,6 +82,24 @@ def barrier(pg, device=None):
             pg.barrier()
 
 
+def decode_traffic():
+    """DRAM bytes per full-size decode launch of the tensor-core kernel, from the committed ncu
+    capture (profiles/decode_tc_traffic.json), or None when the kernel source has changed
+    since that capture (the record keeps the source's sha256)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "decode_tc_traffic.json")) as f:
+            rec = json.load(f)
+        src = os.path.join(ROOT, "compressed_decode_attention_kvk_b200", "csrc", "kvk_decode_tc.cu")
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        if sha != rec["source_sha256"]:
+            return None
+        return rec
+    except Exception:
+        return None
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -267,12 +285,17 @@ def run_kvk(args, rank, world, local, pg):
     total_bytes = wl.decode_bytes * args.steps * world
     value = total_bytes / (t_ms * 1e-3) / 1e9
     roof = None
+    traffic = decode_traffic()
     if dec_ms:
         ach = (wl.decode_bytes / L) / (dec_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(ach / peak, 4), "traffic": None, "peak_kind": peak_kind,
                 "kernel": "kvk_mla_decode (split decode + merge), mean over layers",
                 "launch_ms": round(dec_ms, 5)}
+        if traffic is not None:
+            # DRAM bytes / algorithmic bytes of one captured launch, applied to the mean layer
+            roof["traffic"] = int(traffic["dram_over_algorithmic"] * wl.decode_bytes / L)
+            roof["traffic_note"] = traffic["note"]
 
     # ---- end to end through the C ABI with host buffers -------------------------------
     e2e = None

@@ -51,8 +51,18 @@ constexpr int kConvThreads = 32 * kConvWarps;
 constexpr int kTmaWarp = 12;
 constexpr int kMmaWarp = 13;   // score MMAs; owns TMEM
 constexpr int kMma2Warp = 14;  // output MMAs
+// Register budgets.  The block is launched with kLaunchRegs per thread (the host checks that
+// ptxas allocated exactly that before choosing this kernel); a warpgroup whose budget is
+// above it raises it (setmaxnreg.inc), one below lowers it (.dec) -- never the other way,
+// which would be an illegal instruction -- and the budgets sum to no more than the launch.
+constexpr uint32_t kLaunchRegs = 65536 / kThreads;   // 128
 constexpr uint32_t kRegsSoftmax = 192, kRegsConvert = 120, kRegsIssue = 56;
 static_assert(128 * (kRegsSoftmax + 2 * kRegsConvert + kRegsIssue) <= 65536, "register split");
+template <uint32_t N>
+__device__ __forceinline__ void regs_set() {
+  if constexpr (N > kLaunchRegs) regs_inc<N>();
+  else if constexpr (N < kLaunchRegs) regs_dec<N>();
+}
 constexpr int kTile = kTcTileTokens;   // 64
 constexpr int kAtom = 8192;            // 64 rows x 128 bytes (64 f16 features)
 constexpr int kPair = 2 * kAtom;       // 128 features
@@ -359,7 +369,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   // Roles by warpgroup; each warpgroup first sets its register budget (one call site per
   // warpgroup, executed by all four of its warps).
   if (has_work && warp >= kTmaWarp) {
-    regs_dec<kRegsIssue>();
+    regs_set<kRegsIssue>();
     if (warp == kTmaWarp) {
       // ------------------------------------------------------------------ TMA producer
       if (lane == 0) {
@@ -493,7 +503,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       __syncwarp();
     }
   } else if (has_work && warp >= kConvWarp0) {
-    regs_dec<kRegsConvert>();
+    regs_set<kRegsConvert>();
     // ------------------------------------------------------------------ convert
     // The convert warps leave their loop only together (named_or agreement at the top of
     // every tile), so their named barriers never wait for a warp that has gone.  Warp cw
@@ -669,7 +679,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       cursor_next(c, off, a.batch, lo, hi);
     }
   } else if (has_work) {
-    regs_inc<kRegsSoftmax>();
+    regs_set<kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax
     // TMEM holds S^T with tokens on lanes: the M = 64 layout puts rows 16q .. 16q+15 in
     // lanes 32q .. 32q+15.  Loaded with the 16x256b shape, thread t of warp q holds rows
@@ -1011,10 +1021,44 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
   return pl;
 }
 
+// Registers per thread ptxas allocated to an instance (0 if it cannot be queried, e.g. no GPU).
+template <int BITS, int NH>
+int instance_regs() {
+  static int regs = -1;
+  if (regs < 0) {
+    cudaFuncAttributes fa;
+    regs = (cudaFuncGetAttributes(&fa, decode_tc_kernel<BITS, NH>) == cudaSuccess) ? fa.numRegs : 0;
+  }
+  return regs;
+}
+template <int BITS>
+int instance_regs_nh(int N2) {
+  switch (N2) {
+    case 16: return instance_regs<BITS, 16>();
+    case 32: return instance_regs<BITS, 32>();
+    case 48: return instance_regs<BITS, 48>();
+    case 64: return instance_regs<BITS, 64>();
+  }
+  return 0;
+}
+// The register budgets assume the launch allocation kLaunchRegs; anything else would make
+// the budget changes invalid or leave an increase waiting for registers that never come.
+bool launch_regs_ok(int b, int N2) {
+  int r = 0;
+  switch (b) {
+    case 16: r = instance_regs_nh<16>(N2); break;
+    case 8: r = instance_regs_nh<8>(N2); break;
+    case 4: r = instance_regs_nh<4>(N2); break;
+    case 2: r = instance_regs_nh<2>(N2); break;
+  }
+  return r == (int)kLaunchRegs;
+}
+
 template <int BITS, int NH>
 cudaError_t launch_bits_nh(const TcParams& P, const CUtensorMap& tmap, size_t smem, int grid,
                            cudaStream_t st) {
   auto k = decode_tc_kernel<BITS, NH>;
+  if (instance_regs<BITS, NH>() != (int)kLaunchRegs) return cudaErrorNotSupported;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k<<<grid, kThreads, smem, st>>>(P, tmap);
@@ -1038,7 +1082,8 @@ cudaError_t launch_bits(const TcParams& P, const CUtensorMap& tmap, size_t smem,
 bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H, bool has_keep) {
   if (dtype != KVK_BF16 && dtype != KVK_F16) return false;
   if (has_keep || !A.tmap_ok) return false;
-  return make_plan(A.d, L->d_rope, A.b, H, L->max_batch).ok;
+  const Plan pl = make_plan(A.d, L->d_rope, A.b, H, L->max_batch);
+  return pl.ok && launch_regs_ok(A.b, pl.p.N2);
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, const AnchorDesc& A, int dtype, int,

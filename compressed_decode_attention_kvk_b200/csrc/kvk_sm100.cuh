@@ -185,8 +185,20 @@ __device__ __forceinline__ void mma1_elect(uint32_t d_tmem, uint64_t a, uint64_t
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
+// One MMA with A read from tensor memory (see mma4_ts_elect).
+__device__ __forceinline__ void mma1_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                              uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
 // Four MMAs with A read from tensor memory: D (+)= A_k * B_k, A_k at column a_tmem + k*a_cols
-// (M = 128 lanes, two 16-bit K elements per 32-bit column), B_k by descriptor.
+// (two 16-bit K elements per 32-bit column; rows on lanes as for an accumulator of the same
+// M: lane r for M = 128, lane 32 (r / 16) + r % 16 for M = 64), B_k by descriptor.
 __device__ __forceinline__ void mma4_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint32_t a_cols,
                                               uint64_t b, uint32_t b_step, uint32_t idesc,
                                               uint32_t acc) {
@@ -203,6 +215,31 @@ __device__ __forceinline__ void mma4_ts_elect(uint32_t d_tmem, uint32_t a_tmem, 
       "r"(a_tmem), "r"(a1), "r"(a2), "r"(a3), "l"(b), "l"(b1), "l"(b2), "l"(b3), "r"(idesc),
       "r"(acc)
       : "memory");
+}
+
+// 8-byte shared-memory store by 32-bit shared address
+__device__ __forceinline__ void sts64(uint32_t saddr, uint32_t x, uint32_t y) {
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(saddr), "r"(x), "r"(y) : "memory");
+}
+// 8-byte shared-memory load by 32-bit shared address
+__device__ __forceinline__ uint2 lds64(uint32_t saddr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(saddr) : "memory");
+  return v;
+}
+// 16-byte shared-memory load / store by 32-bit shared address
+__device__ __forceinline__ uint4 lds128(uint32_t saddr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(saddr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t saddr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
 // ldmatrix, four 8x8 16-bit matrices, transposed: thread t supplies the row address of row
