@@ -213,14 +213,14 @@ class DecodeWorkload:
             info = self.lay.layer_info(l)
             self.bytes_per_layer.append(self.B * self.T * (info["row_bytes"] + 2))
         self.decode_bytes = sum(self.bytes_per_layer)
-        self.launches_per_step = len(self.anchors) + 2 * w.n_layers
+        self.launches_per_step = 1 + 2 * w.n_layers   # one append launch for every anchor
 
     def step(self, events=None):
         from compressed_decode_attention_kvk_b200 import kvk
         h = self.lay.handle
-        for l in self.anchors:
-            c, kr = self.app[l]
-            kvk.kvk_quant_write(h, l, c, kr, self.app_pos)
+        # the new token of every anchor layer, quantised and written in one launch
+        kvk.kvk_quant_write_layers(h, self.anchors, [self.app[l][0] for l in self.anchors],
+                                   [self.app[l][1] for l in self.anchors], self.app_pos)
         for l in range(self.w.n_layers):
             ql, qr = self.q[l]
             if events is not None:
@@ -350,7 +350,8 @@ def run_e2e(args, wl, device, pg):
             dc, dk = d_app[l]
             dc.copy_(h_app[l][0], non_blocking=True)
             dk.copy_(h_app[l][1], non_blocking=True)
-            kvk.kvk_quant_write(wl.lay.handle, l, dc, dk, wl.app_pos)
+        kvk.kvk_quant_write_layers(wl.lay.handle, wl.anchors, [d_app[l][0] for l in wl.anchors],
+                                   [d_app[l][1] for l in wl.anchors], wl.app_pos)
         for l in range(L):
             qa, qb = d_q[l]
             qa.copy_(h_q[l][0], non_blocking=True)

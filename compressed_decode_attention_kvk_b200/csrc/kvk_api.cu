@@ -259,6 +259,55 @@ kvk_status kvk_quant_write(kvk_layout* L, int layer, const void* c_kv, int dtype
   return e == cudaSuccess ? KVK_OK : KVK_ERR_CUDA;
 }
 
+kvk_status kvk_quant_write_layers(kvk_layout* L, int n, const int32_t* layers,
+                                  const void* const* c_kv, int dtype,
+                                  const int64_t* c_stride_seq, const int64_t* c_stride_tok,
+                                  const void* const* k_rope, const int64_t* kr_stride_seq,
+                                  const int64_t* kr_stride_tok, int batch,
+                                  const int32_t* dev_start_pos, int n_new, kvk_stream_t stream) {
+  if (!L || n < 1 || n > KVK_MAX_WRITE_LAYERS || !layers || !c_kv || !c_stride_seq ||
+      !c_stride_tok || !k_rope || !kr_stride_seq || !kr_stride_tok)
+    return KVK_ERR_INVALID_ARG;
+  if (!L->arena) return KVK_ERR_INVALID_ARG;
+  if (dtype != KVK_F32 && dtype != KVK_BF16) return KVK_ERR_INVALID_ARG;
+  if (batch < 1 || batch > L->max_batch || n_new < 0) return KVK_ERR_INVALID_ARG;
+  if (!dev_start_pos) return KVK_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(dev_start_pos) & 3u) return KVK_ERR_ALIGNMENT;
+  kvk::QuantLayers Q;
+  for (int k = 0; k < n; ++k) {
+    const int layer = layers[k];
+    if (layer < 0 || layer >= L->n_layers) return KVK_ERR_INVALID_ARG;
+    if (L->anchor[layer] != layer) return KVK_ERR_INHERITING_LAYER;
+    for (int j = 0; j < k; ++j)
+      if (layers[j] == layer) return KVK_ERR_INVALID_ARG;
+    if (!c_kv[k] || (L->d_rope > 0 && !k_rope[k])) return KVK_ERR_INVALID_ARG;
+    if (c_stride_seq[k] < 0 || c_stride_tok[k] < 0 || kr_stride_seq[k] < 0 ||
+        kr_stride_tok[k] < 0)
+      return KVK_ERR_INVALID_ARG;
+    if (!aligned16(c_kv[k]) || (k_rope[k] && !aligned16(k_rope[k]))) return KVK_ERR_ALIGNMENT;
+    if (c_stride_seq[k] % 8 || c_stride_tok[k] % 8 || kr_stride_seq[k] % 8 ||
+        kr_stride_tok[k] % 8)
+      return KVK_ERR_ALIGNMENT;
+    const AnchorDesc& A = L->anchors[L->slot[layer]];
+    kvk::QuantLayer& q = Q.l[k];
+    q.codes = L->arena + A.codes_off;
+    q.scales = reinterpret_cast<__half*>(L->arena + A.scales_off);
+    q.row_bytes = A.row_bytes;
+    q.d = A.d;
+    q.b = A.b;
+    q.c_kv = c_kv[k];
+    q.c_ss = c_stride_seq[k];
+    q.c_st = c_stride_tok[k];
+    q.k_rope = k_rope[k];
+    q.kr_ss = kr_stride_seq[k];
+    q.kr_st = kr_stride_tok[k];
+  }
+  if (n_new == 0) return KVK_OK;
+  cudaError_t e = kvk::launch_quant_write_layers(L, Q, n, dtype, batch, dev_start_pos, n_new,
+                                                 reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVK_OK : KVK_ERR_CUDA;
+}
+
 static int choose_path(const kvk_layout* L, const AnchorDesc& A, int dtype, int H,
                        bool has_keep) {
   if (L->path == KVK_PATH_CUDA_CORE) return KVK_PATH_CUDA_CORE;

@@ -90,6 +90,22 @@ cudaError_t launch_quant_write(const kvk_layout* L, const AnchorDesc& A, const v
                                int dtype, int64_t c_ss, int64_t c_st, const void* k_rope,
                                int64_t kr_ss, int64_t kr_st, int batch, const int32_t* start_pos,
                                int n_new, cudaStream_t stream);
+// One layer of a multi-layer quantise-on-write launch.
+struct QuantLayer {
+  uint8_t* codes;
+  __half* scales;
+  int row_bytes, d, b;
+  const void* c_kv;
+  int64_t c_ss, c_st;
+  const void* k_rope;
+  int64_t kr_ss, kr_st;
+};
+struct QuantLayers {
+  QuantLayer l[KVK_MAX_WRITE_LAYERS];
+};
+cudaError_t launch_quant_write_layers(const kvk_layout* L, const QuantLayers& Q, int n, int dtype,
+                                      int batch, const int32_t* start_pos, int n_new,
+                                      cudaStream_t stream);
 cudaError_t launch_decode_fma(const DecodeArgs& a, int dtype, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeArgs& a, const AnchorDesc& A, int dtype, int num_sms,
                              cudaStream_t stream);

@@ -15,6 +15,7 @@ namespace {
 
 constexpr int kMergeThreads = 128;
 constexpr int kChunk = 256;   // pieces whose weights are staged in shared memory at once
+constexpr int kFew = 8;       // at most this many pieces: single-round register path
 constexpr float kLn2 = 0.6931471805599453f;
 
 template <bool kMax>
@@ -53,6 +54,53 @@ __global__ void __launch_bounds__(kMergeThreads, 4) merge_kernel(DecodeArgs a) {
     const int64_t sh = (int64_t)(c0 + k + i) * a.H + h;
     return *reinterpret_cast<const float2*>(a.ws_ml + 2 * sh);
   };
+  const int d4 = a.d >> 2;   // d is a multiple of 16
+  if (np <= kFew && d4 <= kMergeThreads) {
+    // Few pieces (the usual case): every thread loads all pieces' (m, l) and its four output
+    // features of every piece in one round of independent loads, then reduces in registers.
+    float2 mlv[kFew];
+    float4 ov[kFew];
+    const float4* src =
+        reinterpret_cast<const float4*>(a.ws_o + ((int64_t)(c0 + i) * a.H + h) * a.d) + tid;
+    const int64_t stride = (int64_t)a.H * d4;   // float4s between consecutive pieces
+#pragma unroll
+    for (int k = 0; k < kFew; ++k) {
+      mlv[k] = make_float2(0.f, 0.f);
+      ov[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (k < np) {
+        mlv[k] = ml(k);
+        if (tid < d4) ov[k] = src[k * stride];
+      }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kFew; ++k)
+      if (k < np && mlv[k].y > 0.0f) M = fmaxf(M, mlv[k].x);
+    if (M == -INFINITY) {
+      if (tid < d4) reinterpret_cast<float4*>(out)[tid] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (a.lse && tid == 0) a.lse[(int64_t)i * a.H + h] = -INFINITY;
+      return;
+    }
+    float lsum = 0.0f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < kFew; ++k) {
+      if (k < np && mlv[k].y > 0.0f) {
+        const float w = exp2f(mlv[k].x - M);
+        lsum += w * mlv[k].y;
+        acc.x = fmaf(w, ov[k].x, acc.x);
+        acc.y = fmaf(w, ov[k].y, acc.y);
+        acc.z = fmaf(w, ov[k].z, acc.z);
+        acc.w = fmaf(w, ov[k].w, acc.w);
+      }
+    }
+    const float inv = 1.0f / lsum;
+    if (tid < d4)
+      reinterpret_cast<float4*>(out)[tid] =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    if (a.lse && tid == 0) a.lse[(int64_t)i * a.H + h] = kLn2 * (M + log2f(lsum));
+    return;
+  }
   float M = -INFINITY;
   for (int k = tid; k < np; k += kMergeThreads) {
     const float2 v = ml(k);
@@ -71,7 +119,6 @@ __global__ void __launch_bounds__(kMergeThreads, 4) merge_kernel(DecodeArgs a) {
   }
   const float lsum = block_reduce<false>(ls, red);
   const float inv = 1.0f / lsum;
-  const int d4 = a.d >> 2;   // d is a multiple of 16
   for (int j0 = 0; j0 < d4; j0 += kMergeThreads) {
     const int j = j0 + tid;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);

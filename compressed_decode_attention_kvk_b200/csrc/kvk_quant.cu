@@ -44,15 +44,14 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, flo
   }
 }
 
+// One warp quantises token `tok` (of batch x n_new) of one anchor layer.
 template <typename T>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
-quant_write_kernel(uint8_t* __restrict__ codes, __half* __restrict__ scales, int row_bytes,
-                   int d, int d_rope, int b, int max_tokens, const T* __restrict__ c_kv,
-                   int64_t c_ss, int64_t c_st, const T* __restrict__ k_rope, int64_t kr_ss,
-                   int64_t kr_st, int batch, const int32_t* __restrict__ start_pos, int n_new,
-                   uint32_t* __restrict__ flags) {
+__device__ __forceinline__ void quant_token(
+    int64_t tok, uint8_t* __restrict__ codes, __half* __restrict__ scales, int row_bytes, int d,
+    int d_rope, int b, int max_tokens, const T* __restrict__ c_kv, int64_t c_ss, int64_t c_st,
+    const T* __restrict__ k_rope, int64_t kr_ss, int64_t kr_st, int batch,
+    const int32_t* __restrict__ start_pos, int n_new, uint32_t* __restrict__ flags) {
   const int lane = threadIdx.x & 31;
-  const int64_t tok = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   if (tok >= (int64_t)batch * n_new) return;
   const int seq = (int)(tok / n_new);
   const int j = (int)(tok - (int64_t)seq * n_new);
@@ -139,6 +138,31 @@ quant_write_kernel(uint8_t* __restrict__ codes, __half* __restrict__ scales, int
   if (lane < row_bytes - used) row[used + lane] = 0;
 }
 
+template <typename T>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+quant_write_kernel(uint8_t* __restrict__ codes, __half* __restrict__ scales, int row_bytes,
+                   int d, int d_rope, int b, int max_tokens, const T* __restrict__ c_kv,
+                   int64_t c_ss, int64_t c_st, const T* __restrict__ k_rope, int64_t kr_ss,
+                   int64_t kr_st, int batch, const int32_t* __restrict__ start_pos, int n_new,
+                   uint32_t* __restrict__ flags) {
+  quant_token<T>((int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5), codes, scales,
+                 row_bytes, d, d_rope, b, max_tokens, c_kv, c_ss, c_st, k_rope, kr_ss, kr_st,
+                 batch, start_pos, n_new, flags);
+}
+
+// Several anchor layers in one launch: blockIdx.y picks the layer.
+template <typename T>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+quant_write_layers_kernel(const __grid_constant__ QuantLayers Q, int d_rope, int max_tokens,
+                          int batch, const int32_t* __restrict__ start_pos, int n_new,
+                          uint32_t* __restrict__ flags) {
+  const QuantLayer& l = Q.l[blockIdx.y];
+  quant_token<T>((int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5), l.codes, l.scales,
+                 l.row_bytes, l.d, d_rope, l.b, max_tokens, static_cast<const T*>(l.c_kv),
+                 l.c_ss, l.c_st, static_cast<const T*>(l.k_rope), l.kr_ss, l.kr_st, batch,
+                 start_pos, n_new, flags);
+}
+
 }  // namespace
 
 cudaError_t launch_quant_write(const kvk_layout* L, const AnchorDesc& A, const void* c_kv,
@@ -163,6 +187,23 @@ cudaError_t launch_quant_write(const kvk_layout* L, const AnchorDesc& A, const v
         static_cast<const float*>(c_kv), c_ss, c_st, static_cast<const float*>(k_rope), kr_ss,
         kr_st, batch, start_pos, n_new, flags);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_write_layers(const kvk_layout* L, const QuantLayers& Q, int n, int dtype,
+                                      int batch, const int32_t* start_pos, int n_new,
+                                      cudaStream_t stream) {
+  const int64_t tokens = (int64_t)batch * n_new;
+  const int64_t blocks = (tokens + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  if (blocks > 0x7FFFFFFF || n < 1 || n > KVK_MAX_WRITE_LAYERS) return cudaErrorInvalidValue;
+  uint32_t* flags = reinterpret_cast<uint32_t*>(L->arena);
+  dim3 grid((unsigned)blocks, (unsigned)n), block(kWarpsPerBlock * 32);
+  if (dtype == KVK_BF16)
+    quant_write_layers_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
+        Q, L->d_rope, L->max_tokens, batch, start_pos, n_new, flags);
+  else
+    quant_write_layers_kernel<float><<<grid, block, 0, stream>>>(Q, L->d_rope, L->max_tokens,
+                                                                 batch, start_pos, n_new, flags);
   return cudaGetLastError();
 }
 

@@ -32,7 +32,7 @@ _DTYPE = {torch.float32: KVK_F32, torch.bfloat16: KVK_BF16, torch.float16: KVK_F
 EXPORTED = ("kvk_create_layout", "kvk_destroy", "kvk_get_layer_info", "kvk_quant_write",
             "kvk_decode_workspace_bytes", "kvk_mla_decode", "kvk_read_status",
             "kvk_set_decode_path", "kvk_set_decode_ctas", "kvk_decode_path_for",
-            "kvk_status_string", "kvk_mla_decode_noalloc")
+            "kvk_status_string", "kvk_mla_decode_noalloc", "kvk_quant_write_layers")
 
 # size of the library's built-in scratch array used by kvk_mla_decode_noalloc
 KVK_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -69,6 +69,7 @@ def _lib_handle():
         L.kvk_destroy.restype = None
         L.kvk_get_layer_info.argtypes = [P, i32, P]
         L.kvk_quant_write.argtypes = [P, i32, P, i32, i64, i64, P, i64, i64, i32, P, i32, P]
+        L.kvk_quant_write_layers.argtypes = [P, i32, P, P, i32, P, P, P, P, P, i32, P, i32, P]
         L.kvk_decode_workspace_bytes.argtypes = [P, i32, i32, i32, P]
         L.kvk_mla_decode.argtypes = [P, i32, P, P, i32, i64, i64, i64, i64, i32, i32, P, P, P,
                                      i32, ctypes.c_float, P, P, P, sz, P]
@@ -163,6 +164,32 @@ def kvk_quant_write(handle, layer, c_kv, k_rope, start_pos, stream=None):
                                        k_rope.stride(0), k_rope.stride(1), B, _ptr(start_pos),
                                        n_new, _stream(stream))
     _check("kvk_quant_write", st)
+
+
+def kvk_quant_write_layers(handle, layers, c_kvs, k_ropes, start_pos, stream=None):
+    """kvk_quant_write for several anchor layers in one launch: layers[k] takes c_kvs[k]
+    [B, n_new, >=d] and k_ropes[k] [B, n_new, d_rope] (same dtype, batch and n_new for all)."""
+    n = len(layers)
+    if not (len(c_kvs) == len(k_ropes) == n) or n == 0:
+        raise ValueError("layers, c_kvs and k_ropes must have the same non-zero length")
+    for c_kv, k_rope in zip(c_kvs, k_ropes):
+        _need_cuda(c_kv, "c_kv", (torch.float32, torch.bfloat16))
+        _need_cuda(k_rope, "k_rope", (c_kvs[0].dtype,))
+        if c_kv.dim() != 3 or k_rope.dim() != 3 or c_kv.stride(2) != 1 or k_rope.stride(2) != 1:
+            raise ValueError("c_kv / k_rope must be [batch, n_new, width] with contiguous width")
+        if c_kv.dtype != c_kvs[0].dtype or c_kv.shape[:2] != c_kvs[0].shape[:2]:
+            raise ValueError("every layer needs the same dtype, batch and n_new")
+    B, n_new = c_kvs[0].shape[0], c_kvs[0].shape[1]
+    _need_cuda(start_pos, "start_pos", (torch.int32,))
+    I32 = ctypes.c_int32 * n
+    I64 = ctypes.c_int64 * n
+    VP = ctypes.c_void_p * n
+    st = _lib_handle().kvk_quant_write_layers(
+        handle, n, I32(*layers), VP(*[_ptr(t) for t in c_kvs]), _DTYPE[c_kvs[0].dtype],
+        I64(*[t.stride(0) for t in c_kvs]), I64(*[t.stride(1) for t in c_kvs]),
+        VP(*[_ptr(t) for t in k_ropes]), I64(*[t.stride(0) for t in k_ropes]),
+        I64(*[t.stride(1) for t in k_ropes]), B, _ptr(start_pos), n_new, _stream(stream))
+    _check("kvk_quant_write_layers", st)
 
 
 def kvk_decode_workspace_bytes(handle, layer, batch, n_heads) -> int:
@@ -302,6 +329,9 @@ class Layout:
 
     def quant_write(self, layer, c_kv, k_rope, start_pos, stream=None):
         kvk_quant_write(self.handle, layer, c_kv, k_rope, start_pos, stream)
+
+    def quant_write_layers(self, layers, c_kvs, k_ropes, start_pos, stream=None):
+        kvk_quant_write_layers(self.handle, layers, c_kvs, k_ropes, start_pos, stream)
 
     def workspace_bytes(self, layer, batch, n_heads):
         return kvk_decode_workspace_bytes(self.handle, layer, batch, n_heads)

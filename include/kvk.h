@@ -156,6 +156,24 @@ kvk_status kvk_quant_write(kvk_layout* layout, int layer, const void* c_kv, int 
                            int64_t kr_stride_seq, int64_t kr_stride_tok, int batch,
                            const int32_t* dev_start_pos, int n_new, kvk_stream_t stream);
 
+/*
+ * kvk_quant_write_layers -- the same write for n distinct anchor layers in one launch (for
+ * example one decode step's append to every anchor), all with the same dtype, batch,
+ * dev_start_pos and n_new.  Layer layers[k] takes c_kv[k] / k_rope[k] with strides
+ * c_stride_seq[k], c_stride_tok[k], kr_stride_seq[k], kr_stride_tok[k] (host arrays of n
+ * entries, device tensors as in kvk_quant_write).  The result is the one n separate
+ * kvk_quant_write calls would produce.  1 <= n <= KVK_MAX_WRITE_LAYERS; every argument of
+ * every layer is checked before anything is launched, with kvk_quant_write's statuses, and a
+ * repeated layer is KVK_ERR_INVALID_ARG.
+ */
+#define KVK_MAX_WRITE_LAYERS 64
+kvk_status kvk_quant_write_layers(kvk_layout* layout, int n, const int32_t* layers,
+                                  const void* const* c_kv, int dtype,
+                                  const int64_t* c_stride_seq, const int64_t* c_stride_tok,
+                                  const void* const* k_rope, const int64_t* kr_stride_seq,
+                                  const int64_t* kr_stride_tok, int batch,
+                                  const int32_t* dev_start_pos, int n_new, kvk_stream_t stream);
+
 /* Bytes of device workspace kvk_mla_decode needs for (layer, batch, n_heads), covering
  * both decode kernels. */
 kvk_status kvk_decode_workspace_bytes(const kvk_layout* layout, int layer, int batch,

@@ -136,3 +136,50 @@ def test_quant_write_flags(pkg):
         assert e.value.status == 4
     finally:
         lay.close()
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_quant_write_layers_matches_oracle(pkg, oracle_mod, dtype):
+    """One launch over several anchor layers (different d, b, strided inputs) writes exactly
+    what the oracle gives per layer, and leaves the other layers untouched."""
+    B, T, n_new, r, dR = 4, 96, 3, 512, 64
+    anchor = [0, 0, 2, 3, 3, 5]
+    dd = [512, 0, 384, 128, 0, 256]
+    bb = [16, 0, 8, 2, 0, 4]
+    lay = pkg.Layout(anchor, dd, bb, r, dR, B, T)
+    try:
+        starts = torch.tensor([0, 17, 90, 45], dtype=torch.int32)
+        layers = [5, 0, 3]      # any order, a subset of the anchors
+        cs, ks = [], []
+        for li, layer in enumerate(layers):
+            c, kr = _inputs(B, n_new + 2, r, dR, dtype, seed=1000 + layer)
+            cs.append(c.cuda()[:, 1:1 + n_new])          # strided: skips a token per sequence
+            ks.append(kr.cuda()[:, 1:1 + n_new])
+        codes2, scales2 = lay.cache_views(2)
+        before = (codes2.clone(), scales2.clone())
+        pkg.kvk.kvk_quant_write_layers(lay.handle, layers, cs, ks, starts.cuda())
+        torch.cuda.synchronize()
+        for layer, c, kr in zip(layers, cs, ks):
+            _check_against_oracle(oracle_mod, lay, layer, c.cpu(), kr.cpu(), starts, n_new,
+                                  dd[layer], bb[layer])
+        # anchor 2 is not in the list: its planes are unchanged
+        assert torch.equal(codes2, before[0]) and torch.equal(scales2.view(torch.int16),
+                                                               before[1].view(torch.int16))
+        assert lay.read_status() == 0
+    finally:
+        lay.close()
+
+
+def test_quant_write_layers_arguments(pkg):
+    lay = pkg.Layout([0, 0, 2], [64, 0, 64], [8, 0, 4], 64, 16, 2, 32)
+    try:
+        c = torch.zeros(2, 1, 64, dtype=torch.bfloat16, device="cuda")
+        kr = torch.zeros(2, 1, 16, dtype=torch.bfloat16, device="cuda")
+        pos = torch.zeros(2, dtype=torch.int32, device="cuda")
+        for layers, status in (([0, 0], 1), ([1], 4), ([0, 7], 1)):
+            with pytest.raises(pkg.kvk.KvkError) as e:
+                pkg.kvk.kvk_quant_write_layers(lay.handle, layers, [c] * len(layers),
+                                               [kr] * len(layers), pos)
+            assert e.value.status == status, (layers, e.value.status)
+    finally:
+        lay.close()
