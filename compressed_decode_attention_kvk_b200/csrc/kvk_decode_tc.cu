@@ -73,7 +73,6 @@ constexpr uint32_t kOCol0 = 320;       // O^T group p at 320 + N2 p
 constexpr uint64_t kLimitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kSmemLimit = 232448;
-constexpr int kQH = 6;   // query rows a convert warp loads per round (one round for 48 heads)
 constexpr int kQC = 3;   // 16-byte chunks per lane per query row (rows of up to 768 features)
 // Token-scale ring: per tile a 144-byte window (the tile's 64 fp16 scales from the 16-byte
 // boundary at or below the first), loaded by the TMA warp with a plain bulk copy.
@@ -547,55 +546,55 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         const uint8_t* qlat = static_cast<const uint8_t*>(a.q_lat) + 2 * ((int64_t)c.seq * a.ql_ss);
         const uint8_t* qrope =
             static_cast<const uint8_t*>(a.q_rope) + 2 * ((int64_t)c.seq * a.qr_ss);
-        // one pass: warp cw stages heads cw, cw + 8, ..., kQH at a time with every load in
-        // flight; lane l holds chunks l, l + 32, ... of each row, the warp reduces the row's
-        // max |q|, and the row is written scaled by 2^e_h (max |q_h| in [2^14, 2^15), exact
-        // for bf16 inputs in range).  Rows >= H and chunks >= n are zero.
-        for (int h0 = cw; h0 < P.N1; h0 += kConvWarps * kQH) {
-          uint4 v[kQH][kQC];
+        // One pass: warp cw stages heads cw, cw + 8, ...; lane l holds chunks l, l + 32, ... of
+        // a row, the warp reduces the row's max |q|, and the row is written scaled by 2^e_h
+        // (max |q_h| in [2^14, 2^15), exact for bf16 inputs in range).  Rows >= H and chunks
+        // >= n are zero.  The loop body is one row (a small code footprint: this code runs
+        // once per piece and would otherwise be fetched cold), with the next row's loads
+        // issued before the current row is processed.
+        auto load_row = [&](int h, uint4 (&v)[kQC]) {
 #pragma unroll
-          for (int k = 0; k < kQH; ++k) {
-            const int h = h0 + kConvWarps * k;
+          for (int j = 0; j < kQC; ++j) {
+            const int f0 = 8 * (lane + 32 * j);
+            v[j] = make_uint4(0u, 0u, 0u, 0u);
+            if (h < a.H && f0 < a.n)
+              v[j] = *reinterpret_cast<const uint4*>(
+                  (f0 < a.d) ? qlat + 2 * ((int64_t)h * a.ql_sh + f0)
+                             : qrope + 2 * ((int64_t)h * a.qr_sh + (f0 - a.d)));
+          }
+        };
+        uint4 vc[kQC], vn[kQC];
+        if (cw < P.N1) load_row(cw, vc);
+#pragma unroll 1
+        for (int h = cw; h < P.N1; h += kConvWarps) {
+          if (h + kConvWarps < P.N1) load_row(h + kConvWarps, vn);
+          float f[kQC][8];
+          float mx = 0.f;
 #pragma unroll
-            for (int j = 0; j < kQC; ++j) {
-              const int f0 = 8 * (lane + 32 * j);
-              v[k][j] = make_uint4(0u, 0u, 0u, 0u);
-              if (h < a.H && f0 < a.n)
-                v[k][j] = *reinterpret_cast<const uint4*>(
-                    (f0 < a.d) ? qlat + 2 * ((int64_t)h * a.ql_sh + f0)
-                               : qrope + 2 * ((int64_t)h * a.qr_sh + (f0 - a.d)));
-            }
+          for (int j = 0; j < kQC; ++j) {
+            load8_bits(vc[j], P.qdtype, f[j]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[j][e]));
           }
 #pragma unroll
-          for (int k = 0; k < kQH; ++k) {
-            const int h = h0 + kConvWarps * k;
-            if (h >= P.N1) break;
-            float f[kQC][8];
-            float mx = 0.f;
+          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          const int e = (mx > 0.f && isfinite(mx)) ? 14 - ilogbf(mx) : 0;
+          const float qscale = ldexpf(1.f, e);
+          if (lane == 0) m->qs_inv[c.piece & 1][h] = ldexpf(1.f, -e);
 #pragma unroll
-            for (int j = 0; j < kQC; ++j) {
-              load8_bits(v[k][j], P.qdtype, f[j]);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[j][e]));
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            const int e = (mx > 0.f && isfinite(mx)) ? 14 - ilogbf(mx) : 0;
-            const float qscale = ldexpf(1.f, e);
-            if (lane == 0) m->qs_inv[c.piece & 1][h] = ldexpf(1.f, -e);
-#pragma unroll
-            for (int j = 0; j < kQC; ++j) {
-              const int fc = lane + 32 * j;
-              if (fc >= cpr) break;
-              uint4 o;
-              o.x = h2_bits(__floats2half2_rn(f[j][0] * qscale, f[j][1] * qscale));
-              o.y = h2_bits(__floats2half2_rn(f[j][2] * qscale, f[j][3] * qscale));
-              o.z = h2_bits(__floats2half2_rn(f[j][4] * qscale, f[j][5] * qscale));
-              o.w = h2_bits(__floats2half2_rn(f[j][6] * qscale, f[j][7] * qscale));
-              const int at = fc >> 3, jj = fc & 7;
-              *reinterpret_cast<uint4*>(q_s + at * (P.N1 * 128) + h * 128 + ((jj ^ (h & 7)) << 4)) = o;
-            }
+          for (int j = 0; j < kQC; ++j) {
+            const int fc = lane + 32 * j;
+            if (fc >= cpr) break;
+            uint4 o;
+            o.x = h2_bits(__floats2half2_rn(f[j][0] * qscale, f[j][1] * qscale));
+            o.y = h2_bits(__floats2half2_rn(f[j][2] * qscale, f[j][3] * qscale));
+            o.z = h2_bits(__floats2half2_rn(f[j][4] * qscale, f[j][5] * qscale));
+            o.w = h2_bits(__floats2half2_rn(f[j][6] * qscale, f[j][7] * qscale));
+            const int at = fc >> 3, jj = fc & 7;
+            *reinterpret_cast<uint4*>(q_s + at * (P.N1 * 128) + h * 128 + ((jj ^ (h & 7)) << 4)) = o;
           }
+#pragma unroll
+          for (int j = 0; j < kQC; ++j) vc[j] = vn[j];
         }
         fence_proxy_async_smem();
         named_sync(2, kConvThreads);   // every warp's rows written before q_full

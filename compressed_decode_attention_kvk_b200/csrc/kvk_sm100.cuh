@@ -70,24 +70,36 @@ __device__ __forceinline__ void abort_set(uint32_t saddr) {
   asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(saddr), "r"(1u) : "memory");
 }
 
+// try_wait with a suspend-time hint: the thread may sleep in hardware until the phase
+// completes or about `ns` nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_hint(uint64_t* b, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait: returns false (after setting the abort word) if the phase did not complete
-// within limit_ns, or at once (false) if another role has set the abort word.  The loop
-// spins on try_wait (which suspends the thread in hardware for a while) and looks at the
-// abort word and the clock only every 32 tries, so waiting warps take few issue slots.
+// within limit_ns, or at once (false) if another role has set the abort word.  Between
+// checks of the abort word and the clock the thread sleeps in try_wait (woken when the phase
+// completes), so waiting warps take few issue slots and each call site stays small.
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, uint32_t abort_saddr,
                                           uint64_t limit_ns) {
   if (mbar_try(b, parity)) return true;
   const uint64_t t0 = globaltimer();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try(b, parity)) return true;
+  while (!mbar_try_hint(b, parity, 20000u)) {
     if (abort_read(abort_saddr)) return false;
     if (globaltimer() - t0 > limit_ns) {
       abort_set(abort_saddr);
       return false;
     }
   }
+  return true;
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
