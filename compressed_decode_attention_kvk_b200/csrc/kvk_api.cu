@@ -398,6 +398,7 @@ kvk_status kvk_mla_decode(kvk_layout* L, int layer, const void* q_lat, const voi
   int G = kvk::decode_ctas(L, batch, path);
   size_t need = kvk::decode_workspace(batch, n_heads, A.d, G, workspace, &a);
   if (workspace_bytes < need) return KVK_ERR_WORKSPACE;
+  a.split_x = (path == KVK_PATH_TENSOR) ? kvk::kTcPieceCost : 0;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = (path == KVK_PATH_TENSOR)

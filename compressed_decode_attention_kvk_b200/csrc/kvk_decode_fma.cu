@@ -54,9 +54,10 @@ __global__ void __launch_bounds__(kHG * 32) decode_fma_kernel(DecodeArgs a) {
   block_seq_offsets(a, off, tmp);
   if (blockIdx.x == 0)
     for (int i = tid; i <= a.batch; i += nt) a.seq_off[i] = off[i];
-  const int64_t N = off[a.batch];
+  const int64_t C = off[a.batch] + (int64_t)a.split_x * a.batch;
   const int c = blockIdx.x;
-  const int64_t lo = cta_lo(c, N, a.G), hi = cta_lo(c + 1, N, a.G);
+  const int64_t lo = split_token(off, a.batch, a.split_x, split_cost(c, C, a.G));
+  const int64_t hi = split_token(off, a.batch, a.split_x, split_cost(c + 1, C, a.G));
   if (lo >= hi) return;
   // first sequence whose token range contains lo
   int seq = 0;

@@ -74,6 +74,7 @@ constexpr uint64_t kLimitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kSmemLimit = 232448;
 constexpr int kQC = 3;   // 16-byte chunks per lane per query row (rows of up to 768 features)
+constexpr int kQD = 1;   // query rows in flight per convert warp while staging
 // Token-scale ring: per tile a 144-byte window (the tile's 64 fp16 scales from the 16-byte
 // boundary at or below the first), loaded by the TMA warp with a plain bulk copy.
 constexpr int kScSlots = 4;
@@ -311,7 +312,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   if (tid == 0) {
     for (int i = 0; i < P.PR; ++i) {
       mbar_init(&b_pfull[i], kConvWarps);
-      mbar_init(&b_pempty[i], 1 + kConvWarps);   // score MMAs (commit) + the convert warps
+      // score MMAs (commit), plus the convert warps where they read the slot after q_full
+      mbar_init(&b_pempty[i], BITS == 16 ? 1 : 1 + kConvWarps);
       mbar_init(&b_tfull[i], 1);
     }
     for (int i = 0; i < P.RR; ++i) {
@@ -352,8 +354,9 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   tc_fence_after();
   const uint32_t tmem = m->tmem_base;
 
-  const int64_t N = off[a.batch];
-  const int64_t lo = cta_lo(blockIdx.x, N, a.G), hi = cta_lo(blockIdx.x + 1, N, a.G);
+  const int64_t C = off[a.batch] + (int64_t)a.split_x * a.batch;
+  const int64_t lo = split_token(off, a.batch, a.split_x, split_cost(blockIdx.x, C, a.G));
+  const int64_t hi = split_token(off, a.batch, a.split_x, split_cost(blockIdx.x + 1, C, a.G));
   int seq0 = 0;
   {
     int L = 0, H = a.batch;
@@ -382,6 +385,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         mbar_wait(b_qfull, 0u, abort, kLimitNs);
         Ring sr;   // scale ring
         uint32_t nsc = 0;
+        const uint64_t pol = policy_evict_first();   // the cache and its scales are read once
         while (c.valid && !abort_read(abort)) {
           const int row0 = c.seq * a.max_tokens + c.pos;
           bool ok = true;
@@ -389,8 +393,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
             const uintptr_t sp = reinterpret_cast<uintptr_t>(a.scales + row0);
             if (!(ok = mbar_wait(&b_scempty[sr.slot], sr.phase ^ 1u, abort, kLimitNs))) break;
             mbar_arrive_expect_tx(&b_scfull[sr.slot], kScBytes);
-            bulk_load(m->sc[sr.slot], reinterpret_cast<const void*>(sp & ~uintptr_t(15)),
-                      kScBytes, &b_scfull[sr.slot]);
+            bulk_load_hint(m->sc[sr.slot], reinterpret_cast<const void*>(sp & ~uintptr_t(15)),
+                           kScBytes, &b_scfull[sr.slot], pol);
             sr.next(kScSlots);
             ++nsc;
           }
@@ -401,12 +405,12 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
               const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
               mbar_arrive_expect_tx(&b_tfull[s], nat * kAtom);
               for (int t = 0; t < nat; ++t)
-                tma_load_2d(pairs + s * kPair + t * kAtom, &tmap, (2 * p + t) * 128, row0,
-                            &b_tfull[s]);
+                tma_load_2d_hint(pairs + s * kPair + t * kAtom, &tmap, (2 * p + t) * 128, row0,
+                                 &b_tfull[s], pol);
             } else {
               if (!(ok = mbar_wait(&b_rempty[s], ph ^ 1u, abort, kLimitNs))) break;
               mbar_arrive_expect_tx(&b_rfull[s], P.raw_slot);
-              tma_load_2d(raw + s * P.raw_slot, &tmap, p * 16 * BITS, row0, &b_rfull[s]);
+              tma_load_2d_hint(raw + s * P.raw_slot, &tmap, p * 16 * BITS, row0, &b_rfull[s], pol);
             }
             ++cnt;
             rg.next(slots);
@@ -500,6 +504,25 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       commit_elect(b_final2);
       if (lane == 0) wait_noabort(b_final2, 0);
       __syncwarp();
+    } else {
+      // ------------------------------------------------------------------ spare warp
+      // Warm L2 with the queries of the sequences after the first that this CTA touches
+      // (the convert warps stage the first one at once).
+      Cursor c;
+      cursor_start(c, seq0, off, a.batch, lo, hi);
+      const int lat_lines = (2 * a.d + 127) / 128, rope_lines = (2 * a.d_rope + 127) / 128;
+      const int lines = lat_lines + rope_lines;
+      while (c.valid) {
+        ++c.seq;
+        if (!(c.valid = find_piece(c, off, a.batch, lo, hi))) break;
+        const uint8_t* ql = static_cast<const uint8_t*>(a.q_lat) + 2 * ((int64_t)c.seq * a.ql_ss);
+        const uint8_t* qr = static_cast<const uint8_t*>(a.q_rope) + 2 * ((int64_t)c.seq * a.qr_ss);
+        for (int i = lane; i < a.H * lines; i += 32) {
+          const int h = i / lines, k = i - h * lines;
+          if (k < lat_lines) prefetch_l2(ql + 2 * ((int64_t)h * a.ql_sh) + 128 * k);
+          else prefetch_l2(qr + 2 * ((int64_t)h * a.qr_sh) + 128 * (k - lat_lines));
+        }
+      }
     }
   } else if (has_work && warp >= kConvWarp0) {
     regs_set<kRegsConvert>();
@@ -508,28 +531,12 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     // every tile), so their named barriers never wait for a warp that has gone.  Warp cw
     // sits in TMEM lane quarter cq = cw % 4 and owns features fb .. fb+15 of every group,
     // fb = 32 cq + 16 ch (ch = cw / 4): TMEM lanes fb .. fb+15 of C^T.
-    const int ct = tid - kConvWarp0 * 32, cw = warp - kConvWarp0;
+    const int cw = warp - kConvWarp0;
     const int cq = cw & 3, ch = cw >> 2, fb = 32 * cq + 16 * ch;
     Ring pr, rr;   // f16 group ring, packed group ring
     int last_piece = -1;
     bool fail = false;
     const int cpr = P.NQA * 8;   // 16-byte chunks per staged query row
-    {  // warm L2 with the queries of every sequence this CTA touches
-      Cursor c;
-      cursor_start(c, seq0, off, a.batch, lo, hi);
-      while (c.valid) {
-        const uint8_t* ql = static_cast<const uint8_t*>(a.q_lat) + 2 * ((int64_t)c.seq * a.ql_ss);
-        const uint8_t* qr = static_cast<const uint8_t*>(a.q_rope) + 2 * ((int64_t)c.seq * a.qr_ss);
-        const int lat_lines = (2 * a.d + 127) / 128, rope_lines = (2 * a.d_rope + 127) / 128;
-        for (int i = ct; i < a.H * (lat_lines + rope_lines); i += kConvThreads) {
-          const int h = i / (lat_lines + rope_lines), k = i - h * (lat_lines + rope_lines);
-          if (k < lat_lines) prefetch_l2(ql + 2 * ((int64_t)h * a.ql_sh) + 128 * k);
-          else prefetch_l2(qr + 2 * ((int64_t)h * a.qr_sh) + 128 * (k - lat_lines));
-        }
-        ++c.seq;
-        c.valid = find_piece(c, off, a.batch, lo, hi);
-      }
-    }
     Cursor c;
     cursor_start(c, seq0, off, a.batch, lo, hi);
     while (c.valid) {
@@ -550,8 +557,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         // a row, the warp reduces the row's max |q|, and the row is written scaled by 2^e_h
         // (max |q_h| in [2^14, 2^15), exact for bf16 inputs in range).  Rows >= H and chunks
         // >= n are zero.  The loop body is one row (a small code footprint: this code runs
-        // once per piece and would otherwise be fetched cold), with the next row's loads
-        // issued before the current row is processed.
+        // once per piece and would otherwise be fetched cold); the loads of the next kQD rows
+        // are in flight while a row is processed.
         auto load_row = [&](int h, uint4 (&v)[kQC]) {
 #pragma unroll
           for (int j = 0; j < kQC; ++j) {
@@ -563,24 +570,30 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
                              : qrope + 2 * ((int64_t)h * a.qr_sh + (f0 - a.d)));
           }
         };
-        uint4 vc[kQC], vn[kQC];
-        if (cw < P.N1) load_row(cw, vc);
+        uint4 v[kQD + 1][kQC];
+#pragma unroll
+        for (int i = 0; i < kQD; ++i)
+          if (cw + kConvWarps * i < P.N1) load_row(cw + kConvWarps * i, v[i]);
 #pragma unroll 1
         for (int h = cw; h < P.N1; h += kConvWarps) {
-          if (h + kConvWarps < P.N1) load_row(h + kConvWarps, vn);
+          if (h + kConvWarps * kQD < P.N1) load_row(h + kConvWarps * kQD, v[kQD]);
           float f[kQC][8];
           float mx = 0.f;
 #pragma unroll
           for (int j = 0; j < kQC; ++j) {
-            load8_bits(vc[j], P.qdtype, f[j]);
+            load8_bits(v[0][j], P.qdtype, f[j]);
 #pragma unroll
             for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[j][e]));
           }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          const int e = (mx > 0.f && isfinite(mx)) ? 14 - ilogbf(mx) : 0;
-          const float qscale = ldexpf(1.f, e);
-          if (lane == 0) m->qs_inv[c.piece & 1][h] = ldexpf(1.f, -e);
+          // e = 14 - floor(log2 max |q|) from the exponent field (a subnormal max counts as
+          // 2^-126), at most 126 so that 2^e and 2^-e are normal floats
+          int e = 0;
+          if (mx > 0.f && isfinite(mx))
+            e = min(14 - (max((__float_as_int(mx) >> 23) & 0xff, 1) - 127), 126);
+          const float qscale = __int_as_float((127 + e) << 23);
+          if (lane == 0) m->qs_inv[c.piece & 1][h] = __int_as_float((127 - e) << 23);
 #pragma unroll
           for (int j = 0; j < kQC; ++j) {
             const int fc = lane + 32 * j;
@@ -594,7 +607,9 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
             *reinterpret_cast<uint4*>(q_s + at * (P.N1 * 128) + h * 128 + ((jj ^ (h & 7)) << 4)) = o;
           }
 #pragma unroll
-          for (int j = 0; j < kQC; ++j) vc[j] = vn[j];
+          for (int i = 0; i < kQD; ++i)
+#pragma unroll
+            for (int j = 0; j < kQC; ++j) v[i][j] = v[i + 1][j];
         }
         fence_proxy_async_smem();
         named_sync(2, kConvThreads);   // every warp's rows written before q_full
@@ -610,26 +625,46 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         // 4(cq%2) + 2ch + {0, 1} of every token row; it converts them and later transposes them
         const bool owns = (cq >> 1) < nat;
         if constexpr (BITS == 16) {
+          // In place, 16-bit codes -> f16, in one pass through registers: each 8x8 block
+          // (8 tokens x 8 features) is loaded transposed, converted element by element, stored
+          // back transposed (row-major again, for the score MMAs) and the same registers, now
+          // feature-major, go to C^T in TMEM (lanes fb .. fb+15 of latent group p).  The slot
+          // is not read after q_full, so only the score MMAs release it.
           fail = fail || !mbar_wait(&b_tfull[s], ph, abort, kLimitNs);
-          if (!fail && owns) {
-            uint8_t* atom = pair + (cq >> 1) * kAtom;
-            // in place: 16-bit codes -> f16; every load issued before the first store
-            uint4* q4[4];
-            uint4 v[4];
+          uint32_t cv[16];
+          const bool go = !fail && owns;
+          if (go) {
+            const uint32_t abase = smem_u32(pair + (cq >> 1) * kAtom);
+            const int mi = lane >> 3, r8 = lane & 7;
+            const int cc = 4 * (cq & 1) + 2 * ch + (mi >> 1);
+            uint32_t ad[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int r = conv_row(lane, k), cc = 4 * (cq & 1) + 2 * ch + (lane & 1);
-              q4[k] = reinterpret_cast<uint4*>(atom + r * 128 + ((cc ^ (r & 7)) << 4));
-              v[k] = *q4[k];
+            for (int tg = 0; tg < 4; ++tg) {
+              const int tok = 16 * tg + 8 * (mi & 1) + r8;
+              ad[tg] = abase + tok * 128 + ((cc ^ r8) << 4);
+              uint32_t d4[4];
+              ldsm_x4_trans(ad[tg], d4);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) cv[4 * tg + i] = d4[i];
             }
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              v[k].x = cvt_code16(v[k].x);
-              v[k].y = cvt_code16(v[k].y);
-              v[k].z = cvt_code16(v[k].z);
-              v[k].w = cvt_code16(v[k].w);
-              *q4[k] = v[k];
+            for (int i = 0; i < 16; ++i) cv[i] = cvt_code16(cv[i]);
+#pragma unroll
+            for (int tg = 0; tg < 4; ++tg) {
+              const uint32_t d4[4] = {cv[4 * tg], cv[4 * tg + 1], cv[4 * tg + 2], cv[4 * tg + 3]};
+              stsm_x4_trans(ad[tg], d4);
             }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b_pfull[s]);
+          if (p < P.NPd) {
+            if (p == 0) {   // the output MMAs of tile - 2 have finished reading this buffer
+              fail = fail || !mbar_wait(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u,
+                                        abort, kLimitNs);
+              tc_fence_after();
+            }
+            if (go) tmem_st16x256b_x4(tmem + ((uint32_t)fb << 16) + kCtCol0 + 128u * ctb + 32u * p, cv);
           }
         } else {
           const uint32_t rs = rr.slot, rph = rr.phase;
@@ -639,36 +674,36 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           __syncwarp();
           if (lane == 0) mbar_arrive(&b_rempty[rs]);
           rr.next(P.RR);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&b_pfull[s]);
-        if (p < P.NPd) {
-          // transpose this warp's 16 features x 64 tokens into C^T (TMEM lanes fb .. fb+15
-          // of latent group p): four 16-token blocks
-          if (p == 0) {   // the output MMAs of tile - 2 have finished reading this buffer
-            fail = fail || !mbar_wait(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u, abort,
-                                      kLimitNs);
-            tc_fence_after();
-          }
-          if (!fail && owns) {
-            const uint32_t abase = smem_u32(pair + (cq >> 1) * kAtom);
-            const int mi = lane >> 3, r8 = lane & 7;
-            const int cc = 4 * (cq & 1) + 2 * ch + (mi >> 1);
-            uint32_t rr[16];
-#pragma unroll
-            for (int tg = 0; tg < 4; ++tg) {
-              const int tok = 16 * tg + 8 * (mi & 1) + r8;
-              uint32_t d4[4];
-              ldsm_x4_trans(abase + tok * 128 + ((cc ^ (tok & 7)) << 4), d4);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) rr[4 * tg + i] = d4[i];
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b_pfull[s]);
+          if (p < P.NPd) {
+            // transpose this warp's 16 features x 64 tokens into C^T (TMEM lanes fb .. fb+15
+            // of latent group p): four 16-token blocks
+            if (p == 0) {   // the output MMAs of tile - 2 have finished reading this buffer
+              fail = fail || !mbar_wait(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u, abort,
+                                        kLimitNs);
+              tc_fence_after();
             }
-            tmem_st16x256b_x4(tmem + ((uint32_t)fb << 16) + kCtCol0 + 128u * ctb + 32u * p, rr);
+            if (!fail && owns) {
+              const uint32_t abase = smem_u32(pair + (cq >> 1) * kAtom);
+              const int mi = lane >> 3, r8 = lane & 7;
+              const int cc = 4 * (cq & 1) + 2 * ch + (mi >> 1);
+              uint32_t rr[16];
+#pragma unroll
+              for (int tg = 0; tg < 4; ++tg) {
+                const int tok = 16 * tg + 8 * (mi & 1) + r8;
+                uint32_t d4[4];
+                ldsm_x4_trans(abase + tok * 128 + ((cc ^ (tok & 7)) << 4), d4);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) rr[4 * tg + i] = d4[i];
+              }
+              tmem_st16x256b_x4(tmem + ((uint32_t)fb << 16) + kCtCol0 + 128u * ctb + 32u * p, rr);
+            }
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b_pempty[s]);   // this warp is done reading the slot
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&b_pempty[s]);   // this warp is done reading the slot
         pr.next(P.PR);
       }
       tmem_wait_st();

@@ -16,6 +16,9 @@ namespace kvk {
 constexpr int kMaxRowElems = 2048;      // d + d_rope handled by the write kernel
 constexpr size_t kArenaHeader = 256;    // status flags live in the first bytes of the arena
 constexpr int kTcTileTokens = 64;       // tokens per tile of the tensor-core decode
+// Work-split cost of one piece on the tensor-core decode, in tokens: query staging and the
+// pipeline refill at a sequence boundary take about as long as 2.5 tiles.
+constexpr int kTcPieceCost = 160;
 
 struct AnchorDesc {
   int layer = 0;
@@ -76,6 +79,7 @@ struct DecodeArgs {
   float* ws_ml;              // [slots][H][2]  (running max in log2 units, sum of weights)
   float* ws_o;               // [slots][H][d]  (un-normalised weighted sums)
   int G;                     // CTAs the flattened tokens are split over
+  int split_x;               // cost of a piece in tokens (split_cost / split_token)
   uint32_t* flags;
 };
 
@@ -112,13 +116,31 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, const AnchorDesc& A, int dtype
 bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H, bool has_keep);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
 
-// Position -> CTA of the balanced split: CTA c owns [c*N/G, (c+1)*N/G).
-__host__ __device__ inline int cta_of(int64_t x, int64_t N, int G) {
-  int64_t c = ((x + 1) * (int64_t)G + N - 1) / N - 1;
+// Work split of the flattened tokens over G CTAs.  Sequence i occupies the cost range
+// [off[i] + X i, off[i+1] + X (i+1)): X units standing for the fixed cost of a piece (query
+// staging, partial write-back), then one unit per token; C = N + X batch in all.  CTA c owns
+// the cost range [split_cost(c), split_cost(c+1)), i.e. the tokens t of sequence i whose cost
+// position t + X (i + 1) lies in it: a CTA that takes the start of a sequence takes fewer
+// tokens.  X = 0 is the plain even split of the tokens.
+__host__ __device__ inline int64_t split_cost(int c, int64_t C, int G) {
+  return ((int64_t)c * C) / G;
+}
+// The CTA whose cost range holds position u (the largest c with split_cost(c) <= u).
+__host__ __device__ inline int split_cta(int64_t u, int64_t C, int G) {
+  int64_t c = ((u + 1) * (int64_t)G + C - 1) / C - 1;
   return (int)(c < 0 ? 0 : (c >= G ? G - 1 : c));
 }
-__host__ __device__ inline int64_t cta_lo(int c, int64_t N, int G) {
-  return ((int64_t)c * N) / G;
+// First token whose cost position is >= u (N when there is none); off has batch + 1 entries.
+__host__ __device__ inline int64_t split_token(const int32_t* off, int batch, int X, int64_t u) {
+  int L = 0, H = batch;   // the last i with off[i] + X i <= u
+  while (L < H) {
+    const int mid = (L + H + 1) >> 1;
+    if (off[mid] + (int64_t)X * mid <= u) L = mid; else H = mid - 1;
+  }
+  if (L >= batch) return off[batch];
+  const int64_t len = off[L + 1] - off[L];
+  const int64_t into = u - (off[L] + (int64_t)X * L) - X;   // tokens of sequence L before u
+  return off[L] + (into < 0 ? 0 : (into > len ? len : into));
 }
 
 }  // namespace kvk

@@ -42,15 +42,23 @@ __global__ void __launch_bounds__(kMergeThreads, 4) merge_kernel(DecodeArgs a) {
   __shared__ float w_s[kChunk];
   __shared__ float red[kMergeThreads / 32];
   const int i = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
-  const int64_t N = a.seq_off[a.batch];
+  const int64_t C = a.seq_off[a.batch] + (int64_t)a.split_x * a.batch;
   const int64_t s0 = a.seq_off[i], s1 = a.seq_off[i + 1];
   float* out = a.out + ((int64_t)i * a.H + h) * a.d;
   int c0 = 0, np = 0;
-  if (s1 > s0) {
-    c0 = cta_of(s0, N, a.G);
-    np = cta_of(s1 - 1, N, a.G) - c0 + 1;
+  if (s1 > s0) {   // token t of sequence i sits at cost position t + X (i + 1)
+    const int64_t u = (int64_t)a.split_x * (i + 1);
+    c0 = split_cta(s0 + u, C, a.G);
+    np = split_cta(s1 - 1 + u, C, a.G) - c0 + 1;
   }
+  // CTAs c0 .. c0 + np - 1 hold the pieces; with fewer cost units than CTAs some of them own
+  // nothing and wrote no partials (their slots are skipped)
+  const bool dense = C >= a.G;
+  auto live = [&](int k) {
+    return dense || split_cost(c0 + k + 1, C, a.G) > split_cost(c0 + k, C, a.G);
+  };
   auto ml = [&](int k) -> float2 {   // (m, l) of piece k of this sequence and head
+    if (!live(k)) return make_float2(0.f, 0.f);
     const int64_t sh = (int64_t)(c0 + k + i) * a.H + h;
     return *reinterpret_cast<const float2*>(a.ws_ml + 2 * sh);
   };
@@ -67,7 +75,7 @@ __global__ void __launch_bounds__(kMergeThreads, 4) merge_kernel(DecodeArgs a) {
     for (int k = 0; k < kFew; ++k) {
       mlv[k] = make_float2(0.f, 0.f);
       ov[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (k < np) {
+      if (k < np && live(k)) {
         mlv[k] = ml(k);
         if (tid < d4) ov[k] = src[k * stride];
       }

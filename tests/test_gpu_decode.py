@@ -169,6 +169,50 @@ def test_split_count_invariance_and_paths_agree(pkg, oracle_mod):
         case.close()
 
 
+def test_short_sequences_many_ctas_poisoned_workspace(pkg, oracle_mod):
+    """Far fewer tokens than CTAs (CTAs that own nothing write no partials) with a workspace
+    full of NaN bytes: the merge takes exactly the CTAs that hold a piece of each sequence,
+    on both kernels and for several CTA counts."""
+    d, r, dR, H, B, T = 512, 512, 64, 40, 4, 4096
+    case = Case(pkg, d, 16, r, dR, B, T)
+    try:
+        c = _rand((B, T, r), 41, torch.bfloat16)
+        kr = _rand((B, T, dR), 42, torch.bfloat16)
+        case.write(c, kr)
+        ql, qr = _rand((B, H, r), 43, torch.bfloat16), _rand((B, H, dR), 44, torch.bfloat16)
+        lens = [3, 0, 70, 1]
+        lens_t = torch.tensor(lens, dtype=torch.int32)
+        sigma = 1 / math.sqrt(d + dR)
+        ref_cache = oracle_cache(oracle_mod, c, kr, d, 16)
+        refs = {}
+        for i in range(B):
+            if lens[i]:
+                k, s_, _ = ref_cache[i]
+                refs[i] = oracle_decode(oracle_mod, (k[:lens[i]], s_[:lens[i]], None),
+                                        bf16_or_f32_to_np(ql[i]), bf16_or_f32_to_np(qr[i]), d,
+                                        sigma)
+        lay = case.lay
+        for path in _paths(pkg, case, torch.bfloat16, H):
+            for ctas in (0, 37, 1000):
+                lay.set_decode_path(path)
+                lay.set_decode_ctas(ctas)
+                ws = torch.full((lay.workspace_bytes(0, B, H),), 255, dtype=torch.uint8,
+                                device="cuda")
+                lse = torch.empty(B, H, dtype=torch.float32, device="cuda")
+                out = lay.mla_decode(0, ql.cuda(), qr.cuda(), lens_t.cuda(), sigma, lse=lse,
+                                     workspace=ws)
+                torch.cuda.synchronize()
+                out, lse = out.cpu().numpy(), lse.cpu().numpy()
+                assert not out[1].any() and np.all(np.isneginf(lse[1])), (path, ctas)
+                for i, (o_ref, l_ref) in refs.items():
+                    check_outputs(out[i], lse[i], o_ref, l_ref, f"path {path} ctas {ctas} seq {i}")
+        lay.set_decode_ctas(0)
+        lay.set_decode_path(0)
+        assert lay.read_status() == 0
+    finally:
+        case.close()
+
+
 def test_keep_list_equals_compacted_cache(pkg, oracle_mod):
     d, r, dR, H, B, T = 256, 512, 64, 40, 3, 3000
     case = Case(pkg, d, 8, r, dR, B, T)
