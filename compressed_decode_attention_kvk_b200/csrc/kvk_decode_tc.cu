@@ -733,7 +733,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
 
     float l[2 * NB];    // partial weight sums of this thread's heads
     float mr[2 * NB];   // reference max of this thread's heads (log2 units)
-    const float* qsi = nullptr;   // 2^-e_h of the current piece's heads (shared memory)
+    float qh[2 * NB];   // 2^-e_h of this thread's heads 8j + hc + {0, 1} in the current piece
     int pt = 0;
     Cursor c;
     cursor_start(c, seq0, off, a.batch, lo, hi);
@@ -761,7 +761,10 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       }
       if (c.first) {
         fail = fail || !mbar_wait(b_qfull, (uint32_t)c.piece & 1u, abort, kLimitNs);
-        qsi = m->qs_inv[c.piece & 1] + hc;
+#pragma unroll
+        for (int j = 0; j < NB; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) qh[2 * j + e] = m->qs_inv[c.piece & 1][8 * j + hc + e];
         __syncwarp();
         if (lane == 0) mbar_arrive(b_qseen);
 #pragma unroll
@@ -810,9 +813,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const bool hv = (8 * j + hc + e) < a.H;
-          const float qh = qsi[8 * j + e];
-          x[4 * j + e] = (va && hv) ? x[4 * j + e] * qh * ca : -INFINITY;
-          x[4 * j + 2 + e] = (vb && hv) ? x[4 * j + 2 + e] * qh * cbf : -INFINITY;
+          x[4 * j + e] = (va && hv) ? x[4 * j + e] * qh[2 * j + e] * ca : -INFINITY;
+          x[4 * j + 2 + e] = (vb && hv) ? x[4 * j + 2 + e] * qh[2 * j + e] * cbf : -INFINITY;
           mine = mine || (x[4 * j + e] > mr[2 * j + e] + 8.f) ||
                  (x[4 * j + 2 + e] > mr[2 * j + e] + 8.f);
         }
@@ -908,10 +910,11 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           float ea[2], eb[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const float m0 = mr[2 * j + e];
-            const float xa = x[4 * j + e], xb = x[4 * j + 2 + e];
-            ea[e] = (xa == -INFINITY || m0 == -INFINITY) ? 0.f : exp2f(xa - m0);
-            eb[e] = (xb == -INFINITY || m0 == -INFINITY) ? 0.f : exp2f(xb - m0);
+            // a head whose reference is still -inf has only -inf scores so far (any finite
+            // score takes the slow path), so a finite stand-in gives 2^-inf = 0 without NaN
+            const float m0 = (mr[2 * j + e] == -INFINITY) ? 0.f : mr[2 * j + e];
+            ea[e] = ex2_approx(x[4 * j + e] - m0);
+            eb[e] = ex2_approx(x[4 * j + 2 + e] - m0);
             l[2 * j + e] += ea[e] + eb[e];
           }
           *reinterpret_cast<uint32_t*>(pa + 128 * j) = h2_bits(__floats2half2_rn(ea[0] * wa, ea[1] * wa));

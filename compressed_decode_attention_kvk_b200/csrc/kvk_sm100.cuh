@@ -422,6 +422,13 @@ __device__ __forceinline__ bool named_or(uint32_t id, uint32_t n, bool pred) {
       : "memory");
   return r != 0;
 }
+// 2^x by the special-function unit (PTX ex2.approx.ftz.f32: relative error about 2^-22,
+// 2^-inf = +0, subnormal results flushed to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
