@@ -202,18 +202,39 @@ class DecodeWorkload:
                     for l in self.anchors}
         self.q = {l: workloads.queries(w, l, self.B, device=device) for l in range(w.n_layers)}
         self.lens = torch.full((self.B,), self.T, dtype=torch.int32, device=device)
+        # eviction workloads: one sorted keep list per sequence, shared by all layers
+        self.keep = self.keep_len = None
+        self.n_read = self.T
+        if w.keep:
+            self.keep = workloads.keep_lists(w, self.B, self.T, w.keep, device=device)
+            self.keep_len = torch.full((self.B,), w.keep, dtype=torch.int32, device=device)
+            self.n_read = w.keep
         self.sigma = {l: workloads.softmax_scale(t["d"][t["anchor"][l]], w.d_rope)
                       for l in range(w.n_layers)}
         self.out = {l: torch.empty(self.B, self.H, t["d"][t["anchor"][l]], dtype=torch.float32,
                                    device=device) for l in range(w.n_layers)}
-        wsb = max(self.lay.workspace_bytes(l, self.B, self.H) for l in range(w.n_layers))
+        ks = w.keep if w.keep else None
+        wsb = max(self.lay.workspace_bytes(l, self.B, self.H, keep_stride=ks)
+                  for l in range(w.n_layers))
         self.ws = torch.empty(wsb, dtype=torch.uint8, device=device)
         self.bytes_per_layer = []
         for l in range(w.n_layers):
             info = self.lay.layer_info(l)
-            self.bytes_per_layer.append(self.B * self.T * (info["row_bytes"] + 2))
+            # rows read (the kept ones with a keep list) and their scales, plus 4 B per index
+            self.bytes_per_layer.append(self.B * self.n_read * (info["row_bytes"] + 2) +
+                                        (4 * self.B * w.keep if w.keep else 0))
         self.decode_bytes = sum(self.bytes_per_layer)
-        self.launches_per_step = 1 + 2 * w.n_layers   # one append launch for every anchor
+        mx = max(self.bytes_per_layer)
+        self.l2_note = ("inputs larger than L2 (per-layer cache > 126 MB)" if not w.keep else
+                        f"kept rows {mx / 1e6:.1f} MB per layer (< 126 MB L2), gathered from a "
+                        f"{self.B * self.T * max(self.lay.layer_info(l)['row_bytes'] + 2 for l in range(w.n_layers)) / 1e6:.0f} MB "
+                        "cache: a layer that inherits the previous layer's anchor may find them in L2")
+        # one append launch for every anchor; per layer split decode + merge, and with a keep
+        # list on the tensor-core kernel the compaction of the kept rows
+        per_layer = 2
+        if w.keep and self.lay.decode_path_for(0, self.q[0][0].dtype, self.H, True) == 1:
+            per_layer = 3
+        self.launches_per_step = 1 + per_layer * w.n_layers
 
     def step(self, events=None):
         from compressed_decode_attention_kvk_b200 import kvk
@@ -225,7 +246,8 @@ class DecodeWorkload:
             ql, qr = self.q[l]
             if events is not None:
                 events[l][0].record()
-            kvk.kvk_mla_decode(h, l, ql, qr, self.lens, self.sigma[l], self.out[l], self.ws)
+            kvk.kvk_mla_decode(h, l, ql, qr, self.lens, self.sigma[l], self.out[l], self.ws,
+                               keep_idx=self.keep, keep_len=self.keep_len)
             if events is not None:
                 events[l][1].record()
 
@@ -319,7 +341,7 @@ def run_kvk(args, rank, world, local, pg):
                        "d_rope": wl.w.d_rope, "batch": wl.B, "tokens": wl.T,
                        "bits_per_token": wl.lay.bits_per_token,
                        "decode_bytes_per_step": wl.decode_bytes,
-                       "l2": "inputs larger than L2 (per-layer cache > 126 MB)",
+                       "l2": wl.l2_note,
                        "graph": bool(graph), "parallelism": f"replicas x{world}"},
             "roofline": roof, "e2e": e2e, "cpu_baseline": cpu,
             "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks,
@@ -344,8 +366,16 @@ def run_e2e(args, wl, device, pg):
                                                 b.numel() * b.element_size()
                                                 for a, b in h_q.values())
     d2h = sum(o.numel() * o.element_size() for o in h_out.values())
+    # a keep list is a per-step input too (eviction decisions change from step to step)
+    h_keep = d_keep = None
+    if wl.keep is not None:
+        h_keep = wl.keep.cpu().pin_memory()
+        d_keep = torch.empty_like(wl.keep)
+        h2d += h_keep.numel() * h_keep.element_size()
 
     def step():
+        if h_keep is not None:
+            d_keep.copy_(h_keep, non_blocking=True)
         for l in wl.anchors:
             dc, dk = d_app[l]
             dc.copy_(h_app[l][0], non_blocking=True)
@@ -356,7 +386,8 @@ def run_e2e(args, wl, device, pg):
             qa, qb = d_q[l]
             qa.copy_(h_q[l][0], non_blocking=True)
             qb.copy_(h_q[l][1], non_blocking=True)
-            kvk.kvk_mla_decode(wl.lay.handle, l, qa, qb, wl.lens, wl.sigma[l], wl.out[l], wl.ws)
+            kvk.kvk_mla_decode(wl.lay.handle, l, qa, qb, wl.lens, wl.sigma[l], wl.out[l], wl.ws,
+                               keep_idx=d_keep, keep_len=wl.keep_len)
             h_out[l].copy_(wl.out[l], non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
@@ -395,6 +426,7 @@ class OracleSampler:
         self.device = device
         self.layer, self.seq = 0, 0
         self._cached = None   # (anchor, latent, rope) of the current anchor
+        self._keep = None     # keep lists of an eviction workload
 
     def _next_unit(self):
         w, t = self.w, self.t
@@ -411,23 +443,27 @@ class OracleSampler:
                                                         kr[seq].float().cpu().numpy(), d, b)
         qln = ql[seq].double().cpu().numpy()
         qrn = qr[seq].double().cpu().numpy()
+        if w.keep and self._keep is None:
+            self._keep = workloads.keep_lists(w, w.batch, w.tokens, w.keep).numpy()
+        tok = self._keep[seq] if w.keep else None
         self.seq += 1
         if self.seq == w.batch:
             self.seq = 0
             self.layer = (self.layer + 1) % w.n_layers
-        return layer, d, (qln, qrn, codes, scales, rows.shape[1])
+        return layer, d, (qln, qrn, codes, scales, rows.shape[1], tok)
 
     def run(self, budget_s, min_units=1):
         """Decode units until `budget_s` seconds of timed oracle work (at least `min_units`).
         Returns (algorithmic bytes, seconds, units, layers touched)."""
         nbytes, dt, units, layers = 0, 0.0, 0, set()
         while dt < budget_s or units < min_units:
-            layer, d, (ql, qr, codes, scales, row_bytes) = self._next_unit()
+            layer, d, (ql, qr, codes, scales, row_bytes, tok) = self._next_unit()
             sigma = workloads.softmax_scale(d, self.w.d_rope)
             t0 = time.perf_counter()
-            self.oracle.decode_sequence(ql, qr, codes, scales, d, sigma)
+            self.oracle.decode_sequence(ql, qr, codes, scales, d, sigma, tok)
             dt += time.perf_counter() - t0
-            nbytes += codes.shape[0] * (row_bytes + 2)
+            nbytes += (codes.shape[0] * (row_bytes + 2) if tok is None
+                       else len(tok) * (row_bytes + 6))
             units += 1
             layers.add(layer)
         return nbytes, dt, units, layers

@@ -308,10 +308,11 @@ kvk_status kvk_quant_write_layers(kvk_layout* L, int n, const int32_t* layers,
   return e == cudaSuccess ? KVK_OK : KVK_ERR_CUDA;
 }
 
-static int choose_path(const kvk_layout* L, const AnchorDesc& A, int dtype, int H,
-                       bool has_keep) {
+// The kernel a call takes (a keep list does not change it: the tensor-core kernel then
+// reads a compacted copy of the kept rows, given workspace for it).
+static int choose_path(const kvk_layout* L, const AnchorDesc& A, int dtype, int H) {
   if (L->path == KVK_PATH_CUDA_CORE) return KVK_PATH_CUDA_CORE;
-  bool tc = kvk::tc_supported(L, A, dtype, H, has_keep);
+  bool tc = kvk::tc_supported(L, A, dtype, H);
   if (L->path == KVK_PATH_TENSOR) return tc ? KVK_PATH_TENSOR : -1;
   return tc ? KVK_PATH_TENSOR : KVK_PATH_CUDA_CORE;
 }
@@ -328,11 +329,23 @@ kvk_status kvk_decode_workspace_bytes(const kvk_layout* L, int layer, int batch,
   return KVK_OK;
 }
 
+kvk_status kvk_decode_workspace_bytes_keep(const kvk_layout* L, int layer, int batch,
+                                           int n_heads, int keep_stride, size_t* bytes) {
+  if (keep_stride < 0) return KVK_ERR_INVALID_ARG;
+  size_t base = 0;
+  kvk_status st = kvk_decode_workspace_bytes(L, layer, batch, n_heads, &base);
+  if (st != KVK_OK) return st;
+  const AnchorDesc& A = L->anchors[L->slot[layer]];
+  *bytes = align_up(base, kAlign) + kvk::compact_workspace_bytes(batch, keep_stride, A.row_bytes);
+  return KVK_OK;
+}
+
 kvk_status kvk_decode_path_for(const kvk_layout* L, int layer, int dtype, int n_heads,
                                int has_keep, int* path) {
   if (!L || !path || layer < 0 || layer >= L->n_layers || n_heads < 1) return KVK_ERR_INVALID_ARG;
   if (dtype != KVK_F32 && dtype != KVK_BF16 && dtype != KVK_F16) return KVK_ERR_INVALID_ARG;
-  int p = choose_path(L, L->anchors[L->slot[layer]], dtype, n_heads, has_keep != 0);
+  (void)has_keep;
+  int p = choose_path(L, L->anchors[L->slot[layer]], dtype, n_heads);
   if (p < 0) return KVK_ERR_UNSUPPORTED;
   *path = p;
   return KVK_OK;
@@ -366,8 +379,30 @@ kvk_status kvk_mla_decode(kvk_layout* L, int layer, const void* q_lat, const voi
       q_rope_stride_head % 8)
     return KVK_ERR_ALIGNMENT;
   const AnchorDesc& A = L->anchors[L->slot[layer]];
-  int path = choose_path(L, A, dtype, n_heads, dev_keep_idx != nullptr);
+  int path = choose_path(L, A, dtype, n_heads);
   if (path < 0) return KVK_ERR_UNSUPPORTED;
+  // With a keep list the tensor-core kernel reads a dense copy of the kept rows, placed after
+  // the decode's own workspace; without room for it (or a tensor map over it) the call takes
+  // the CUDA-core kernel, unless the tensor-core kernel was asked for.
+  const bool keep = dev_keep_idx != nullptr;
+  CUtensorMap keep_tmap;
+  size_t keep_off = 0;
+  if (keep && path == KVK_PATH_TENSOR) {
+    const int Gt = kvk::decode_ctas(L, batch, KVK_PATH_TENSOR);
+    keep_off = align_up(kvk::decode_workspace(batch, n_heads, A.d, Gt, nullptr, nullptr), kAlign);
+    const bool room =
+        workspace_bytes >= keep_off + kvk::compact_workspace_bytes(batch, keep_stride, A.row_bytes);
+    kvk::CompactArgs probe;
+    if (room) kvk::compact_carve(static_cast<uint8_t*>(workspace) + keep_off, batch, keep_stride,
+                                 A.row_bytes, &probe);
+    const bool ok = room && keep_stride > 0 &&
+                    make_codes_tmap(&keep_tmap, probe.dst_codes, (int64_t)batch * keep_stride,
+                                    A.row_bytes, A.b, kvk::kTcTileTokens);
+    if (!ok) {
+      if (L->path == KVK_PATH_TENSOR) return room ? KVK_ERR_UNSUPPORTED : KVK_ERR_WORKSPACE;
+      path = KVK_PATH_CUDA_CORE;
+    }
+  }
 
   kvk::DecodeArgs a;
   memset(&a, 0, sizeof(a));
@@ -401,9 +436,36 @@ kvk_status kvk_mla_decode(kvk_layout* L, int layer, const void* q_lat, const voi
   a.split_x = (path == KVK_PATH_TENSOR) ? kvk::kTcPieceCost : 0;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = (path == KVK_PATH_TENSOR)
-                      ? kvk::launch_decode_tc(a, A, dtype, L->num_sms, st)
-                      : kvk::launch_decode_fma(a, dtype, st);
+  cudaError_t e = cudaSuccess;
+  if (path == KVK_PATH_TENSOR && keep) {
+    kvk::CompactArgs c;
+    memset(&c, 0, sizeof(c));
+    c.codes = a.codes;
+    c.scales = a.scales;
+    c.row_bytes = A.row_bytes;
+    c.max_tokens = L->max_tokens;
+    c.seq_lens = dev_seq_lens;
+    c.keep_idx = dev_keep_idx;
+    c.keep_len = dev_keep_len;
+    c.keep_stride = keep_stride;
+    c.flags = a.flags;
+    kvk::compact_carve(static_cast<uint8_t*>(workspace) + keep_off, batch, keep_stride,
+                       A.row_bytes, &c);
+    e = kvk::launch_compact(c, batch, st);
+    // the decode proper: the dense copy as a cache of keep_stride rows per sequence
+    a.codes = c.dst_codes;
+    a.scales = c.dst_scales;
+    a.max_tokens = keep_stride;
+    a.seq_lens = c.cnt;
+    a.keep_idx = nullptr;
+    a.keep_len = nullptr;
+    a.keep_stride = 0;
+    if (e == cudaSuccess) e = kvk::launch_decode_tc(a, keep_tmap, dtype, st);
+  } else if (path == KVK_PATH_TENSOR) {
+    e = kvk::launch_decode_tc(a, A.tmap_tile, dtype, st);
+  } else {
+    e = kvk::launch_decode_fma(a, dtype, st);
+  }
   if (e == cudaSuccess) e = kvk::launch_merge(a, st);
   return e == cudaSuccess ? KVK_OK : KVK_ERR_CUDA;
 }

@@ -1116,24 +1116,24 @@ cudaError_t launch_bits(const TcParams& P, const CUtensorMap& tmap, size_t smem,
 
 }  // namespace
 
-bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H, bool has_keep) {
+bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H) {
   if (dtype != KVK_BF16 && dtype != KVK_F16) return false;
-  if (has_keep || !A.tmap_ok) return false;
+  if (!A.tmap_ok) return false;
   const Plan pl = make_plan(A.d, L->d_rope, A.b, H, L->max_batch);
   return pl.ok && launch_regs_ok(A.b, pl.p.N2);
 }
 
-cudaError_t launch_decode_tc(const DecodeArgs& a, const AnchorDesc& A, int dtype, int,
+cudaError_t launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tmap, int dtype,
                              cudaStream_t st) {
   Plan pl = make_plan(a.d, a.d_rope, a.b, a.H, a.batch);
   if (!pl.ok) return cudaErrorInvalidValue;
   pl.p.a = a;
   pl.p.qdtype = dtype;
   switch (a.b) {
-    case 16: return launch_bits<16>(pl.p, A.tmap_tile, pl.smem, a.G, st);
-    case 8: return launch_bits<8>(pl.p, A.tmap_tile, pl.smem, a.G, st);
-    case 4: return launch_bits<4>(pl.p, A.tmap_tile, pl.smem, a.G, st);
-    case 2: return launch_bits<2>(pl.p, A.tmap_tile, pl.smem, a.G, st);
+    case 16: return launch_bits<16>(pl.p, tmap, pl.smem, a.G, st);
+    case 8: return launch_bits<8>(pl.p, tmap, pl.smem, a.G, st);
+    case 4: return launch_bits<4>(pl.p, tmap, pl.smem, a.G, st);
+    case 2: return launch_bits<2>(pl.p, tmap, pl.smem, a.G, st);
   }
   return cudaErrorInvalidValue;
 }

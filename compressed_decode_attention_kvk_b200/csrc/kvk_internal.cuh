@@ -111,9 +111,32 @@ cudaError_t launch_quant_write_layers(const kvk_layout* L, const QuantLayers& Q,
                                       int batch, const int32_t* start_pos, int n_new,
                                       cudaStream_t stream);
 cudaError_t launch_decode_fma(const DecodeArgs& a, int dtype, cudaStream_t stream);
-cudaError_t launch_decode_tc(const DecodeArgs& a, const AnchorDesc& A, int dtype, int num_sms,
+// tmap: the codes plane the kernel streams (the anchor's, or a compacted keep-list copy)
+cudaError_t launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tmap, int dtype,
                              cudaStream_t stream);
-bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H, bool has_keep);
+bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H);
+
+inline size_t align_up_sz(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Keep-list compaction ahead of the tensor-core decode (kvk_compact.cu): the kept rows and
+// scales of sequence i go, in keep order and without invalid entries, to rows
+// [i * keep_stride, i * keep_stride + cnt[i]) of a dense scratch cache.
+struct CompactArgs {
+  const uint8_t* codes;      // anchor's codes plane [max_batch * max_tokens][row_bytes]
+  const __half* scales;      // anchor's scale plane
+  int row_bytes, max_tokens;
+  const int32_t* seq_lens;
+  const int32_t* keep_idx;   // [batch][keep_stride]
+  const int32_t* keep_len;
+  int keep_stride;
+  int32_t* cnt;              // [batch] valid kept entries per sequence (written)
+  uint8_t* dst_codes;        // [batch * keep_stride][row_bytes]
+  __half* dst_scales;        // [batch * keep_stride] (+ slack for the decode's scale windows)
+  uint32_t* flags;
+};
+size_t compact_workspace_bytes(int batch, int keep_stride, int row_bytes);
+void compact_carve(void* base, int batch, int keep_stride, int row_bytes, CompactArgs* c);
+cudaError_t launch_compact(const CompactArgs& c, int batch, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
 
 // Work split of the flattened tokens over G CTAs.  Sequence i occupies the cost range

@@ -32,7 +32,8 @@ _DTYPE = {torch.float32: KVK_F32, torch.bfloat16: KVK_BF16, torch.float16: KVK_F
 EXPORTED = ("kvk_create_layout", "kvk_destroy", "kvk_get_layer_info", "kvk_quant_write",
             "kvk_decode_workspace_bytes", "kvk_mla_decode", "kvk_read_status",
             "kvk_set_decode_path", "kvk_set_decode_ctas", "kvk_decode_path_for",
-            "kvk_status_string", "kvk_mla_decode_noalloc", "kvk_quant_write_layers")
+            "kvk_status_string", "kvk_mla_decode_noalloc", "kvk_quant_write_layers",
+            "kvk_decode_workspace_bytes_keep")
 
 # size of the library's built-in scratch array used by kvk_mla_decode_noalloc
 KVK_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -71,6 +72,7 @@ def _lib_handle():
         L.kvk_quant_write.argtypes = [P, i32, P, i32, i64, i64, P, i64, i64, i32, P, i32, P]
         L.kvk_quant_write_layers.argtypes = [P, i32, P, P, i32, P, P, P, P, P, i32, P, i32, P]
         L.kvk_decode_workspace_bytes.argtypes = [P, i32, i32, i32, P]
+        L.kvk_decode_workspace_bytes_keep.argtypes = [P, i32, i32, i32, i32, P]
         L.kvk_mla_decode.argtypes = [P, i32, P, P, i32, i64, i64, i64, i64, i32, i32, P, P, P,
                                      i32, ctypes.c_float, P, P, P, sz, P]
         L.kvk_mla_decode_noalloc.argtypes = [P, i32, P, P, i32, i64, i64, i64, i64, i32, i32,
@@ -197,6 +199,14 @@ def kvk_decode_workspace_bytes(handle, layer, batch, n_heads) -> int:
     _check("kvk_decode_workspace_bytes",
            _lib_handle().kvk_decode_workspace_bytes(handle, layer, batch, n_heads,
                                                     ctypes.byref(out)))
+    return out.value
+
+
+def kvk_decode_workspace_bytes_keep(handle, layer, batch, n_heads, keep_stride) -> int:
+    out = ctypes.c_size_t(0)
+    _check("kvk_decode_workspace_bytes_keep",
+           _lib_handle().kvk_decode_workspace_bytes_keep(handle, layer, batch, n_heads,
+                                                         keep_stride, ctypes.byref(out)))
     return out.value
 
 
@@ -333,12 +343,16 @@ class Layout:
     def quant_write_layers(self, layers, c_kvs, k_ropes, start_pos, stream=None):
         kvk_quant_write_layers(self.handle, layers, c_kvs, k_ropes, start_pos, stream)
 
-    def workspace_bytes(self, layer, batch, n_heads):
-        return kvk_decode_workspace_bytes(self.handle, layer, batch, n_heads)
+    def workspace_bytes(self, layer, batch, n_heads, keep_stride=None):
+        """keep_stride: the row stride of a keep list the calls will pass (None: no keep
+        list), so that such calls can take the tensor-core kernel."""
+        if keep_stride is None:
+            return kvk_decode_workspace_bytes(self.handle, layer, batch, n_heads)
+        return kvk_decode_workspace_bytes_keep(self.handle, layer, batch, n_heads, keep_stride)
 
-    def new_workspace(self, layer, batch, n_heads):
-        return torch.empty(self.workspace_bytes(layer, batch, n_heads), dtype=torch.uint8,
-                           device=self.arena.device)
+    def new_workspace(self, layer, batch, n_heads, keep_stride=None):
+        return torch.empty(self.workspace_bytes(layer, batch, n_heads, keep_stride),
+                           dtype=torch.uint8, device=self.arena.device)
 
     def mla_decode(self, layer, q_lat, q_rope, seq_lens, softmax_scale, out=None, lse=None,
                    workspace=None, keep_idx=None, keep_len=None, stream=None):
@@ -347,7 +361,8 @@ class Layout:
         if out is None:
             out = torch.empty(B, H, d, dtype=torch.float32, device=q_lat.device)
         if workspace is None:
-            workspace = self.new_workspace(layer, B, H)
+            workspace = self.new_workspace(
+                layer, B, H, None if keep_idx is None else keep_idx.stride(0))
         kvk_mla_decode(self.handle, layer, q_lat, q_rope, seq_lens, softmax_scale, out,
                        workspace, lse=lse, keep_idx=keep_idx, keep_len=keep_len, stream=stream)
         return out

@@ -179,6 +179,14 @@ kvk_status kvk_quant_write_layers(kvk_layout* layout, int n, const int32_t* laye
 kvk_status kvk_decode_workspace_bytes(const kvk_layout* layout, int layer, int batch,
                                       int n_heads, size_t* bytes);
 
+/* Bytes of device workspace for a call with a keep list of row stride keep_stride to take
+ * the tensor-core kernel: the bytes above plus a dense copy of the kept rows
+ * (batch * keep_stride * row_bytes of the layer's anchor) and their scales.  With less, such
+ * a call takes the CUDA-core kernel (or returns KVK_ERR_WORKSPACE when the tensor-core
+ * kernel is forced).  keep_stride < 0 is KVK_ERR_INVALID_ARG. */
+kvk_status kvk_decode_workspace_bytes_keep(const kvk_layout* layout, int layer, int batch,
+                                           int n_heads, int keep_stride, size_t* bytes);
+
 /*
  * kvk_mla_decode -- one decode step of attention for one layer over its anchor's cache.
  *
@@ -202,7 +210,11 @@ kvk_status kvk_decode_workspace_bytes(const kvk_layout* layout, int layer, int b
  *   softmax_scale  sigma above
  *   out          device fp32 [batch][n_heads][d], written completely
  *   lse          nullable device fp32 [batch][n_heads] (natural log)
- *   workspace    device, >= kvk_decode_workspace_bytes(); contents are scratch
+ *   workspace    device, >= kvk_decode_workspace_bytes(); contents are scratch.  With a
+ *                keep list and at least kvk_decode_workspace_bytes_keep() bytes, the kept
+ *                rows are first copied densely into the workspace (one extra launch) and the
+ *                tensor-core kernel reads that copy; otherwise the CUDA-core kernel gathers
+ *                them itself.
  */
 kvk_status kvk_mla_decode(kvk_layout* layout, int layer, const void* q_lat, const void* q_rope,
                           int dtype, int64_t q_lat_stride_seq, int64_t q_lat_stride_head,

@@ -135,6 +135,11 @@ def test_planning_layout_cannot_launch(kvk):
         assert lib.kvk_decode_workspace_bytes(handle, 1, 1, 8, ctypes.byref(ws)) == 0
         assert ws.value > 0
         assert lib.kvk_decode_workspace_bytes(handle, 1, 2, 8, ctypes.byref(ws)) == 1  # batch > max
+        wk = ctypes.c_size_t(0)
+        assert lib.kvk_decode_workspace_bytes_keep(handle, 1, 1, 8, 100, ctypes.byref(wk)) == 0
+        assert lib.kvk_decode_workspace_bytes(handle, 1, 1, 8, ctypes.byref(ws)) == 0
+        assert wk.value > ws.value                              # room for the dense kept rows
+        assert lib.kvk_decode_workspace_bytes_keep(handle, 1, 1, 8, -1, ctypes.byref(wk)) == 1
         path = ctypes.c_int(-1)
         assert lib.kvk_decode_path_for(handle, 0, 0, 8, 0, ctypes.byref(path)) == 0
         assert path.value == kvk.KVK_PATH_CUDA_CORE            # fp32 queries

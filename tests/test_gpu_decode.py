@@ -247,16 +247,73 @@ def test_keep_list_equals_compacted_cache(pkg, oracle_mod):
         for i in range(B):
             assert rel_err(kept[i], dense[i]) <= 2e-3
         assert case.lay.read_status() == 0
-        # an index beyond seq_len is skipped and flagged
+        # an index beyond seq_len is skipped and flagged, by both kernels (the tensor-core one
+        # through the dense copy of the kept rows)
         bad = keep_t.clone()
         bad[2, 0] = 39
         bad[2, 1] = 45   # >= seq_len 40
-        out, _ = _decode(case, 0, ql, qr, torch.tensor(lens, dtype=torch.int32), sigma, 2,
-                         keep=bad, keep_len=torch.tensor([400, 312, 2], dtype=torch.int32))
-        assert case.lay.read_status(clear=True) & pkg.KVK_FLAG_KEEP_INDEX
-        o_ref, _ = oracle_decode(oracle_mod, ref_cache[2], bf16_or_f32_to_np(ql[2]),
-                                 bf16_or_f32_to_np(qr[2]), d, sigma, tok=[39])
-        check_outputs(out[2], None, o_ref, None, "bad keep entry skipped")
+        bad[0, 5] = -3   # negative, in the middle of a list
+        for path in _paths(pkg, case, torch.bfloat16, H, has_keep=True):
+            out, _ = _decode(case, 0, ql, qr, torch.tensor(lens, dtype=torch.int32), sigma, path,
+                             keep=bad, keep_len=torch.tensor([400, 312, 2], dtype=torch.int32))
+            assert case.lay.read_status(clear=True) & pkg.KVK_FLAG_KEEP_INDEX
+            o_ref, _ = oracle_decode(oracle_mod, ref_cache[2], bf16_or_f32_to_np(ql[2]),
+                                     bf16_or_f32_to_np(qr[2]), d, sigma, tok=[39])
+            check_outputs(out[2], None, o_ref, None, f"bad keep entry skipped, path {path}")
+            tok0 = np.delete(keep[0, :400], 5)
+            o_ref, _ = oracle_decode(oracle_mod, ref_cache[0], bf16_or_f32_to_np(ql[0]),
+                                     bf16_or_f32_to_np(qr[0]), d, sigma, tok=tok0)
+            check_outputs(out[0], None, o_ref, None, f"negative keep entry skipped, path {path}")
+    finally:
+        case.close()
+
+
+def test_keep_list_tensor_core_workspace(pkg, oracle_mod):
+    """A keep list on the tensor-core kernel: with the keep workspace (NaN-filled) the kept
+    rows are copied densely and decoded there; with only the plain workspace the automatic
+    choice falls back to the CUDA-core kernel, and a forced tensor-core call is refused."""
+    d, r, dR, H, B, T = 512, 512, 64, 40, 3, 2500
+    case = Case(pkg, d, 16, r, dR, B, T)
+    try:
+        c = _rand((B, T, r), 51, torch.bfloat16)
+        kr = _rand((B, T, dR), 52, torch.bfloat16)
+        case.write(c, kr)
+        ql, qr = _rand((B, H, r), 53, torch.bfloat16), _rand((B, H, dR), 54, torch.bfloat16)
+        lens = [2500, 1800, 90]
+        K = 333   # not a multiple of the 64-row tile
+        klen = [333, 200, 90]
+        g = np.random.default_rng(5)
+        keep = np.zeros((B, K), dtype=np.int32)
+        for i in range(B):
+            keep[i, :klen[i]] = np.sort(g.choice(lens[i], klen[i], replace=False))
+        sigma = 1 / math.sqrt(d + dR)
+        ref_cache = oracle_cache(oracle_mod, c, kr, d, 16)
+        refs = [oracle_decode(oracle_mod, ref_cache[i], bf16_or_f32_to_np(ql[i]),
+                              bf16_or_f32_to_np(qr[i]), d, sigma, tok=keep[i, :klen[i]])
+                for i in range(B)]
+        lay = case.lay
+        args = (ql.cuda(), qr.cuda(), torch.tensor(lens, dtype=torch.int32).cuda(), sigma)
+        kw = dict(keep_idx=torch.from_numpy(keep).cuda(),
+                  keep_len=torch.tensor(klen, dtype=torch.int32).cuda())
+        big = lay.workspace_bytes(0, B, H, keep_stride=K)
+        small = lay.workspace_bytes(0, B, H)
+        assert big > small
+        for mode, nbytes in ((1, big), (0, big), (0, small)):
+            lay.set_decode_path(mode)
+            ws = torch.full((nbytes,), 255, dtype=torch.uint8, device="cuda")
+            lse = torch.empty(B, H, dtype=torch.float32, device="cuda")
+            out = lay.mla_decode(0, *args, lse=lse, workspace=ws, **kw)
+            torch.cuda.synchronize()
+            out, lse = out.cpu().numpy(), lse.cpu().numpy()
+            for i in range(B):
+                check_outputs(out[i], lse[i], refs[i][0], refs[i][1],
+                              f"mode {mode} workspace {nbytes} seq {i}")
+        lay.set_decode_path(1)
+        with pytest.raises(pkg.KvkError):
+            lay.mla_decode(0, *args, workspace=torch.empty(small, dtype=torch.uint8,
+                                                           device="cuda"), **kw)
+        lay.set_decode_path(0)
+        assert lay.read_status() == 0
     finally:
         case.close()
 
