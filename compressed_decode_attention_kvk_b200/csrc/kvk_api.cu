@@ -205,8 +205,7 @@ kvk_status kvk_create_layout(int n_layers, const int32_t* anchor, const int32_t*
     for (AnchorDesc& A : L->anchors) {
       void* base = L->arena + A.codes_off;
       A.tmap_ok = make_codes_tmap(&A.tmap_tile, base, (int64_t)tokens, A.row_bytes, A.b,
-                                  kvk::kTcTileTokens) &&
-                  make_codes_tmap(&A.tmap_gather, base, (int64_t)tokens, A.row_bytes, A.b, 1);
+                                  kvk::kTcTileTokens);
     }
   }
   *out = L;

@@ -30,7 +30,6 @@ struct AnchorDesc {
   int64_t scales_off = 0;
   bool tmap_ok = false;
   CUtensorMap tmap_tile;     // 2D [rows = max_batch*max_tokens][row_bytes] uint8, 64-row box
-  CUtensorMap tmap_gather;   // same tensor, one-row box for tile::gather4
 };
 
 }  // namespace kvk

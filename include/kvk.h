@@ -269,7 +269,9 @@ kvk_status kvk_set_decode_path(kvk_layout* layout, int path);
 kvk_status kvk_set_decode_ctas(kvk_layout* layout, int ctas);
 
 /* Which kernel kvk_mla_decode would run for these arguments (KVK_PATH_TENSOR or
- * KVK_PATH_CUDA_CORE), without launching anything.  has_keep != 0: a keep list is given. */
+ * KVK_PATH_CUDA_CORE), without launching anything.  has_keep != 0: a keep list is given;
+ * it does not change the answer, but a keep-list call takes the tensor-core kernel only with
+ * a workspace of kvk_decode_workspace_bytes_keep() bytes (else the CUDA-core kernel). */
 kvk_status kvk_decode_path_for(const kvk_layout* layout, int layer, int dtype, int n_heads,
                                int has_keep, int* path);
 
