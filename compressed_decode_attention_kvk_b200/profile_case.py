@@ -1,13 +1,17 @@
 """One decode layer of a chosen shape, for timing sweeps and ncu captures.
 
   python -m compressed_decode_attention_kvk_b200.profile_case --d 512 --b 16 --heads 40 \\
-      --batch 32 --tokens 8192 --iters 20 [--path tensor|cuda_core] [--ctas N]
+      --batch 32 --tokens 8192 --iters 20 [--path tensor|cuda_core] [--ctas N] [--op write]
 
 Fills one anchor layer's cache through kvk_quant_write with seeded N(0,1) bf16 data, then
 runs kvk_mla_decode `iters` times and prints the mean device time per call (CUDA events on
 the launching stream, after warm-up) and the algorithmic bytes per second
 (batch * tokens * (row_bytes + 2) per call).  At the default shape the cache is ~300 MB,
 larger than the 126 MB L2.
+
+--op write times the quantise-on-write of the whole cache instead (a prefill of batch x
+tokens tokens): algorithmic bytes per call = batch * tokens * ((d + d_rope) * 2 read from
+the bf16 inputs + row_bytes + 2 written).
 """
 from __future__ import annotations
 
@@ -31,6 +35,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--path", default="auto", choices=["auto", "tensor", "cuda_core"])
     ap.add_argument("--ctas", type=int, default=0)
+    ap.add_argument("--op", default="decode", choices=["decode", "write"])
     args = ap.parse_args()
 
     from . import build as kb
@@ -48,6 +53,24 @@ def main():
     c = torch.randn(B, T, args.r, generator=g, device=dev).to(torch.bfloat16)
     kr = torch.randn(B, T, args.d_rope, generator=g, device=dev).to(torch.bfloat16)
     lay.quant_write(0, c, kr, zero)
+    if args.op == "write":
+        for _ in range(args.warmup):
+            lay.quant_write(0, c, kr, zero)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.iters):
+            lay.quant_write(0, c, kr, zero)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / args.iters
+        row = lay.layer_info(0)["row_bytes"]
+        nbytes = B * T * ((args.d + args.d_rope) * 2 + row + 2)
+        print(json.dumps({"op": "write", "d": args.d, "b": args.b, "batch": B, "tokens": T,
+                          "ms_per_call": round(ms, 5), "bytes_per_call": nbytes,
+                          "GBps": round(nbytes / ms / 1e6, 1), "status": lay.read_status()}))
+        lay.close()
+        return
     del c, kr
     ql = torch.randn(B, H, args.r, generator=g, device=dev).to(torch.bfloat16)
     qr = torch.randn(B, H, args.d_rope, generator=g, device=dev).to(torch.bfloat16)
