@@ -82,18 +82,38 @@ def barrier(pg, device=None):
             pg.barrier()
 
 
+# Sources whose code makes up the tensor-core decode kernel (the kernel file and the headers
+# it includes); the traffic record is tied to a comment- and whitespace-insensitive hash.
+KERNEL_SOURCES = ("compressed_decode_attention_kvk_b200/csrc/kvk_decode_tc.cu",
+                  "compressed_decode_attention_kvk_b200/csrc/kvk_sm100.cuh",
+                  "compressed_decode_attention_kvk_b200/csrc/kvk_decode_common.cuh",
+                  "compressed_decode_attention_kvk_b200/csrc/kvk_internal.cuh",
+                  "include/kvk.h")
+
+
+def kernel_code_hash(root=None):
+    """sha256 over KERNEL_SOURCES with comments removed and whitespace collapsed."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(root or ROOT, rel)) as f:
+            s = f.read()
+        s = re.sub(r"/\*.*?\*/", " ", s, flags=re.S)
+        s = re.sub(r"//[^\n]*", " ", s)
+        h.update(" ".join(s.split()).encode())
+        h.update(b"\0")
+    return h.hexdigest()
+
+
 def decode_traffic():
     """DRAM bytes per full-size decode launch of the tensor-core kernel, from the committed ncu
-    capture (profiles/decode_tc_traffic.json), or None when the kernel source has changed
-    since that capture (the record keeps the source's sha256)."""
-    import hashlib
+    capture (profiles/decode_tc_traffic.json), or None when the kernel's code has changed
+    since that capture (the record keeps kernel_code_hash())."""
     try:
         with open(os.path.join(ROOT, "profiles", "decode_tc_traffic.json")) as f:
             rec = json.load(f)
-        src = os.path.join(ROOT, "compressed_decode_attention_kvk_b200", "csrc", "kvk_decode_tc.cu")
-        with open(src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
-        if sha != rec["source_sha256"]:
+        if kernel_code_hash() != rec["code_sha256"]:
             return None
         return rec
     except Exception:

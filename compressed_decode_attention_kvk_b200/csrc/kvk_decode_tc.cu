@@ -7,31 +7,39 @@
 // attention over the dequantised cache; KV-Kaizen "Background": each decode step reads the
 // whole cache).
 //
-// One persistent CTA per SM walks a balanced slice of the flattened token space in tiles of
+// One persistent CTA per SM walks its slice of the flattened token space (the split charges
+// each piece a fixed cost, so a CTA that starts a sequence takes fewer tokens) in tiles of
 // 64 tokens.  Warp roles (512 threads, four warpgroups with their own register budgets):
 //   warps 0-3  softmax: read S from TMEM, per-token scale, lazy online softmax, write P
 //              (f16) to shared memory, rescale O in TMEM when a max grows, write partials
 //   warps 4-11 convert: packed b-bit codes -> f16 operand tiles (UMMA 128-byte-swizzled,
 //              K-major) and their transpose into TMEM; staged query (power-of-two scaled).
 //              Two warps per SM sub-partition, 16 features of every 128-feature group each.
-//   warp 12    TMA producer: 128-feature groups of 64 packed rows into a ring
+//   warp 12    TMA producer: 128-feature groups of 64 packed rows into a ring, and each
+//              tile's token scales; the stream is read once, so it carries an evict-first
+//              L2 policy
 //   warp 13    score-MMA issuer (one thread) and TMEM owner
-//   warp 14    output-MMA issuer (one thread); warp 15 idle
+//   warp 14    output-MMA issuer (one thread)
+//   warp 15    warms L2 with the queries of the CTA's later pieces
 // Launched with 128 registers per thread; the softmax warpgroup raises its budget to
 // kRegsSoftmax, the conversion warpgroups lower theirs to kRegsConvert and the last
 // warpgroup to kRegsIssue (4 x 32 x (192 + 2 x 120 + 56) = 62464 <= 65536).
 // Per tile:  S^T[64 tok x N1 heads]  = C[64 x n] . Q^T         (M=64, A in smem, TMEM f32)
 //            O^T[128 feat x N2 heads] += C^T[128 x 64] . P    (M=128 per 128 latent features,
 //                                                               A = C^T in TMEM)
-// Heads sit on N, so 40 heads cost N = 40 / 48, never M = 128.  After the convert warps have
-// turned a 128-feature group into f16 (UMMA 128-byte swizzled, K-major: the score MMA's A),
-// each of them transposes its 16 features of it into TMEM (ldmatrix.trans -> tcgen05.st),
-// so a ring slot is free as soon as the score MMA has read it; the output MMA reads TMEM.
+// Heads sit on N, so 40 heads cost N = 40 / 48, never M = 128.  The convert warps turn each
+// 128-feature group into f16 in place (UMMA 128-byte swizzled, K-major: the score MMA's A)
+// and put their 16 features of it, transposed, into TMEM (tcgen05.st), so a ring slot is free
+// as soon as the score MMA has read it; the output MMA reads C^T from TMEM.  For 16-bit
+// codes both happen in one register pass (ldmatrix.trans, convert, stmatrix.trans back, the
+// same registers to TMEM); narrower codes are unpacked from a raw ring first and then
+// transposed with ldmatrix.trans.
 // The transpose fragment orders the 16 tokens of each K step as 0,1,8,9,2,3,10,11,4,5,12,13,
 // 6,7,14,15; the softmax warps write P's K rows in that same order.
 // Dequantisation: codes of b <= 8 bits are exact in f16; 16-bit codes are rounded to f16
 // (relative 2^-12).  The per-token scale s_t multiplies the S row and is folded into P as
-// p * s_t / S_max, with S_max a power of two >= every scale of the CTA's slice.
+// p * s_t / S_run, with S_run a running power of two >= every scale seen so far (when it
+// grows, O is rescaled by the exact ratio).
 // Every wait is bounded in time; on expiry the kernel records KVK_FLAG_TIMEOUT, drains its
 // own TMA loads and MMAs, frees TMEM and exits.
 #include <string.h>

@@ -54,3 +54,24 @@ def test_measured_peaks_present():
     assert peak > 1000
     if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")):
         assert kind == "measured"
+
+
+def test_traffic_record_follows_kernel_code_not_comments(tmp_path):
+    """The ncu traffic record applies while the kernel's code is the captured code: a comment
+    edit keeps the hash, a code edit changes it (checked on a copy of the sources)."""
+    import shutil
+    import bench
+    for rel in bench.KERNEL_SOURCES:
+        dst = tmp_path / rel
+        dst.parent.mkdir(parents=True, exist_ok=True)
+        shutil.copy(os.path.join(ROOT, rel), dst)
+    base = bench.kernel_code_hash(str(tmp_path))
+    assert base == bench.kernel_code_hash()
+    k = tmp_path / bench.KERNEL_SOURCES[0]
+    src = k.read_text()
+    k.write_text(src.replace("// ", "//  note: ", 3) + "\n/* trailing remark */\n")
+    assert bench.kernel_code_hash(str(tmp_path)) == base
+    k.write_text(src.replace("kScSlots = 4", "kScSlots = 5", 1))
+    assert bench.kernel_code_hash(str(tmp_path)) != base
+    rec = json.load(open(os.path.join(ROOT, "profiles", "decode_tc_traffic.json")))
+    assert rec["code_sha256"] == base        # the committed record matches the committed kernel
