@@ -237,7 +237,10 @@ kvk_status kvk_mla_decode(kvk_layout* layout, int layer, const void* q_lat, cons
  *
  * Arguments and results are those of kvk_mla_decode minus (workspace, workspace_bytes).
  * A call whose workspace need (kvk_decode_workspace_bytes) exceeds
- * KVK_NOALLOC_SCRATCH_BYTES returns KVK_ERR_WORKSPACE and launches nothing.  This entry
+ * KVK_NOALLOC_SCRATCH_BYTES returns KVK_ERR_WORKSPACE and launches nothing.  A call with a
+ * keep list takes the tensor-core kernel only if the scratch also holds the dense copy of
+ * the kept rows (kvk_decode_workspace_bytes_keep <= KVK_NOALLOC_SCRATCH_BYTES), else the
+ * CUDA-core kernel.  This entry
  * point allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *
  * Set-up: the first call on a device (the device current at the call) looks up the
