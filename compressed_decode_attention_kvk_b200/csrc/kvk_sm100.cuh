@@ -110,7 +110,7 @@ __device__ __forceinline__ void fence_mbar_init() {
 }
 
 // ---------------------------------------------------------------------------------------
-// TMA: 2D tile load global -> shared, completion counted on an mbarrier (no multicast)
+// TMA: 2D tile load global -> shared, completion counted on an mbarrier (this CTA only)
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y,
                                             uint64_t* bar) {
@@ -121,7 +121,7 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, 
       : "memory");
 }
 // Bulk copy (no tensor map) of `bytes` (multiple of 16) from global to shared memory; both
-// addresses 16-byte aligned; completion counted on an mbarrier (no multicast).
+// addresses 16-byte aligned; completion counted on an mbarrier (this CTA only).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
                                           uint64_t* bar) {
   asm volatile(
