@@ -373,7 +373,14 @@ def run_kvk(args, rank, world, local, pg):
 def run_e2e(args, wl, device, pg):
     """Same metric through the public API with host buffers: every step copies the step's
     inputs (new tokens, all layers' queries) from pinned host memory and reads every
-    layer's output back to pinned host memory."""
+    layer's output back to pinned host memory.
+
+    The copies overlap the decode: host-to-device copies run on one stream, device-to-host
+    copies on another (the two directions of the link work at once), and per-layer events
+    order them against the compute stream -- layer l's query is copied in once the previous
+    step's decode of layer l has consumed the buffer, layer l decodes once its query has
+    landed and the previous step's read-back of its output buffer has finished, and layer l's
+    output is read back as soon as its decode is done."""
     from compressed_decode_attention_kvk_b200 import kvk
     L = wl.w.n_layers
     h_app = {l: (c.cpu().pin_memory(), k.cpu().pin_memory()) for l, (c, k) in wl.app.items()}
@@ -393,38 +400,78 @@ def run_e2e(args, wl, device, pg):
         d_keep = torch.empty_like(wl.keep)
         h2d += h_keep.numel() * h_keep.element_size()
 
+    comp = torch.cuda.current_stream(device)
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    ev_app, ev_qw = ev(), ev()
+    ev_q = [ev() for _ in range(L)]
+    ev_dec = [ev() for _ in range(L)]
+    ev_d2h = [ev() for _ in range(L)]
+    first = [True]
+
     def step():
-        if h_keep is not None:
-            d_keep.copy_(h_keep, non_blocking=True)
-        for l in wl.anchors:
-            dc, dk = d_app[l]
-            dc.copy_(h_app[l][0], non_blocking=True)
-            dk.copy_(h_app[l][1], non_blocking=True)
+        # inputs: new tokens (and keep lists) once the previous step's write has read them
+        with torch.cuda.stream(s_in):
+            if not first[0]:
+                s_in.wait_event(ev_qw)
+            if h_keep is not None:
+                if not first[0]:
+                    s_in.wait_event(ev_dec[L - 1])
+                d_keep.copy_(h_keep, non_blocking=True)
+            for l in wl.anchors:
+                dc, dk = d_app[l]
+                dc.copy_(h_app[l][0], non_blocking=True)
+                dk.copy_(h_app[l][1], non_blocking=True)
+            ev_app.record(s_in)
+            for l in range(L):
+                if not first[0]:
+                    s_in.wait_event(ev_dec[l])     # the previous step's decode of l is done
+                qa, qb = d_q[l]
+                qa.copy_(h_q[l][0], non_blocking=True)
+                qb.copy_(h_q[l][1], non_blocking=True)
+                ev_q[l].record(s_in)
+        comp.wait_event(ev_app)
         kvk.kvk_quant_write_layers(wl.lay.handle, wl.anchors, [d_app[l][0] for l in wl.anchors],
-                                   [d_app[l][1] for l in wl.anchors], wl.app_pos)
+                                   [d_app[l][1] for l in wl.anchors], wl.app_pos, stream=comp)
+        ev_qw.record(comp)
         for l in range(L):
+            comp.wait_event(ev_q[l])
+            if not first[0]:
+                comp.wait_event(ev_d2h[l])         # the previous step's read-back of out[l]
             qa, qb = d_q[l]
-            qa.copy_(h_q[l][0], non_blocking=True)
-            qb.copy_(h_q[l][1], non_blocking=True)
             kvk.kvk_mla_decode(wl.lay.handle, l, qa, qb, wl.lens, wl.sigma[l], wl.out[l], wl.ws,
-                               keep_idx=d_keep, keep_len=wl.keep_len)
-            h_out[l].copy_(wl.out[l], non_blocking=True)
+                               keep_idx=d_keep, keep_len=wl.keep_len, stream=comp)
+            ev_dec[l].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_dec[l])
+                h_out[l].copy_(wl.out[l], non_blocking=True)
+                ev_d2h[l].record(s_out)
+        first[0] = False
+
+    def finish():
+        comp.wait_stream(s_out)
+        comp.wait_stream(s_in)
 
     for _ in range(max(1, args.warmup)):
         step()
+    finish()
     torch.cuda.synchronize(device)
     barrier(pg, device)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
+    a.record(comp)
+    s_in.wait_stream(comp)                         # no copy of the timed steps starts before a
+    s_out.wait_stream(comp)
     for _ in range(args.steps):
         step()
-    b.record()
+    finish()                                       # every output is back on the host
+    b.record(comp)
     torch.cuda.synchronize(device)
     t_ms = max_over_ranks(a.elapsed_time(b), pg, device)
     world = 1 if pg is None else pg.get_world_size()
     v = wl.decode_bytes * args.steps * world / (t_ms * 1e-3) / 1e9
     return {"value": round(v, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": round(t_ms / args.steps, 4)}
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(t_ms / args.steps, 4),
+            "copies": "H2D and D2H on their own streams, overlapping the decode"}
 
 
 # ---------------------------------------------------------------------------

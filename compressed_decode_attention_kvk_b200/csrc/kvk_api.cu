@@ -17,6 +17,18 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// A layout's arena lives on one device; a call made with another device current would
+// hand that arena (and, for the no-allocation decode, that device's scratch array) to
+// kernels running elsewhere.  Such calls are refused before anything is launched.
+kvk_status check_device(const kvk_layout* L) {
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) {
+    cudaGetLastError();
+    return KVK_ERR_CUDA;
+  }
+  return cur == L->device ? KVK_OK : KVK_ERR_INVALID_ARG;
+}
+
 int row_bytes_of(int n, int b) {
   int raw = (n * b + 7) / 8;
   return (raw + 15) / 16 * 16;
@@ -50,7 +62,8 @@ bool make_codes_tmap(CUtensorMap* m, void* base, int64_t rows, int row_bytes, in
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   int inner = 128 * b / 8;   // 32, 64, 128 or 256 bytes
-  if (b == 16) inner = 128;  // b = 16: one 64-feature atom per box (two boxes per group)
+  // 16-bit elements (codes or bf16 values): one 64-feature atom per box (two boxes per group)
+  if (b == 16 || b == KVK_BITS_BF16) inner = 128;
   CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_NONE;
   if (inner == 128) sw = CU_TENSOR_MAP_SWIZZLE_128B;
   else if (inner == 64) sw = CU_TENSOR_MAP_SWIZZLE_64B;
@@ -130,15 +143,18 @@ kvk_status kvk_create_layout(int n_layers, const int32_t* anchor, const int32_t*
   if ((int64_t)max_batch * (int64_t)max_tokens >= (int64_t(1) << 31)) return KVK_ERR_INVALID_ARG;
 
   // depth axis: anchor[0] == 0; every other layer is an anchor or points at the nearest
-  // preceding anchor.  rank / precision axes: 16 <= d <= r, d % 16 == 0, b in {2,4,8,16}.
+  // preceding anchor.  rank / precision axes: 16 <= d <= r, d % 16 == 0, b in {2,4,8,16};
+  // b = 0 keeps the anchor uncompressed (bf16 rows, 16 bits per element, no scale).
   int64_t bits = 0;
   int last = -1;
   for (int l = 0; l < n_layers; ++l) {
     if (anchor[l] == l) {
       if (d[l] < 16 || d[l] > r || d[l] % 16 != 0) return KVK_ERR_BAD_TABLE;
-      if (b[l] != 2 && b[l] != 4 && b[l] != 8 && b[l] != 16) return KVK_ERR_BAD_TABLE;
+      if (b[l] != 2 && b[l] != 4 && b[l] != 8 && b[l] != 16 && b[l] != KVK_BITS_BF16)
+        return KVK_ERR_BAD_TABLE;
       if (d[l] + d_rope > kvk::kMaxRowElems) return KVK_ERR_UNSUPPORTED;
-      bits += (int64_t)(d[l] + d_rope) * b[l] + 16;
+      bits += (b[l] == KVK_BITS_BF16) ? (int64_t)(d[l] + d_rope) * 16
+                                      : (int64_t)(d[l] + d_rope) * b[l] + 16;
       last = l;
     } else {
       if (l == 0 || anchor[l] != last) return KVK_ERR_BAD_TABLE;
@@ -166,7 +182,7 @@ kvk_status kvk_create_layout(int n_layers, const int32_t* anchor, const int32_t*
       A.d = d[l];
       A.b = b[l];
       A.n = d[l] + d_rope;
-      A.row_bytes = row_bytes_of(A.n, A.b);
+      A.row_bytes = row_bytes_of(A.n, A.b == KVK_BITS_BF16 ? 16 : A.b);
       off = align_up(off, kAlign);
       A.codes_off = (int64_t)off;
       off += tokens * (size_t)A.row_bytes;
@@ -242,6 +258,7 @@ kvk_status kvk_quant_write(kvk_layout* L, int layer, const void* c_kv, int dtype
   if (dtype != KVK_F32 && dtype != KVK_BF16) return KVK_ERR_INVALID_ARG;
   if (batch < 1 || batch > L->max_batch || n_new < 0) return KVK_ERR_INVALID_ARG;
   if (n_new == 0) return KVK_OK;
+  if (kvk_status ds = check_device(L)) return ds;
   if (!c_kv || !dev_start_pos || (L->d_rope > 0 && !k_rope)) return KVK_ERR_INVALID_ARG;
   if (c_stride_seq < 0 || c_stride_tok < 0 || kr_stride_seq < 0 || kr_stride_tok < 0)
     return KVK_ERR_INVALID_ARG;
@@ -302,6 +319,7 @@ kvk_status kvk_quant_write_layers(kvk_layout* L, int n, const int32_t* layers,
     q.kr_st = kr_stride_tok[k];
   }
   if (n_new == 0) return KVK_OK;
+  if (kvk_status ds = check_device(L)) return ds;
   cudaError_t e = kvk::launch_quant_write_layers(L, Q, n, dtype, batch, dev_start_pos, n_new,
                                                  reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVK_OK : KVK_ERR_CUDA;
@@ -350,13 +368,25 @@ kvk_status kvk_decode_path_for(const kvk_layout* L, int layer, int dtype, int n_
   return KVK_OK;
 }
 
-kvk_status kvk_mla_decode(kvk_layout* L, int layer, const void* q_lat, const void* q_rope,
-                          int dtype, int64_t q_lat_stride_seq, int64_t q_lat_stride_head,
-                          int64_t q_rope_stride_seq, int64_t q_rope_stride_head, int batch,
-                          int n_heads, const int32_t* dev_seq_lens, const int32_t* dev_keep_idx,
-                          const int32_t* dev_keep_len, int keep_stride, float softmax_scale,
-                          float* out, float* lse, void* workspace, size_t workspace_bytes,
-                          kvk_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The new tokens of a fused append + decode (kvk_mla_decode_append).
+struct Append {
+  const void* c;
+  const void* kr;
+  int64_t c_ss, kr_ss;
+  int dtype;
+};
+
+kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* q_rope,
+                       int dtype, int64_t q_lat_stride_seq, int64_t q_lat_stride_head,
+                       int64_t q_rope_stride_seq, int64_t q_rope_stride_head, int batch,
+                       int n_heads, const int32_t* dev_seq_lens, const int32_t* dev_keep_idx,
+                       const int32_t* dev_keep_len, int keep_stride, float softmax_scale,
+                       float* out, float* lse, void* workspace, size_t workspace_bytes,
+                       kvk_stream_t stream, const Append* app) {
   if (!L || layer < 0 || layer >= L->n_layers || !L->arena) return KVK_ERR_INVALID_ARG;
   if (dtype != KVK_F32 && dtype != KVK_BF16 && dtype != KVK_F16) return KVK_ERR_INVALID_ARG;
   if (batch < 1 || batch > L->max_batch || n_heads < 1 || n_heads > 4096)
@@ -377,6 +407,17 @@ kvk_status kvk_mla_decode(kvk_layout* L, int layer, const void* q_lat, const voi
   if (q_lat_stride_seq % 8 || q_lat_stride_head % 8 || q_rope_stride_seq % 8 ||
       q_rope_stride_head % 8)
     return KVK_ERR_ALIGNMENT;
+  if (kvk_status ds = check_device(L)) return ds;
+  if (app) {
+    if (L->anchor[layer] != layer) return KVK_ERR_INHERITING_LAYER;
+    if (dev_keep_idx) return KVK_ERR_INVALID_ARG;
+    if (app->dtype != KVK_F32 && app->dtype != KVK_BF16) return KVK_ERR_INVALID_ARG;
+    if (!app->c || (L->d_rope > 0 && !app->kr) || app->c_ss < 0 || app->kr_ss < 0)
+      return KVK_ERR_INVALID_ARG;
+    if (!aligned16(app->c) || (app->kr && !aligned16(app->kr)) || app->c_ss % 8 ||
+        app->kr_ss % 8)
+      return KVK_ERR_ALIGNMENT;
+  }
   const AnchorDesc& A = L->anchors[L->slot[layer]];
   int path = choose_path(L, A, dtype, n_heads);
   if (path < 0) return KVK_ERR_UNSUPPORTED;
@@ -429,6 +470,7 @@ kvk_status kvk_mla_decode(kvk_layout* L, int layer, const void* q_lat, const voi
   a.out = out;
   a.lse = lse;
   a.flags = reinterpret_cast<uint32_t*>(L->arena);
+  a.limit_ns = L->wait_limit_ns ? L->wait_limit_ns : kvk::kDefaultWaitLimitNs;
   int G = kvk::decode_ctas(L, batch, path);
   size_t need = kvk::decode_workspace(batch, n_heads, A.d, G, workspace, &a);
   if (workspace_bytes < need) return KVK_ERR_WORKSPACE;
@@ -461,16 +503,60 @@ kvk_status kvk_mla_decode(kvk_layout* L, int layer, const void* q_lat, const voi
     a.keep_stride = 0;
     if (e == cudaSuccess) e = kvk::launch_decode_tc(a, keep_tmap, dtype, st);
   } else if (path == KVK_PATH_TENSOR) {
+    if (app) {   // the decode kernel writes the new tokens itself
+      a.app_c = app->c;
+      a.app_kr = app->kr;
+      a.app_c_ss = app->c_ss;
+      a.app_kr_ss = app->kr_ss;
+      a.app_dtype = app->dtype;
+    }
     e = kvk::launch_decode_tc(a, A.tmap_tile, dtype, st);
   } else {
-    e = kvk::launch_decode_fma(a, dtype, st);
+    if (app)
+      e = kvk::launch_quant_append(L, A, app->c, app->dtype, app->c_ss, app->kr, app->kr_ss,
+                                   batch, dev_seq_lens, st);
+    if (e == cudaSuccess) e = kvk::launch_decode_fma(a, dtype, st);
   }
   if (e == cudaSuccess) e = kvk::launch_merge(a, st);
   return e == cudaSuccess ? KVK_OK : KVK_ERR_CUDA;
 }
 
+}  // namespace
+
+extern "C" {
+
+kvk_status kvk_mla_decode(kvk_layout* L, int layer, const void* q_lat, const void* q_rope,
+                          int dtype, int64_t q_lat_stride_seq, int64_t q_lat_stride_head,
+                          int64_t q_rope_stride_seq, int64_t q_rope_stride_head, int batch,
+                          int n_heads, const int32_t* dev_seq_lens, const int32_t* dev_keep_idx,
+                          const int32_t* dev_keep_len, int keep_stride, float softmax_scale,
+                          float* out, float* lse, void* workspace, size_t workspace_bytes,
+                          kvk_stream_t stream) {
+  return decode_impl(L, layer, q_lat, q_rope, dtype, q_lat_stride_seq, q_lat_stride_head,
+                     q_rope_stride_seq, q_rope_stride_head, batch, n_heads, dev_seq_lens,
+                     dev_keep_idx, dev_keep_len, keep_stride, softmax_scale, out, lse, workspace,
+                     workspace_bytes, stream, nullptr);
+}
+
+kvk_status kvk_mla_decode_append(kvk_layout* L, int layer, const void* c_new,
+                                 const void* k_rope_new, int new_dtype, int64_t c_new_stride_seq,
+                                 int64_t k_rope_new_stride_seq, const void* q_lat,
+                                 const void* q_rope, int dtype, int64_t q_lat_stride_seq,
+                                 int64_t q_lat_stride_head, int64_t q_rope_stride_seq,
+                                 int64_t q_rope_stride_head, int batch, int n_heads,
+                                 const int32_t* dev_seq_lens, float softmax_scale, float* out,
+                                 float* lse, void* workspace, size_t workspace_bytes,
+                                 kvk_stream_t stream) {
+  const Append app{c_new, k_rope_new, c_new_stride_seq, k_rope_new_stride_seq, new_dtype};
+  return decode_impl(L, layer, q_lat, q_rope, dtype, q_lat_stride_seq, q_lat_stride_head,
+                     q_rope_stride_seq, q_rope_stride_head, batch, n_heads, dev_seq_lens, nullptr,
+                     nullptr, 0, softmax_scale, out, lse, workspace, workspace_bytes, stream,
+                     &app);
+}
+
 kvk_status kvk_read_status(kvk_layout* L, uint32_t* flags, int clear, kvk_stream_t stream) {
   if (!L || !flags || !L->arena) return KVK_ERR_INVALID_ARG;
+  if (kvk_status ds = check_device(L)) return ds;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint32_t v = 0;
   if (cudaMemcpyAsync(&v, L->arena, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
@@ -494,6 +580,12 @@ kvk_status kvk_set_decode_path(kvk_layout* L, int path) {
 kvk_status kvk_set_decode_ctas(kvk_layout* L, int ctas) {
   if (!L || ctas < 0 || ctas > 65536) return KVK_ERR_INVALID_ARG;
   L->ctas = ctas;
+  return KVK_OK;
+}
+
+kvk_status kvk_set_wait_limit(kvk_layout* L, uint64_t ns) {
+  if (!L) return KVK_ERR_INVALID_ARG;
+  L->wait_limit_ns = ns;
   return KVK_OK;
 }
 

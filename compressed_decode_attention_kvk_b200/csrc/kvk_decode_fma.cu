@@ -71,8 +71,10 @@ __global__ void __launch_bounds__(kHG * 32) decode_fma_kernel(DecodeArgs a) {
   }
   const Tq* qlat = static_cast<const Tq*>(a.q_lat);
   const Tq* qrope = static_cast<const Tq*>(a.q_rope);
-  const int b = a.b;
-  const uint32_t mask = (b == 32) ? 0xffffffffu : ((1u << b) - 1u);
+  // b = KVK_BITS_BF16: 16-bit fields holding bf16 values instead of offset-binary codes
+  const bool bf16_rows = (a.b == KVK_BITS_BF16);
+  const int b = bf16_rows ? 16 : a.b;
+  const uint32_t mask = (1u << b) - 1u;
   const int zero_off = 1 << (b - 1);
   const float zscale = a.sigma * kLog2e;
 
@@ -119,7 +121,8 @@ __global__ void __launch_bounds__(kHG * 32) decode_fma_kernel(DecodeArgs a) {
                 reinterpret_cast<const uint32_t*>(a.codes + (seq_row0 + t) * a.row_bytes);
             const int bit = k * b;
             const uint32_t w = __ldg(row + (bit >> 5));
-            v = (float)((int)((w >> (bit & 31)) & mask) - zero_off);
+            const uint32_t u = (w >> (bit & 31)) & mask;
+            v = bf16_rows ? __uint_as_float(u << 16) : (float)((int)u - zero_off);
           }
           cs[i * ldc + k] = v;
         }

@@ -45,6 +45,7 @@
 #include <string.h>
 
 #include "kvk_decode_common.cuh"
+#include "kvk_quant_common.cuh"
 #include "kvk_sm100.cuh"
 
 namespace kvk {
@@ -66,6 +67,10 @@ constexpr int kMma2Warp = 14;  // output MMAs
 constexpr uint32_t kLaunchRegs = 65536 / kThreads;   // 128
 constexpr uint32_t kRegsSoftmax = 192, kRegsConvert = 120, kRegsIssue = 56;
 static_assert(128 * (kRegsSoftmax + 2 * kRegsConvert + kRegsIssue) <= 65536, "register split");
+// 16-bit rows (int16 codes, or the bf16 values of an uncompressed anchor) are converted in
+// place in the slot the tensor memory accelerator filled; narrower codes go through a raw ring
+template <int BITS>
+constexpr bool kInPlace = (BITS == 16 || BITS == KVK_BITS_BF16);
 template <uint32_t N>
 __device__ __forceinline__ void regs_set() {
   if constexpr (N > kLaunchRegs) regs_inc<N>();
@@ -78,7 +83,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol = 0;          // scores S^T, one buffer (N1 <= 64 columns)
 constexpr uint32_t kCtCol0 = 64;       // C^T double buffer: 64 + 128 b, latent group p at + 32 p
 constexpr uint32_t kOCol0 = 320;       // O^T group p at 320 + N2 p
-constexpr uint64_t kLimitNs = 2000000000ull;
+// limit of the waits that drain a stopping kernel's own loads and MMAs (they always end)
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kSmemLimit = 232448;
 constexpr int kQC = 3;   // 16-byte chunks per lane per query row (rows of up to 768 features)
@@ -88,8 +94,8 @@ constexpr int kQD = 1;   // query rows in flight per convert warp while staging
 constexpr int kScSlots = 4;
 constexpr uint32_t kScBytes = 144;
 // barriers besides the rings: s full/empty, P full/empty (2), C^T full/empty (2), q full/empty,
-// o empty, two MMA drains, q seen, scale full/empty (kScSlots each)
-constexpr int kFixedBars = 2 + 4 + 4 + 6 + 2 * kScSlots;
+// o empty, two MMA drains, q seen, appended, scale full/empty (kScSlots each)
+constexpr int kFixedBars = 2 + 4 + 4 + 7 + 2 * kScSlots;
 
 struct TcParams {
   DecodeArgs a;
@@ -175,9 +181,16 @@ __device__ __forceinline__ void cursor_next(Cursor& c, const int32_t* off, int b
 __device__ __forceinline__ bool wait_noabort(uint64_t* b, uint32_t parity) {
   const uint64_t t0 = globaltimer();
   while (!mbar_try(b, parity)) {
-    if (globaltimer() - t0 > kLimitNs) return false;
+    if (globaltimer() - t0 > kDrainLimitNs) return false;
   }
   return true;
+}
+
+// mbar_wait by every lane of a warp, with one warp-uniform answer (the lanes of a warp then
+// never diverge around the .sync.aligned instructions that follow a wait).
+__device__ __forceinline__ bool wait_warp(uint64_t* b, uint32_t parity, uint32_t abort_saddr,
+                                          uint64_t limit_ns) {
+  return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_saddr, limit_ns));
 }
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
@@ -189,6 +202,11 @@ __device__ __forceinline__ uint32_t cvt_code16(uint32_t w) {
   const __half2 hs = __hsub2(bits_h2(__byte_perm(w, 0x64u, 0x4341u)), __float2half2_rn(1152.f));
   const __half2 ls = __hsub2(bits_h2(__byte_perm(w, 0x64u, 0x4240u)), __float2half2_rn(1024.f));
   return h2_bits(__hfma2(hs, __float2half2_rn(256.f), ls));
+}
+// two bf16 values -> f16x2, round to nearest: exact for values in the f16 normal range
+// (bf16 keeps 8 significant bits, f16 11); beyond +-65504 a value becomes +-inf
+__device__ __forceinline__ uint32_t cvt_bf16x2(uint32_t w) {
+  return h2_bits(__floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
 }
 // bytes of w selected by `sel` (each a field u < 1024) -> f16x2 of (u - bias), exact
 __device__ __forceinline__ uint32_t cvt_small(uint32_t w, uint32_t sel, __half2 bias) {
@@ -211,13 +229,16 @@ __device__ __forceinline__ int conv_row(int lane, int k) {
 }
 
 // Packed b-bit group (64 rows x 128 features, TMA-swizzled) -> f16 pair slot, for the 16
-// features fb .. fb+15 (eight-feature groups g = fb/8 + {0, 1} of every row).  All four
-// packed words of a lane are loaded before the first store.
+// features fb .. fb+15 (eight-feature groups g = fb/8 + {0, 1} of every row), in two halves:
+// load_group reads this lane's packed words (all four rows before any use), store_group
+// unpacks them and writes the f16 rows.
 template <int BITS>
-__device__ __forceinline__ void convert_group(const uint8_t* rawslot, uint8_t* pair, int lane,
-                                              int fb) {
+constexpr int kPackedWords = (BITS == 8) ? 2 : 1;   // 32-bit words per row chunk of a lane
+
+template <int BITS>
+__device__ __forceinline__ void load_group(const uint8_t* rawslot, int lane, int fb,
+                                           uint32_t (&w)[4][kPackedWords<BITS>]) {
   const int g = (fb >> 3) + (lane & 1);
-  uint32_t w[4][BITS == 8 ? 2 : 1];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int r = conv_row(lane, k);
@@ -225,7 +246,7 @@ __device__ __forceinline__ void convert_group(const uint8_t* rawslot, uint8_t* p
       const uint2 u = *reinterpret_cast<const uint2*>(rawslot + r * 128 +
                                                       (((g >> 1) ^ (r & 7)) << 4) + ((g & 1) << 3));
       w[k][0] = u.x;
-      w[k][BITS == 8 ? 1 : 0] = u.y;
+      w[k][kPackedWords<BITS> - 1] = u.y;
     } else if constexpr (BITS == 4) {
       w[k][0] = *reinterpret_cast<const uint32_t*>(
           rawslot + r * 64 + (((g >> 2) ^ ((r >> 1) & 3)) << 4) + ((g & 3) << 2));
@@ -234,6 +255,12 @@ __device__ __forceinline__ void convert_group(const uint8_t* rawslot, uint8_t* p
           rawslot + r * 32 + (((g >> 3) ^ ((r >> 2) & 1)) << 4) + ((g & 7) << 1));
     }
   }
+}
+
+template <int BITS>
+__device__ __forceinline__ void store_group(const uint32_t (&w)[4][kPackedWords<BITS>],
+                                            uint8_t* pair, int lane, int fb) {
+  const int g = (fb >> 3) + (lane & 1);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int r = conv_row(lane, k);
@@ -242,8 +269,8 @@ __device__ __forceinline__ void convert_group(const uint8_t* rawslot, uint8_t* p
       const __half2 bias = __float2half2_rn(1152.f);
       o.x = cvt_small(w[k][0], 0x4140u, bias);
       o.y = cvt_small(w[k][0], 0x4342u, bias);
-      o.z = cvt_small(w[k][BITS == 8 ? 1 : 0], 0x4140u, bias);
-      o.w = cvt_small(w[k][BITS == 8 ? 1 : 0], 0x4342u, bias);
+      o.z = cvt_small(w[k][kPackedWords<BITS> - 1], 0x4140u, bias);
+      o.w = cvt_small(w[k][kPackedWords<BITS> - 1], 0x4342u, bias);
     } else if constexpr (BITS == 4) {
       const __half2 bias = __float2half2_rn(1032.f);
       const uint32_t x = w[k][0] & 0x0F0F0F0Fu, y = (w[k][0] >> 4) & 0x0F0F0F0Fu;
@@ -309,7 +336,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   uint64_t* b_final = b_oempty + 1;       // score-MMA drain
   uint64_t* b_final2 = b_final + 1;       // output-MMA drain
   uint64_t* b_qseen = b_final2 + 1;       // softmax has taken the piece's query scale
-  uint64_t* b_scfull = b_qseen + 1;       // [kScSlots] scale window landed
+  uint64_t* b_app = b_qseen + 1;          // fused append: new tokens written
+  uint64_t* b_scfull = b_app + 1;         // [kScSlots] scale window landed
   uint64_t* b_scempty = b_scfull + kScSlots;   // [kScSlots] scale window read (last)
   Misc* m = reinterpret_cast<Misc*>(smem + P.off_misc);
   int32_t* off = reinterpret_cast<int32_t*>(m + 1);
@@ -321,7 +349,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     for (int i = 0; i < P.PR; ++i) {
       mbar_init(&b_pfull[i], kConvWarps);
       // score MMAs (commit), plus the convert warps where they read the slot after q_full
-      mbar_init(&b_pempty[i], BITS == 16 ? 1 : 1 + kConvWarps);
+      mbar_init(&b_pempty[i], kInPlace<BITS> ? 1 : 1 + kConvWarps);
       mbar_init(&b_tfull[i], 1);
     }
     for (int i = 0; i < P.RR; ++i) {
@@ -342,6 +370,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     mbar_init(b_final, 1);
     mbar_init(b_final2, 1);
     mbar_init(b_qseen, 4);
+    mbar_init(b_app, 1);
     for (int i = 0; i < kScSlots; ++i) {
       mbar_init(&b_scfull[i], 1);
       mbar_init(&b_scempty[i], 4);
@@ -387,19 +416,21 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         cursor_start(c, seq0, off, a.batch, lo, hi);
         uint32_t cnt = 0;
         Ring rg;
-        const int slots = (BITS == 16) ? P.PR : P.RR;
+        const int slots = kInPlace<BITS> ? P.PR : P.RR;
         // hold the first cache loads until the first query is staged: its loads then do not
         // queue behind every CTA's ring fill
-        mbar_wait(b_qfull, 0u, abort, kLimitNs);
+        mbar_wait(b_qfull, 0u, abort, a.limit_ns);
+        // a fused append writes this CTA's new tokens first (the spare warp)
+        if (a.app_c) mbar_wait(b_app, 0u, abort, a.limit_ns);
         Ring sr;   // scale ring
         uint32_t nsc = 0;
         const uint64_t pol = policy_evict_first();   // the cache and its scales are read once
         while (c.valid && !abort_read(abort)) {
           const int row0 = c.seq * a.max_tokens + c.pos;
           bool ok = true;
-          {   // this tile's scale window (the arena has tail slack for the last one)
+          if constexpr (BITS != 0) {   // this tile's scale window (the arena has tail slack)
             const uintptr_t sp = reinterpret_cast<uintptr_t>(a.scales + row0);
-            if (!(ok = mbar_wait(&b_scempty[sr.slot], sr.phase ^ 1u, abort, kLimitNs))) break;
+            if (!(ok = mbar_wait(&b_scempty[sr.slot], sr.phase ^ 1u, abort, a.limit_ns))) break;
             mbar_arrive_expect_tx(&b_scfull[sr.slot], kScBytes);
             bulk_load_hint(m->sc[sr.slot], reinterpret_cast<const void*>(sp & ~uintptr_t(15)),
                            kScBytes, &b_scfull[sr.slot], pol);
@@ -408,15 +439,15 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           }
           for (int p = 0; p < P.NP && ok; ++p) {
             const uint32_t s = rg.slot, ph = rg.phase;
-            if (BITS == 16) {
-              if (!(ok = mbar_wait(&b_pempty[s], ph ^ 1u, abort, kLimitNs))) break;
+            if (kInPlace<BITS>) {
+              if (!(ok = mbar_wait(&b_pempty[s], ph ^ 1u, abort, a.limit_ns))) break;
               const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
               mbar_arrive_expect_tx(&b_tfull[s], nat * kAtom);
               for (int t = 0; t < nat; ++t)
                 tma_load_2d_hint(pairs + s * kPair + t * kAtom, &tmap, (2 * p + t) * 128, row0,
                                  &b_tfull[s], pol);
             } else {
-              if (!(ok = mbar_wait(&b_rempty[s], ph ^ 1u, abort, kLimitNs))) break;
+              if (!(ok = mbar_wait(&b_rempty[s], ph ^ 1u, abort, a.limit_ns))) break;
               mbar_arrive_expect_tx(&b_rfull[s], P.raw_slot);
               tma_load_2d_hint(raw + s * P.raw_slot, &tmap, p * 16 * BITS, row0, &b_rfull[s], pol);
             }
@@ -426,14 +457,15 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           if (!ok) break;
           cursor_next(c, off, a.batch, lo, hi);
         }
-        if (abort_read(abort)) {  // let the loads already issued land before the block exits
-          for (uint32_t k = nsc > (uint32_t)kScSlots ? nsc - kScSlots : 0u; k < nsc; ++k)
-            wait_noabort(&b_scfull[k % kScSlots], (k / kScSlots) & 1u);
-          const uint32_t first = cnt > (uint32_t)slots ? cnt - slots : 0u;
-          for (uint32_t k = first; k < cnt; ++k) {
-            const uint32_t s = k % slots, ph = (k / slots) & 1u;
-            wait_noabort(BITS == 16 ? &b_tfull[s] : &b_rfull[s], ph);
-          }
+        // Let every load this thread issued land before the block exits.  A slot is re-armed
+        // only after its consumers saw the previous load complete, so only the last load of
+        // each slot can still be in flight (after an abort); in a normal run all have landed.
+        for (uint32_t k = nsc > (uint32_t)kScSlots ? nsc - kScSlots : 0u; k < nsc; ++k)
+          wait_noabort(&b_scfull[k % kScSlots], (k / kScSlots) & 1u);
+        const uint32_t first = cnt > (uint32_t)slots ? cnt - slots : 0u;
+        for (uint32_t k = first; k < cnt; ++k) {
+          const uint32_t s = k % slots, ph = (k / slots) & 1u;
+          wait_noabort(kInPlace<BITS> ? &b_tfull[s] : &b_rfull[s], ph);
         }
       }
     } else if (warp == kMmaWarp) {
@@ -450,12 +482,12 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       const uint32_t q_atom = (uint32_t)P.N1 * 128u;
       bool ok = true;
       while (g.valid && ok) {
-        ok = mbar_wait(b_sempty, ((uint32_t)g.tile & 1u) ^ 1u, abort, kLimitNs);
-        if (ok && g.first) ok = mbar_wait(b_qfull, (uint32_t)g.piece & 1u, abort, kLimitNs);
+        ok = mbar_wait(b_sempty, ((uint32_t)g.tile & 1u) ^ 1u, abort, a.limit_ns);
+        if (ok && g.first) ok = mbar_wait(b_qfull, (uint32_t)g.piece & 1u, abort, a.limit_ns);
         ok = __all_sync(0xffffffffu, ok);
         for (int p = 0; p < P.NP && ok; ++p) {
           const uint32_t s = rg.slot;
-          ok = __all_sync(0xffffffffu, mbar_wait(&b_pfull[s], rg.phase, abort, kLimitNs));
+          ok = __all_sync(0xffffffffu, mbar_wait(&b_pfull[s], rg.phase, abort, a.limit_ns));
           if (!ok) break;
           tc_fence_after();
           for (int t = 0; t < 2; ++t) {
@@ -491,10 +523,10 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       bool ok = true;
       while (g.valid && ok) {
         const int sb = g.tile & 1;
-        ok = mbar_wait(&b_Pfull[sb], (uint32_t)(g.tile >> 1) & 1u, abort, kLimitNs);
-        if (ok) ok = mbar_wait(&b_ctfull[sb], (uint32_t)(g.tile >> 1) & 1u, abort, kLimitNs);
+        ok = mbar_wait(&b_Pfull[sb], (uint32_t)(g.tile >> 1) & 1u, abort, a.limit_ns);
+        if (ok) ok = mbar_wait(&b_ctfull[sb], (uint32_t)(g.tile >> 1) & 1u, abort, a.limit_ns);
         if (ok && g.first && g.piece > 0)
-          ok = mbar_wait(b_oempty, (uint32_t)(g.piece - 1) & 1u, abort, kLimitNs);
+          ok = mbar_wait(b_oempty, (uint32_t)(g.piece - 1) & 1u, abort, a.limit_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
@@ -514,6 +546,36 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       __syncwarp();
     } else {
       // ------------------------------------------------------------------ spare warp
+      // Fused append: the new token of every sequence whose last position this CTA owns is
+      // quantised (the write kernel's arithmetic) and stored before the TMA warp issues any
+      // load; the proxy fence makes those generic stores visible to its async-proxy reads.
+      if (a.app_c) {
+        uint8_t* codes_w = const_cast<uint8_t*>(a.codes);
+        __half* scales_w = const_cast<__half*>(a.scales);
+        bool ok = true;
+        for (int i = seq0; i < a.batch && off[i] < hi; ++i) {
+          const int len = off[i + 1] - off[i];
+          const int64_t last = (int64_t)off[i + 1] - 1;
+          if (len == 0 || last < lo || last >= hi) continue;
+          const int64_t r = (int64_t)i * a.max_tokens + (len - 1);
+          if (a.app_dtype == KVK_BF16)
+            ok = write_token_two_pass<__nv_bfloat16>(
+                     static_cast<const __nv_bfloat16*>(a.app_c) + (int64_t)i * a.app_c_ss,
+                     static_cast<const __nv_bfloat16*>(a.app_kr) + (int64_t)i * a.app_kr_ss,
+                     a.d, a.d_rope, a.b, codes_w + r * a.row_bytes, a.row_bytes, scales_w + r) &&
+                 ok;
+          else
+            ok = write_token_two_pass<float>(
+                     static_cast<const float*>(a.app_c) + (int64_t)i * a.app_c_ss,
+                     static_cast<const float*>(a.app_kr) + (int64_t)i * a.app_kr_ss, a.d,
+                     a.d_rope, a.b, codes_w + r * a.row_bytes, a.row_bytes, scales_w + r) &&
+                 ok;
+        }
+        if (!ok && lane == 0) atomicOr(a.flags, KVK_FLAG_NONFINITE);
+        fence_proxy_async_global();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b_app);
+      }
       // Warm L2 with the queries of the sequences after the first that this CTA touches
       // (the convert warps stage the first one at once).
       Cursor c;
@@ -535,29 +597,46 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   } else if (has_work && warp >= kConvWarp0) {
     regs_set<kRegsConvert>();
     // ------------------------------------------------------------------ convert
-    // The convert warps leave their loop only together (named_or agreement at the top of
-    // every tile), so their named barriers never wait for a warp that has gone.  Warp cw
-    // sits in TMEM lane quarter cq = cw % 4 and owns features fb .. fb+15 of every group,
-    // fb = 32 cq + 16 ch (ch = cw / 4): TMEM lanes fb .. fb+15 of C^T.
+    // Warp cw sits in TMEM lane quarter cq = cw % 4 and owns features fb .. fb+15 of every
+    // group, fb = 32 cq + 16 ch (ch = cw / 4): TMEM lanes fb .. fb+15 of C^T.  The groups of a
+    // tile are software-pipelined: the codes of group p+1 are loaded while group p is
+    // converted and stored, so each warp keeps two groups in flight.  The warps share no
+    // barrier among themselves (every hand-off is an mbarrier), so a warp that stops on a
+    // failed wait leaves its loop alone; it then arrives on nothing more, and everything
+    // downstream of the group it stopped at waits until it sees the abort word.
     const int cw = warp - kConvWarp0;
     const int cq = cw & 3, ch = cw >> 2, fb = 32 * cq + 16 * ch;
     Ring pr, rr;   // f16 group ring, packed group ring
     int last_piece = -1;
     bool fail = false;
     const int cpr = P.NQA * 8;   // 16-byte chunks per staged query row
+    // this lane's ldmatrix row address inside a group slot, per 16-token block tg: atom cq/2,
+    // 16-byte chunk 4(cq%2) + 2ch + (lane/8)/2 of token 16tg + 8((lane/8)%2) + lane%8
+    uint32_t aoff[4];
+    {
+      const int mi = lane >> 3, r8 = lane & 7;
+      const int cc = 4 * (cq & 1) + 2 * ch + (mi >> 1);
+#pragma unroll
+      for (int tg = 0; tg < 4; ++tg)
+        aoff[tg] = (uint32_t)((cq >> 1) * kAtom + (16 * tg + 8 * (mi & 1) + r8) * 128 +
+                              ((cc ^ r8) << 4));
+    }
+    const uint32_t pairs_u = smem_u32(pairs);
+    // does this warp own features of group p (the last group may hold only one atom)?
+    auto owns_group = [&](int p) { return (cq >> 1) < (((2 * p + 1) * 64 < a.n) ? 2 : 1); };
     Cursor c;
     cursor_start(c, seq0, off, a.batch, lo, hi);
     while (c.valid) {
-      if (named_or(2, kConvThreads, fail || abort_read(abort))) break;
+      if (fail || abort_read(abort)) break;
       if (c.piece != last_piece) {
         // Stage this sequence's query as f16 rows [N1][n], scaled by 2^e so that max |q|
         // lands in [2^14, 2^15) (exact for bf16 inputs in range); rows >= H and features
         // >= n are zero.  Wait until the previous piece's scores no longer read it and the
         // softmax warps have taken the previous piece's scale (bounds q_full to one phase
         // ahead of its slowest waiter).
-        fail = fail || !mbar_wait(b_qempty, ((uint32_t)c.piece & 1u) ^ 1u, abort, kLimitNs);
+        fail = fail || !wait_warp(b_qempty, ((uint32_t)c.piece & 1u) ^ 1u, abort, a.limit_ns);
         if (c.piece > 0)
-          fail = fail || !mbar_wait(b_qseen, ((uint32_t)c.piece - 1u) & 1u, abort, kLimitNs);
+          fail = fail || !wait_warp(b_qseen, ((uint32_t)c.piece - 1u) & 1u, abort, a.limit_ns);
         const uint8_t* qlat = static_cast<const uint8_t*>(a.q_lat) + 2 * ((int64_t)c.seq * a.ql_ss);
         const uint8_t* qrope =
             static_cast<const uint8_t*>(a.q_rope) + 2 * ((int64_t)c.seq * a.qr_ss);
@@ -619,107 +698,133 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
 #pragma unroll
             for (int j = 0; j < kQC; ++j) v[i][j] = v[i + 1][j];
         }
+        // q_full counts one arrival per convert warp, each after its own rows are written
         fence_proxy_async_smem();
-        named_sync(2, kConvThreads);   // every warp's rows written before q_full
-        if (lane == 0) mbar_arrive(b_qfull);
+        __syncwarp();
+        if (lane == 0 && !fail) mbar_arrive(b_qfull);
         last_piece = c.piece;
       }
       const int ctb = c.tile & 1;   // C^T buffer of this tile
-      for (int p = 0; p < P.NP; ++p) {
-        const uint32_t s = pr.slot, ph = pr.phase;
-        uint8_t* pair = pairs + s * kPair;
-        const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
-        // this warp owns features fb .. fb+15 of the group: atom cq/2, chunks
-        // 4(cq%2) + 2ch + {0, 1} of every token row; it converts them and later transposes them
-        const bool owns = (cq >> 1) < nat;
-        if constexpr (BITS == 16) {
-          // In place, 16-bit codes -> f16, in one pass through registers: each 8x8 block
-          // (8 tokens x 8 features) is loaded transposed, converted element by element, stored
-          // back transposed (row-major again, for the score MMAs) and the same registers, now
-          // feature-major, go to C^T in TMEM (lanes fb .. fb+15 of latent group p).  The slot
-          // is not read after q_full, so only the score MMAs release it.
-          fail = fail || !mbar_wait(&b_tfull[s], ph, abort, kLimitNs);
-          uint32_t cv[16];
-          const bool go = !fail && owns;
+      const uint32_t ct_addr = tmem + ((uint32_t)fb << 16) + kCtCol0 + 128u * ctb;
+      if constexpr (kInPlace<BITS>) {
+        // In place, 16-bit codes (or bf16 values) -> f16, in one pass through registers: each 8x8 block
+        // (8 tokens x 8 features) is loaded transposed, converted element by element, stored
+        // back transposed (row-major again, for the score MMAs) and the same registers, now
+        // feature-major, go to C^T in TMEM (lanes fb .. fb+15 of latent group p).  The slot
+        // is not read after q_full, so only the score MMAs release it.
+        uint32_t xa[16], xb[16];
+        auto load16 = [&](uint32_t slot, uint32_t (&x)[16]) {
+          const uint32_t base = pairs_u + slot * (uint32_t)kPair;
+#pragma unroll
+          for (int tg = 0; tg < 4; ++tg) {
+            uint32_t d4[4];
+            ldsm_x4_trans(base + aoff[tg], d4);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) x[4 * tg + i] = d4[i];
+          }
+        };
+        // group p is in x (loaded); convert it, load group p+1 into y, store and hand off x
+        auto step16 = [&](int p, uint32_t (&x)[16], uint32_t (&y)[16]) {
+          const uint32_t s = pr.slot;
+          const bool go = !fail && owns_group(p);
           if (go) {
-            const uint32_t abase = smem_u32(pair + (cq >> 1) * kAtom);
-            const int mi = lane >> 3, r8 = lane & 7;
-            const int cc = 4 * (cq & 1) + 2 * ch + (mi >> 1);
-            uint32_t ad[4];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = (BITS == 0) ? cvt_bf16x2(x[i]) : cvt_code16(x[i]);
+          }
+          if (p + 1 < P.NP) {
+            Ring nx = pr;
+            nx.next(P.PR);
+            fail = fail || !wait_warp(&b_tfull[nx.slot], nx.phase, abort, a.limit_ns);
+            if (!fail && owns_group(p + 1)) load16(nx.slot, y);
+          }
+          if (go) {
+            const uint32_t base = pairs_u + s * (uint32_t)kPair;
 #pragma unroll
             for (int tg = 0; tg < 4; ++tg) {
-              const int tok = 16 * tg + 8 * (mi & 1) + r8;
-              ad[tg] = abase + tok * 128 + ((cc ^ r8) << 4);
-              uint32_t d4[4];
-              ldsm_x4_trans(ad[tg], d4);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) cv[4 * tg + i] = d4[i];
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) cv[i] = cvt_code16(cv[i]);
-#pragma unroll
-            for (int tg = 0; tg < 4; ++tg) {
-              const uint32_t d4[4] = {cv[4 * tg], cv[4 * tg + 1], cv[4 * tg + 2], cv[4 * tg + 3]};
-              stsm_x4_trans(ad[tg], d4);
+              const uint32_t d4[4] = {x[4 * tg], x[4 * tg + 1], x[4 * tg + 2], x[4 * tg + 3]};
+              stsm_x4_trans(base + aoff[tg], d4);
             }
           }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&b_pfull[s]);
+          if (lane == 0 && !fail) mbar_arrive(&b_pfull[s]);
           if (p < P.NPd) {
             if (p == 0) {   // the output MMAs of tile - 2 have finished reading this buffer
-              fail = fail || !mbar_wait(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u,
-                                        abort, kLimitNs);
+              fail = fail || !wait_warp(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u,
+                                        abort, a.limit_ns);
               tc_fence_after();
             }
-            if (go) tmem_st16x256b_x4(tmem + ((uint32_t)fb << 16) + kCtCol0 + 128u * ctb + 32u * p, cv);
+            if (go && !fail) tmem_st16x256b_x4(ct_addr + 32u * p, x);
           }
-        } else {
-          const uint32_t rs = rr.slot, rph = rr.phase;
-          fail = fail || !mbar_wait(&b_rfull[rs], rph, abort, kLimitNs);
-          fail = fail || !mbar_wait(&b_pempty[s], ph ^ 1u, abort, kLimitNs);
-          if (!fail) convert_group<BITS>(raw + rs * P.raw_slot, pair, lane, fb);
+          pr.next(P.PR);
+        };
+        fail = fail || !wait_warp(&b_tfull[pr.slot], pr.phase, abort, a.limit_ns);
+        if (!fail && owns_group(0)) load16(pr.slot, xa);
+        for (int p = 0; p < P.NP; p += 2) {
+          step16(p, xa, xb);
+          if (p + 1 < P.NP) step16(p + 1, xb, xa);
+        }
+      } else {
+        // Packed codes: group p's words are loaded into registers (and its raw slot released)
+        // before group p-1 is converted; then each group is unpacked into its f16 slot, and
+        // this warp's 16 features are read back transposed into C^T.
+        constexpr int NW = kPackedWords<BITS>;
+        uint32_t wa[4][NW], wb[4][NW];
+        auto loadw = [&](uint32_t (&w)[4][NW]) {
+          const uint32_t rs = rr.slot;
+          fail = fail || !wait_warp(&b_rfull[rs], rr.phase, abort, a.limit_ns);
+          if (!fail) load_group<BITS>(raw + rs * P.raw_slot, lane, fb, w);
           __syncwarp();
-          if (lane == 0) mbar_arrive(&b_rempty[rs]);
+          if (lane == 0 && !fail) mbar_arrive(&b_rempty[rs]);
           rr.next(P.RR);
+        };
+        auto stepw = [&](int p, uint32_t (&w)[4][NW], uint32_t (&wn)[4][NW]) {
+          const uint32_t s = pr.slot, ph = pr.phase;
+          uint8_t* pair = pairs + s * kPair;
+          if (p + 1 < P.NP) loadw(wn);
+          fail = fail || !wait_warp(&b_pempty[s], ph ^ 1u, abort, a.limit_ns);
+          if (!fail) store_group<BITS>(w, pair, lane, fb);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&b_pfull[s]);
+          if (lane == 0 && !fail) mbar_arrive(&b_pfull[s]);
           if (p < P.NPd) {
             // transpose this warp's 16 features x 64 tokens into C^T (TMEM lanes fb .. fb+15
             // of latent group p): four 16-token blocks
             if (p == 0) {   // the output MMAs of tile - 2 have finished reading this buffer
-              fail = fail || !mbar_wait(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u, abort,
-                                        kLimitNs);
+              fail = fail || !wait_warp(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u,
+                                        abort, a.limit_ns);
               tc_fence_after();
             }
-            if (!fail && owns) {
-              const uint32_t abase = smem_u32(pair + (cq >> 1) * kAtom);
-              const int mi = lane >> 3, r8 = lane & 7;
-              const int cc = 4 * (cq & 1) + 2 * ch + (mi >> 1);
-              uint32_t rr[16];
+            if (!fail && owns_group(p)) {
+              const uint32_t base = smem_u32(pair);
+              uint32_t x[16];
 #pragma unroll
               for (int tg = 0; tg < 4; ++tg) {
-                const int tok = 16 * tg + 8 * (mi & 1) + r8;
                 uint32_t d4[4];
-                ldsm_x4_trans(abase + tok * 128 + ((cc ^ (tok & 7)) << 4), d4);
+                ldsm_x4_trans(base + aoff[tg], d4);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) rr[4 * tg + i] = d4[i];
+                for (int i = 0; i < 4; ++i) x[4 * tg + i] = d4[i];
               }
-              tmem_st16x256b_x4(tmem + ((uint32_t)fb << 16) + kCtCol0 + 128u * ctb + 32u * p, rr);
+              tmem_st16x256b_x4(ct_addr + 32u * p, x);
             }
           }
           __syncwarp();
-          if (lane == 0) mbar_arrive(&b_pempty[s]);   // this warp is done reading the slot
+          if (lane == 0 && !fail) mbar_arrive(&b_pempty[s]);   // this warp is done with the slot
+          pr.next(P.PR);
+        };
+        loadw(wa);
+        for (int p = 0; p < P.NP; p += 2) {
+          stepw(p, wa, wb);
+          if (p + 1 < P.NP) stepw(p + 1, wb, wa);
         }
-        pr.next(P.PR);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&b_ctfull[ctb]);
+      if (lane == 0 && !fail) mbar_arrive(&b_ctfull[ctb]);
       cursor_next(c, off, a.batch, lo, hi);
     }
+    tmem_wait_st();   // no TMEM store of this warp is outstanding when the role ends
   } else if (has_work) {
     regs_set<kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax
@@ -756,25 +861,28 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     while (c.valid) {
       const int t = c.tile, sb = t & 1;
       float s_a = 0.f, s_b = 0.f;
-      {
-        fail = fail || !mbar_wait(&b_scfull[sr.slot], sr.phase, abort, kLimitNs);
+      if constexpr (BITS == 0) {   // uncompressed rows: every token's scale is 1
+        s_a = (ra < c.cnt) ? 1.f : 0.f;
+        s_b = (rb < c.cnt) ? 1.f : 0.f;
+      } else {
+        fail = fail || !mbar_wait(&b_scfull[sr.slot], sr.phase, abort, a.limit_ns);
         const __half* w = reinterpret_cast<const __half*>(m->sc[sr.slot]) +
                           ((reinterpret_cast<uintptr_t>(a.scales + (int64_t)c.seq * a.max_tokens +
                                                         c.pos) & 15u) >> 1);
         if (ra < c.cnt) s_a = __half2float(w[ra]);
         if (rb < c.cnt) s_b = __half2float(w[rb]);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&b_scempty[sr.slot]);
+        if (lane == 0 && !fail) mbar_arrive(&b_scempty[sr.slot]);
         sr.next(kScSlots);
       }
       if (c.first) {
-        fail = fail || !mbar_wait(b_qfull, (uint32_t)c.piece & 1u, abort, kLimitNs);
+        fail = fail || !mbar_wait(b_qfull, (uint32_t)c.piece & 1u, abort, a.limit_ns);
 #pragma unroll
         for (int j = 0; j < NB; ++j)
 #pragma unroll
           for (int e = 0; e < 2; ++e) qh[2 * j + e] = m->qs_inv[c.piece & 1][8 * j + hc + e];
         __syncwarp();
-        if (lane == 0) mbar_arrive(b_qseen);
+        if (lane == 0 && !fail) mbar_arrive(b_qseen);
 #pragma unroll
         for (int i = 0; i < 2 * NB; ++i) {
           l[i] = 0.f;
@@ -784,7 +892,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       }
       const bool va = ra < c.cnt, vb = rb < c.cnt;
       const float ca = coef0 * s_a, cbf = coef0 * s_b;
-      fail = fail || !mbar_wait(b_sfull, (uint32_t)t & 1u, abort, kLimitNs);
+      fail = fail || !mbar_wait(b_sfull, (uint32_t)t & 1u, abort, a.limit_ns);
       tc_fence_after();
       float x[4 * NB];
       if constexpr (NB == 8) {
@@ -814,7 +922,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(b_sempty);
+      if (lane == 0 && !fail) mbar_arrive(b_sempty);
       bool mine = (pt == 0) || s_a > srun || s_b > srun;
 #pragma unroll
       for (int j = 0; j < NB; ++j) {
@@ -884,7 +992,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           // rescale O once the previous tile's output MMAs are done
           const int tp = t - 1;
           fail = fail ||
-                 !mbar_wait(&b_Pempty[tp & 1], (uint32_t)(tp >> 1) & 1u, abort, kLimitNs);
+                 !mbar_wait(&b_Pempty[tp & 1], (uint32_t)(tp >> 1) & 1u, abort, a.limit_ns);
           tc_fence_after();
           for (int p = 0; p < P.NPd; ++p) {
 #pragma unroll
@@ -907,7 +1015,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       // (k/8) lbo_p + 128 j + (k%8) 16; this thread's word for heads 8j + hc + {0, 1} is at
       // + 4 (lane % 4).  lbo_p = 16 N2 + 32 puts the two core rows a warp writes in
       // disjoint banks.
-      fail = fail || !mbar_wait(&b_Pempty[sb], ((uint32_t)(t >> 1) & 1u) ^ 1u, abort, kLimitNs);
+      fail = fail || !mbar_wait(&b_Pempty[sb], ((uint32_t)(t >> 1) & 1u) ^ 1u, abort, a.limit_ns);
       {
         const float wa = s_a * inv_srun, wb = s_b * inv_srun;
         uint8_t* pbuf = p_s + sb * P.p_bytes + 4 * (lane & 3);
@@ -931,12 +1039,12 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&b_Pfull[sb]);
+      if (lane == 0 && !fail) mbar_arrive(&b_Pfull[sb]);
       ++pt;
 
       if (c.last) {
         // -------- epilogue of the piece: partials to the workspace slot blockIdx.x + seq
-        fail = fail || !mbar_wait(&b_Pempty[sb], (uint32_t)(t >> 1) & 1u, abort, kLimitNs);
+        fail = fail || !mbar_wait(&b_Pempty[sb], (uint32_t)(t >> 1) & 1u, abort, a.limit_ns);
         tc_fence_after();
 #pragma unroll
         for (int j = 0; j < NB; ++j) {
@@ -976,7 +1084,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(b_oempty);
+        if (lane == 0 && !fail) mbar_arrive(b_oempty);
         named_sync(1, 128);   // red / m_ref reads done before the next piece writes them
       }
       cursor_next(c, off, a.batch, lo, hi);
@@ -1023,7 +1131,8 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
   P.p_bytes = 8u * P.lbo_p;
   const size_t p_bytes = 2 * (size_t)P.p_bytes;
   const size_t misc_bytes = sizeof(Misc) + sizeof(int32_t) * (size_t)(batch + 1);
-  const int raw_slot = (b == 16) ? 0 : 64 * 16 * b;
+  const bool in_place = (b == 16 || b == KVK_BITS_BF16);
+  const int raw_slot = in_place ? 0 : 64 * 16 * b;
   P.raw_slot = raw_slot;
   // try the largest rings that fit
   const size_t fixed = align_up(q_bytes, 1024) + align_up(p_bytes, 1024);
@@ -1036,7 +1145,7 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
     return off + 1024;   // runtime alignment slack of the dynamic shared memory base
   };
   int PR = 0, RR = 0;
-  if (b == 16) {
+  if (in_place) {
     for (PR = 3 * P.NP; PR >= P.NP; --PR)
       if (total_for(PR, 0) <= (size_t)kSmemLimit) break;
   } else {
@@ -1047,7 +1156,7 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
       if (RR >= 2 && total_for(PR, RR) <= (size_t)kSmemLimit) break;
     }
   }
-  if (PR < P.NP || (b != 16 && RR < 2)) return pl;
+  if (PR < P.NP || (!in_place && RR < 2)) return pl;
   P.PR = PR;
   P.RR = RR;
   size_t off = fixed;
@@ -1092,6 +1201,7 @@ bool launch_regs_ok(int b, int N2) {
   int r = 0;
   switch (b) {
     case 16: r = instance_regs_nh<16>(N2); break;
+    case KVK_BITS_BF16: r = instance_regs_nh<KVK_BITS_BF16>(N2); break;
     case 8: r = instance_regs_nh<8>(N2); break;
     case 4: r = instance_regs_nh<4>(N2); break;
     case 2: r = instance_regs_nh<2>(N2); break;
@@ -1139,6 +1249,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tmap, int d
   pl.p.qdtype = dtype;
   switch (a.b) {
     case 16: return launch_bits<16>(pl.p, tmap, pl.smem, a.G, st);
+    case KVK_BITS_BF16: return launch_bits<KVK_BITS_BF16>(pl.p, tmap, pl.smem, a.G, st);
     case 8: return launch_bits<8>(pl.p, tmap, pl.smem, a.G, st);
     case 4: return launch_bits<4>(pl.p, tmap, pl.smem, a.G, st);
     case 2: return launch_bits<2>(pl.p, tmap, pl.smem, a.G, st);

@@ -19,6 +19,8 @@ constexpr int kTcTileTokens = 64;       // tokens per tile of the tensor-core de
 // Work-split cost of one piece on the tensor-core decode, in tokens: query staging and the
 // pipeline refill at a sequence boundary take about as long as 2.5 tiles.
 constexpr int kTcPieceCost = 160;
+// Default time limit of one wait inside the tensor-core decode (kvk_set_wait_limit).
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 
 struct AnchorDesc {
   int layer = 0;
@@ -50,6 +52,7 @@ struct kvk_layout {
   int ctas = 0;
   int device = -1;
   int num_sms = 0;
+  uint64_t wait_limit_ns = 0;             // tensor-core decode wait limit (0: the default)
 };
 
 namespace kvk {
@@ -80,6 +83,15 @@ struct DecodeArgs {
   int G;                     // CTAs the flattened tokens are split over
   int split_x;               // cost of a piece in tokens (split_cost / split_token)
   uint32_t* flags;
+  uint64_t limit_ns;         // time limit of one wait in the tensor-core kernel
+  // fused append (kvk_mla_decode_append): before the decode reads it, the new token of
+  // sequence i -- app_c[i * app_c_ss + k] (k < d) and app_kr[i * app_kr_ss + k] (k < d_rope),
+  // dtype app_dtype -- is written at position seq_len_i - 1 of the cache.  app_c == nullptr:
+  // no append.
+  const void* app_c;
+  const void* app_kr;
+  int64_t app_c_ss, app_kr_ss;
+  int app_dtype;
 };
 
 // Workspace carve-up: returns total bytes; fills pointers when base != nullptr.
@@ -109,6 +121,12 @@ struct QuantLayers {
 cudaError_t launch_quant_write_layers(const kvk_layout* L, const QuantLayers& Q, int n, int dtype,
                                       int batch, const int32_t* start_pos, int n_new,
                                       cudaStream_t stream);
+// One new token per sequence written at position clamp(seq_lens[i], 0, max_tokens) - 1 (none
+// for an empty sequence): the append of a fused append + decode when its decode kernel cannot
+// take the append itself.
+cudaError_t launch_quant_append(const kvk_layout* L, const AnchorDesc& A, const void* c_new,
+                                int dtype, int64_t c_ss, const void* kr_new, int64_t kr_ss,
+                                int batch, const int32_t* seq_lens, cudaStream_t stream);
 cudaError_t launch_decode_fma(const DecodeArgs& a, int dtype, cudaStream_t stream);
 // tmap: the codes plane the kernel streams (the anchor's, or a compacted keep-list copy)
 cudaError_t launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tmap, int dtype,

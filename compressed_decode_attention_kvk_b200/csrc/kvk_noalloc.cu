@@ -15,15 +15,11 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[KVK_NOALLOC_SCR
 constexpr int kMaxDevices = 64;
 std::atomic<void*> g_scratch_ptr[kMaxDevices];
 
-// Device address of the scratch array on the current device, looked up once per device.
-// The array's name in host code is only a host-side handle; the kernels must be given the
-// address cudaGetSymbolAddress returns.
-kvk_status scratch_for_current_device(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    cudaGetLastError();
-    return KVK_ERR_CUDA;
-  }
+// Device address of the scratch array on device `dev` (which is current), looked up once per
+// device.  The array's name in host code is only a host-side handle; the kernels must be
+// given the address cudaGetSymbolAddress returns.
+kvk_status scratch_for_device(int dev, void** out) {
+  if (dev < 0 || dev >= kMaxDevices) return KVK_ERR_INVALID_ARG;
   void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
   if (!p) {
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
@@ -44,14 +40,19 @@ extern "C" kvk_status kvk_mla_decode_noalloc(
     int64_t q_rope_stride_head, int batch, int n_heads, const int32_t* dev_seq_lens,
     const int32_t* dev_keep_idx, const int32_t* dev_keep_len, int keep_stride,
     float softmax_scale, float* out, float* lse, kvk_stream_t stream) {
-  if (!layout) return KVK_ERR_INVALID_ARG;
-  size_t need = 0;
-  kvk_status st = kvk_decode_workspace_bytes(layout, layer, batch, n_heads, &need);
-  if (st != KVK_OK) return st;
-  if (need > KVK_NOALLOC_SCRATCH_BYTES) return KVK_ERR_WORKSPACE;
+  if (!layout || !layout->arena) return KVK_ERR_INVALID_ARG;
+  // the scratch address is per device: look it up only with the layout's device current
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) {
+    cudaGetLastError();
+    return KVK_ERR_CUDA;
+  }
+  if (cur != layout->device) return KVK_ERR_INVALID_ARG;
   void* scratch = nullptr;
-  st = scratch_for_current_device(&scratch);
+  kvk_status st = scratch_for_device(cur, &scratch);
   if (st != KVK_OK) return st;
+  // kvk_mla_decode checks the workspace against the need of the kernel it takes and
+  // returns KVK_ERR_WORKSPACE (launching nothing) when the scratch is too small for it
   return kvk_mla_decode(layout, layer, q_lat, q_rope, dtype, q_lat_stride_seq,
                         q_lat_stride_head, q_rope_stride_seq, q_rope_stride_head, batch,
                         n_heads, dev_seq_lens, dev_keep_idx, dev_keep_len, keep_stride,

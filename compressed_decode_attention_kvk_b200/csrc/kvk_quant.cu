@@ -13,36 +13,13 @@
 // group's packed bytes (b bytes per group) -- consecutive lanes write consecutive bytes.
 // The kernel is HBM bound: it reads (d + d_R) * sizeof(input) and writes row + 2 bytes
 // per token.
-#include "kvk_internal.cuh"
+#include "kvk_quant_common.cuh"
 
 namespace kvk {
 namespace {
 
 constexpr int kWarpsPerBlock = 8;
 constexpr int kMaxRounds = kMaxRowElems / (8 * 32);  // groups of 8 per lane
-
-template <typename T>
-__device__ __forceinline__ void load8(const T* p, float (&v)[8]);
-
-template <>
-__device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
-  float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-
-template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
-  uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    // a bf16 is the high half of a binary32: widening is exact
-    v[2 * k] = __uint_as_float(w[k] << 16);
-    v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-  }
-}
 
 // One warp quantises token `tok` (of batch x n_new) of one anchor layer.
 template <typename T>
@@ -87,54 +64,31 @@ __device__ __forceinline__ void quant_token(
     return;
   }
 
-  const int q = (1 << (b - 1)) - 1;
-  const float s32 = __fdiv_rn(amax, (float)q);          // IEEE binary32 division
-  const __half s16 = __float2half_ru(s32);               // rounded toward +inf
+  uint8_t* row = codes + ((int64_t)seq * max_tokens + pos) * row_bytes;
+  // uncompressed anchor: the bf16 of every element (round to nearest even) and scale 1
+  const __half s16 = (b == KVK_BITS_BF16) ? __float2half(1.0f) : quant_scale(amax, b);
   const float s = __half2float(s16);
   if (lane == 0) {
-    if (!finite || isinf(s)) atomicOr(flags, KVK_FLAG_NONFINITE);
+    if (!finite || (b != KVK_BITS_BF16 && isinf(s))) atomicOr(flags, KVK_FLAG_NONFINITE);
     scales[(int64_t)seq * max_tokens + pos] = s16;
   }
-  uint8_t* row = codes + ((int64_t)seq * max_tokens + pos) * row_bytes;
-  const uint32_t off = 1u << (b - 1);
-
+  const int gb = group_bytes(b);
 #pragma unroll
   for (int r = 0; r < kMaxRounds; ++r) {
     const int g = r * 32 + lane;
     if (g >= groups) continue;
-    uint32_t u[8];
+    uint8_t* dst = row + (int64_t)g * gb;                // 8 elements: b bytes (16 for bf16)
+    if (b == KVK_BITS_BF16) {
+      store_bf16x8(dst, v[r]);
+    } else {
+      uint32_t u[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      int c = 0;
-      if (s != 0.0f) {
-        c = __float2int_rn(__fdiv_rn(v[r][k], s));       // round half to even
-        c = min(max(c, -q), q);
-      }
-      u[k] = (uint32_t)(c + (int)off);
-    }
-    uint8_t* dst = row + (int64_t)g * b;                 // 8 elements * b bits = b bytes
-    if (b == 16) {
-      uint4 w = make_uint4(u[0] | (u[1] << 16), u[2] | (u[3] << 16), u[4] | (u[5] << 16),
-                           u[6] | (u[7] << 16));
-      *reinterpret_cast<uint4*>(dst) = w;
-    } else if (b == 8) {
-      uint2 w = make_uint2(u[0] | (u[1] << 8) | (u[2] << 16) | (u[3] << 24),
-                           u[4] | (u[5] << 8) | (u[6] << 16) | (u[7] << 24));
-      *reinterpret_cast<uint2*>(dst) = w;
-    } else if (b == 4) {
-      uint32_t w = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) w |= u[k] << (4 * k);
-      *reinterpret_cast<uint32_t*>(dst) = w;
-    } else {  // b == 2
-      uint32_t w = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) w |= u[k] << (2 * k);
-      *reinterpret_cast<uint16_t*>(dst) = (uint16_t)w;
+      for (int k = 0; k < 8; ++k) u[k] = quant_field(v[r][k], s, b);
+      store_fields8(dst, u, b);
     }
   }
   // zero the row padding (fewer than 16 bytes)
-  const int used = groups * b;
+  const int used = groups * gb;
   if (lane < row_bytes - used) row[used + lane] = 0;
 }
 
@@ -163,7 +117,45 @@ quant_write_layers_kernel(const __grid_constant__ QuantLayers Q, int d_rope, int
                  start_pos, n_new, flags);
 }
 
+// One warp per sequence: the new token goes to position clamp(len, 0, max_tokens) - 1.
+template <typename T>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+quant_append_kernel(uint8_t* __restrict__ codes, __half* __restrict__ scales, int row_bytes,
+                    int d, int d_rope, int b, int max_tokens, const T* __restrict__ c_new,
+                    int64_t c_ss, const T* __restrict__ kr_new, int64_t kr_ss, int batch,
+                    const int32_t* __restrict__ seq_lens, uint32_t* __restrict__ flags) {
+  const int i = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  if (i >= batch) return;
+  const int len = min(max(__ldg(seq_lens + i), 0), max_tokens);
+  if (len == 0) return;
+  const int64_t r = (int64_t)i * max_tokens + (len - 1);
+  if (!write_token_two_pass<T>(c_new + (int64_t)i * c_ss, kr_new + (int64_t)i * kr_ss, d,
+                               d_rope, b, codes + r * row_bytes, row_bytes, scales + r) &&
+      (threadIdx.x & 31) == 0)
+    atomicOr(flags, KVK_FLAG_NONFINITE);
+}
+
 }  // namespace
+
+cudaError_t launch_quant_append(const kvk_layout* L, const AnchorDesc& A, const void* c_new,
+                                int dtype, int64_t c_ss, const void* kr_new, int64_t kr_ss,
+                                int batch, const int32_t* seq_lens, cudaStream_t stream) {
+  uint8_t* codes = L->arena + A.codes_off;
+  __half* scales = reinterpret_cast<__half*>(L->arena + A.scales_off);
+  uint32_t* flags = reinterpret_cast<uint32_t*>(L->arena);
+  dim3 grid((unsigned)((batch + kWarpsPerBlock - 1) / kWarpsPerBlock)), block(kWarpsPerBlock * 32);
+  if (dtype == KVK_BF16)
+    quant_append_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
+        codes, scales, A.row_bytes, A.d, L->d_rope, A.b, L->max_tokens,
+        static_cast<const __nv_bfloat16*>(c_new), c_ss, static_cast<const __nv_bfloat16*>(kr_new),
+        kr_ss, batch, seq_lens, flags);
+  else
+    quant_append_kernel<float><<<grid, block, 0, stream>>>(
+        codes, scales, A.row_bytes, A.d, L->d_rope, A.b, L->max_tokens,
+        static_cast<const float*>(c_new), c_ss, static_cast<const float*>(kr_new), kr_ss, batch,
+        seq_lens, flags);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quant_write(const kvk_layout* L, const AnchorDesc& A, const void* c_kv,
                                int dtype, int64_t c_ss, int64_t c_st, const void* k_rope,

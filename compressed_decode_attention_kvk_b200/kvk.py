@@ -33,7 +33,7 @@ EXPORTED = ("kvk_create_layout", "kvk_destroy", "kvk_get_layer_info", "kvk_quant
             "kvk_decode_workspace_bytes", "kvk_mla_decode", "kvk_read_status",
             "kvk_set_decode_path", "kvk_set_decode_ctas", "kvk_decode_path_for",
             "kvk_status_string", "kvk_mla_decode_noalloc", "kvk_quant_write_layers",
-            "kvk_decode_workspace_bytes_keep")
+            "kvk_decode_workspace_bytes_keep", "kvk_set_wait_limit", "kvk_mla_decode_append")
 
 # size of the library's built-in scratch array used by kvk_mla_decode_noalloc
 KVK_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -75,11 +75,14 @@ def _lib_handle():
         L.kvk_decode_workspace_bytes_keep.argtypes = [P, i32, i32, i32, i32, P]
         L.kvk_mla_decode.argtypes = [P, i32, P, P, i32, i64, i64, i64, i64, i32, i32, P, P, P,
                                      i32, ctypes.c_float, P, P, P, sz, P]
+        L.kvk_mla_decode_append.argtypes = [P, i32, P, P, i32, i64, i64, P, P, i32, i64, i64, i64,
+                                            i64, i32, i32, P, ctypes.c_float, P, P, P, sz, P]
         L.kvk_mla_decode_noalloc.argtypes = [P, i32, P, P, i32, i64, i64, i64, i64, i32, i32,
                                              P, P, P, i32, ctypes.c_float, P, P, P]
         L.kvk_read_status.argtypes = [P, P, i32, P]
         L.kvk_set_decode_path.argtypes = [P, i32]
         L.kvk_set_decode_ctas.argtypes = [P, i32]
+        L.kvk_set_wait_limit.argtypes = [P, ctypes.c_uint64]
         L.kvk_decode_path_for.argtypes = [P, i32, i32, i32, i32, P]
         L.kvk_status_string.argtypes = [i32]
         L.kvk_status_string.restype = ctypes.c_char_p
@@ -239,6 +242,36 @@ def kvk_mla_decode(handle, layer, q_lat, q_rope, seq_lens, softmax_scale, out, w
     _check("kvk_mla_decode", st)
 
 
+def kvk_mla_decode_append(handle, layer, c_new, k_rope_new, q_lat, q_rope, seq_lens,
+                          softmax_scale, out, workspace, lse=None, stream=None):
+    """Append each sequence's new token (c_new [B, >=d], k_rope_new [B, d_rope], fp32 or bf16)
+    at position seq_lens[i] - 1 of the anchor layer's cache and decode over the cache that
+    includes it (one launch on the tensor-core kernel).  Other arguments as kvk_mla_decode."""
+    _need_cuda(c_new, "c_new", (torch.float32, torch.bfloat16))
+    _need_cuda(k_rope_new, "k_rope_new", (c_new.dtype,))
+    _need_cuda(q_lat, "q_lat", tuple(_DTYPE))
+    _need_cuda(q_rope, "q_rope", (q_lat.dtype,))
+    _need_cuda(seq_lens, "seq_lens", (torch.int32,))
+    _need_cuda(out, "out", (torch.float32,))
+    _need_cuda(lse, "lse", (torch.float32,))
+    _need_cuda(workspace, "workspace")
+    if c_new.dim() != 2 or k_rope_new.dim() != 2 or c_new.stride(1) != 1 or \
+            k_rope_new.stride(1) != 1:
+        raise ValueError("c_new / k_rope_new must be [batch, width] with contiguous width")
+    if q_lat.stride(2) != 1 or q_rope.stride(2) != 1:
+        raise ValueError("q_lat / q_rope last dim must be contiguous")
+    if not out.is_contiguous() or (lse is not None and not lse.is_contiguous()):
+        raise ValueError("out / lse must be contiguous")
+    B, H = q_lat.shape[0], q_lat.shape[1]
+    st = _lib_handle().kvk_mla_decode_append(
+        handle, layer, _ptr(c_new), _ptr(k_rope_new), _DTYPE[c_new.dtype], c_new.stride(0),
+        k_rope_new.stride(0), _ptr(q_lat), _ptr(q_rope), _DTYPE[q_lat.dtype], q_lat.stride(0),
+        q_lat.stride(1), q_rope.stride(0), q_rope.stride(1), B, H, _ptr(seq_lens),
+        float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("kvk_mla_decode_append", st)
+
+
 def kvk_mla_decode_noalloc(handle, layer, q_lat, q_rope, seq_lens, softmax_scale, out,
                            lse=None, keep_idx=None, keep_len=None, stream=None):
     """kvk_mla_decode with the library's built-in scratch instead of a workspace tensor,
@@ -277,6 +310,10 @@ def kvk_set_decode_path(handle, path):
 
 def kvk_set_decode_ctas(handle, ctas):
     _check("kvk_set_decode_ctas", _lib_handle().kvk_set_decode_ctas(handle, ctas))
+
+
+def kvk_set_wait_limit(handle, ns):
+    _check("kvk_set_wait_limit", _lib_handle().kvk_set_wait_limit(handle, int(ns)))
 
 
 def kvk_decode_path_for(handle, layer, dtype, n_heads, has_keep=False) -> int:
@@ -367,6 +404,18 @@ class Layout:
                        workspace, lse=lse, keep_idx=keep_idx, keep_len=keep_len, stream=stream)
         return out
 
+    def mla_decode_append(self, layer, c_new, k_rope_new, q_lat, q_rope, seq_lens, softmax_scale,
+                          out=None, lse=None, workspace=None, stream=None):
+        B, H = q_lat.shape[0], q_lat.shape[1]
+        d = self.layer_info(layer)["d"]
+        if out is None:
+            out = torch.empty(B, H, d, dtype=torch.float32, device=q_lat.device)
+        if workspace is None:
+            workspace = self.new_workspace(layer, B, H)
+        kvk_mla_decode_append(self.handle, layer, c_new, k_rope_new, q_lat, q_rope, seq_lens,
+                              softmax_scale, out, workspace, lse=lse, stream=stream)
+        return out
+
     def read_status(self, clear=False, stream=None):
         return kvk_read_status(self.handle, clear, stream)
 
@@ -375,6 +424,9 @@ class Layout:
 
     def set_decode_ctas(self, ctas):
         kvk_set_decode_ctas(self.handle, ctas)
+
+    def set_wait_limit(self, ns):
+        kvk_set_wait_limit(self.handle, ns)
 
     def decode_path_for(self, layer, dtype, n_heads, has_keep=False):
         return kvk_decode_path_for(self.handle, layer, dtype, n_heads, has_keep)

@@ -6,7 +6,8 @@
 Fills one anchor layer's cache through kvk_quant_write with seeded N(0,1) bf16 data, then
 runs kvk_mla_decode `iters` times and prints the mean device time per call (CUDA events on
 the launching stream, after warm-up) and the algorithmic bytes per second
-(batch * tokens * (row_bytes + 2) per call).  At the default shape the cache is ~300 MB,
+(batch * tokens * (row_bytes + 2) per call; b = 0, the uncompressed bf16 anchor, reads no
+scales).  At the default shape the cache is ~300 MB,
 larger than the 126 MB L2.
 
 --op write times the quantise-on-write of the whole cache instead (a prefill of batch x
@@ -89,7 +90,8 @@ def main():
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / args.iters
     row = lay.layer_info(0)["row_bytes"]
-    nbytes = B * T * (row + 2)
+    # rows and their scales (an uncompressed bf16 anchor, b = 0, reads no scale)
+    nbytes = B * T * (row + (0 if args.b == 0 else 2))
     path = lay.decode_path_for(0, torch.bfloat16, H)
     print(json.dumps({"d": args.d, "b": args.b, "heads": H, "batch": B, "tokens": T,
                       "path": {1: "tensor", 2: "cuda_core"}[path], "ms_per_call": round(ms, 5),

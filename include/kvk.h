@@ -20,6 +20,9 @@
  *     offending item and sets a sticky flag, read with kvk_read_status().
  *   - Every device pointer must be 16-byte aligned (the arena: 256-byte aligned), or the
  *     call returns KVK_ERR_ALIGNMENT.
+ *   - A layout belongs to the device that was current when it was created with an arena.
+ *     Every call that launches work (writes, decodes, kvk_read_status) must be made with
+ *     that device current; otherwise it returns KVK_ERR_INVALID_ARG and launches nothing.
  *   - Nothing here allocates device memory except kvk_create_layout's one synchronous
  *     cudaMemset of the arena header; nothing falls back to the CPU.
  */
@@ -62,6 +65,11 @@ typedef enum { KVK_F32 = 0, KVK_BF16 = 1, KVK_F16 = 2 } kvk_dtype;
 #define KVK_FLAG_TIMEOUT     0x10u /* decode: a tensor-core kernel wait exceeded its time limit and
                                       the kernel stopped early; that call's outputs are unspecified */
 
+/* Bit width of an anchor that keeps its cache uncompressed: rows of bfloat16 values (16 bits
+ * per element, no quantisation and no scale) -- the bf16 MLA cache the compressed choices are
+ * measured against.  Such an anchor costs (d + d_rope) * 16 bits per token. */
+#define KVK_BITS_BF16 0
+
 /* Decode kernel selection (kvk_set_decode_path). */
 #define KVK_PATH_AUTO      0 /* tensor-core kernel where it applies, else the CUDA-core kernel  */
 #define KVK_PATH_TENSOR    1 /* tcgen05 kernel only (KVK_ERR_UNSUPPORTED where it cannot run)   */
@@ -75,13 +83,15 @@ typedef enum { KVK_F32 = 0, KVK_BF16 = 1, KVK_F16 = 2 } kvk_dtype;
  * coordinates plus the d_rope-wide RoPE key) and the precision axis (b-bit symmetric
  * codes, one scale per token) -- "Three Non-Eviction Compression Axes"; and the budget
  * check of "Action Space and Cost Model" with the fp16 scale counted:
- *     bits_per_token = sum over anchors l of ((d_l + d_rope) * b_l + 16).
+ *     bits_per_token = sum over anchors l of ((d_l + d_rope) * b_l + 16)
+ * (an uncompressed bf16 anchor counts (d_l + d_rope) * 16).
  *
  *   n_layers            L >= 1
  *   anchor[L]           anchor[l] == l for an anchor; otherwise the largest l' < l with
  *                       anchor[l'] == l' (the nearest preceding anchor).  anchor[0] == 0.
- *   d[L], b[L]          for anchors: 16 <= d <= r, d % 16 == 0; b in {2, 4, 8, 16}.
- *                       Ignored for inheriting layers.
+ *   d[L], b[L]          for anchors: 16 <= d <= r, d % 16 == 0; b in {2, 4, 8, 16}, or
+ *                       KVK_BITS_BF16 (0) for an uncompressed bf16 anchor.  Ignored for
+ *                       inheriting layers.
  *   r, d_rope           latent width (multiple of 16) and RoPE width (multiple of 8, >= 0)
  *   max_batch, max_tokens  capacity of every anchor's cache (max_batch <= 4096,
  *                       max_batch * max_tokens < 2^31)
@@ -99,6 +109,9 @@ typedef enum { KVK_F32 = 0, KVK_BF16 = 1, KVK_F16 = 2 } kvk_dtype;
  * row_bytes = ceil((d + d_rope) * b / 8) rounded up to 16.
  * Packed row format: field u_i = code_i + 2^(b-1) (offset binary) at bit i*b of the row
  * read as a little-endian bit stream, i over [c[0..d) || k^R[0..d_rope)], zero padding.
+ * An uncompressed anchor (b = KVK_BITS_BF16) stores element i as the bfloat16 of v_i
+ * (round to nearest even) at bytes 2i, 2i+1 of the row, row_bytes = 2 (d + d_rope) rounded up
+ * to 16, and its scale plane holds 1.0 for every written token.
  */
 kvk_status kvk_create_layout(int n_layers, const int32_t* anchor, const int32_t* d,
                              const int32_t* b, int r, int d_rope, int max_batch, int max_tokens,
@@ -138,6 +151,7 @@ kvk_status kvk_get_layer_info(const kvk_layout* layout, int layer, kvk_layer_inf
  *     s = fp16(s32) rounded toward +inf, stored in the scale plane;
  *     code_i = clamp(round_half_even(v_i / s), -(2^(b-1)-1), 2^(b-1)-1) with the stored
  *     scale (IEEE fp32 division); s == 0 gives all-zero codes.
+ * An uncompressed anchor (KVK_BITS_BF16) stores bf16(v_i) instead, and the scale 1.0.
  * Token j (0 <= j < n_new) of sequence i (0 <= i < batch) goes to position
  * dev_start_pos[i] + j of sequence i's cache.
  *
@@ -225,6 +239,38 @@ kvk_status kvk_mla_decode(kvk_layout* layout, int layer, const void* q_lat, cons
                           kvk_stream_t stream);
 
 /*
+ * kvk_mla_decode_append -- one decode step of an anchor layer with its new token: quantise
+ * and store the token, then decode over the cache that includes it, in one launch where the
+ * tensor-core kernel runs ("Three Non-Eviction Compression Axes", item 3, applied to the
+ * token a decode step appends, followed by the decode of kvk_mla_decode).
+ *
+ * The result is the one of kvk_quant_write (n_new = 1, dev_start_pos[i] = seq_len_i - 1)
+ * followed by kvk_mla_decode over seq_len_i tokens: dev_seq_lens counts the new token.  In
+ * the tensor-core kernel the CTA that owns position seq_len_i - 1 writes the token before
+ * it loads that position; the CUDA-core kernel (fp32 queries, shapes the tensor-core kernel
+ * does not take) gets the write as a separate launch first.
+ *
+ *   layer        an anchor layer (an inheriting layer -> KVK_ERR_INHERITING_LAYER: its
+ *                anchor's step writes the token)
+ *   c_new        device [batch][>= d] at c_new[i * c_new_stride_seq + k]; dtype new_dtype
+ *                (KVK_BF16 or KVK_F32); k_rope_new [batch][d_rope] likewise.  Strides in
+ *                elements, multiples of 8.
+ *   dev_seq_lens clamped to [0, max_tokens] as in kvk_mla_decode; a sequence of length 0
+ *                appends nothing
+ *   the query, output and workspace arguments are those of kvk_mla_decode (no keep list:
+ *   with token eviction write with kvk_quant_write and decode with kvk_mla_decode).
+ */
+kvk_status kvk_mla_decode_append(kvk_layout* layout, int layer, const void* c_new,
+                                 const void* k_rope_new, int new_dtype, int64_t c_new_stride_seq,
+                                 int64_t k_rope_new_stride_seq, const void* q_lat,
+                                 const void* q_rope, int dtype, int64_t q_lat_stride_seq,
+                                 int64_t q_lat_stride_head, int64_t q_rope_stride_seq,
+                                 int64_t q_rope_stride_head, int batch, int n_heads,
+                                 const int32_t* dev_seq_lens, float softmax_scale, float* out,
+                                 float* lse, void* workspace, size_t workspace_bytes,
+                                 kvk_stream_t stream);
+
+/*
  * kvk_mla_decode_noalloc -- kvk_mla_decode without a caller-provided workspace.
  *
  * The paper has no counterpart to this entry point; it exists for callers that cannot
@@ -236,19 +282,23 @@ kvk_status kvk_mla_decode(kvk_layout* layout, int layer, const void* q_lat, cons
  * which every GPU that loads the library holds until the process exits.
  *
  * Arguments and results are those of kvk_mla_decode minus (workspace, workspace_bytes).
- * A call whose workspace need (kvk_decode_workspace_bytes) exceeds
- * KVK_NOALLOC_SCRATCH_BYTES returns KVK_ERR_WORKSPACE and launches nothing.  A call with a
- * keep list takes the tensor-core kernel only if the scratch also holds the dense copy of
- * the kept rows (kvk_decode_workspace_bytes_keep <= KVK_NOALLOC_SCRATCH_BYTES), else the
- * CUDA-core kernel.  This entry
- * point allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ * The call takes the kernel kvk_mla_decode would take (kvk_decode_path_for) and needs, for
+ * that kernel, the workspace kvk_mla_decode needs; when that exceeds
+ * KVK_NOALLOC_SCRATCH_BYTES it returns KVK_ERR_WORKSPACE and launches nothing.  (The
+ * tensor-core kernel needs (G + batch) * n_heads * (d + 2) * 4 bytes plus a little, G the
+ * SM count; kvk_decode_workspace_bytes, which covers both kernels, can be larger.)  A call
+ * with a keep list takes the tensor-core kernel only if the scratch also holds the dense
+ * copy of the kept rows, else the CUDA-core kernel.  This entry point allocates nothing: no
+ * cudaMalloc, no cudaFree, no allocating library routine.
  *
- * Set-up: the first call on a device (the device current at the call) looks up the
- * array's device address with cudaGetSymbolAddress and caches it; make that first call
- * before any stream capture.  All calls share the one array and it keeps the previous
- * call's contents (no part of it needs to start at zero), so calls whose executions
- * overlap on the GPU -- on different streams, or from different host threads -- race on
- * it and give undefined results; order them on one stream or serialise them.
+ * Set-up: the first call on a device (the layout's device, which must be current) looks
+ * up the array's device address with cudaGetSymbolAddress and caches it per device; make
+ * that first call before any stream capture.  The cached address is that of the library's
+ * module in the device's primary context: after cudaDeviceReset it is stale, and calls
+ * made after a reset are unsupported.  All calls share the one array and it keeps the
+ * previous call's contents (no part of it needs to start at zero), so calls whose
+ * executions overlap on the GPU -- on different streams, or from different host threads --
+ * race on it and give undefined results; order them on one stream or serialise them.
  */
 #define KVK_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 
@@ -270,6 +320,14 @@ kvk_status kvk_read_status(kvk_layout* layout, uint32_t* flags, int clear, kvk_s
  * the same definition. */
 kvk_status kvk_set_decode_path(kvk_layout* layout, int path);
 kvk_status kvk_set_decode_ctas(kvk_layout* layout, int ctas);
+
+/* Failure detection of the tensor-core decode: every wait inside the kernel (for a tile to
+ * land, for a stage of the pipeline to finish) gives up after `ns` nanoseconds; the kernel
+ * then sets KVK_FLAG_TIMEOUT, lets its own loads and tensor-core operations finish, and
+ * exits, so the stream and the context stay usable and the call's outputs are unspecified.
+ * ns = 0 restores the default limit of 2 s.  A short limit (microseconds) makes a wait run
+ * out on purpose, to exercise that path. */
+kvk_status kvk_set_wait_limit(kvk_layout* layout, uint64_t ns);
 
 /* Which kernel kvk_mla_decode would run for these arguments (KVK_PATH_TENSOR or
  * KVK_PATH_CUDA_CORE), without launching anything.  has_keep != 0: a keep list is given;

@@ -124,6 +124,54 @@ uint16_t kvko_f32_to_f16_ru(float xf)
 }
 
 /* ------------------------------------------------------------------------ */
+/* bfloat16, for the uncompressed cache the compressed one is measured        */
+/* against: 1 sign bit, 8 exponent bits, 7 fraction bits, i.e. exactly the     */
+/* binary32 values whose low 16 bits are zero.                                */
+/* ------------------------------------------------------------------------ */
+
+double kvko_bf16_to_f64(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* binary32 -> bfloat16, round to nearest, ties to even: of the two bf16 values
+ * that bracket x (truncation of the low 16 bits, and the next one away from
+ * zero), take the nearer in exact arithmetic; on a tie the one whose last
+ * fraction bit is 0.  The next value past the largest finite one is +-inf,
+ * reached (as in IEEE arithmetic) from half an ulp beyond the largest. */
+uint16_t kvko_f32_to_bf16_rne(float x)
+{
+    if (isnan(x)) return 0x7FC0;
+    uint32_t u;
+    memcpy(&u, &x, sizeof u);
+    if ((u & 0x7FFFFFFFu) >= 0x7F800000u) return (uint16_t)(u >> 16);   /* +-inf */
+    uint32_t lo_bits = u & 0xFFFF0000u, hi_bits = lo_bits + 0x10000u;
+    float lo, hi;
+    memcpy(&lo, &lo_bits, sizeof lo);
+    double dlo = (double)lo, dhi;
+    if ((hi_bits & 0x7FFFFFFFu) == 0x7F800000u) {
+        dhi = ldexp(1.0, 128);                   /* where +-inf sits in the rounding rule */
+        if (signbit(x)) dhi = -dhi;
+    } else {
+        memcpy(&hi, &hi_bits, sizeof hi);
+        dhi = (double)hi;
+    }
+    double dx = (double)x;
+    double elo = fabs(dx - dlo), ehi = fabs(dhi - dx);
+    if (elo < ehi) return (uint16_t)(lo_bits >> 16);
+    if (ehi < elo) return (uint16_t)(hi_bits >> 16);
+    return ((lo_bits >> 16) & 1u) ? (uint16_t)(hi_bits >> 16) : (uint16_t)(lo_bits >> 16);
+}
+
+void kvko_bf16_round(const float* v, int64_t n, uint16_t* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = kvko_f32_to_bf16_rne(v[i]);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Quantiser (R1-R3): one token vector v[0..n) -> fp16 scale + integer codes  */
 /* ------------------------------------------------------------------------ */
 
@@ -261,14 +309,19 @@ void kvko_attend(const double* q_lat, const double* q_rope, const double* rows,
 /* ------------------------------------------------------------------------ */
 
 /* Bits per token of a plan: anchors pay (d+d_R)*b (+16 for the fp16 scale
- * when with_scale != 0); inheriting layers pay 0. */
+ * when with_scale != 0); inheriting layers pay 0.  b = 0 marks an anchor kept
+ * uncompressed in bfloat16 (the cache C_0's 16 bits per element, no scale): it
+ * pays (d+d_R)*16. */
 int64_t kvko_bits_per_token(int n_layers, const int32_t* anchor, const int32_t* d,
                             const int32_t* b, int d_R, int with_scale)
 {
     int64_t s = 0;
     for (int l = 0; l < n_layers; ++l) {
         if (anchor[l] != l) continue;
-        s += (int64_t)(d[l] + d_R) * b[l] + (with_scale ? 16 : 0);
+        if (b[l] == 0)
+            s += (int64_t)(d[l] + d_R) * 16;
+        else
+            s += (int64_t)(d[l] + d_R) * b[l] + (with_scale ? 16 : 0);
     }
     return s;
 }

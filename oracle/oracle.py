@@ -62,6 +62,11 @@ def lib():
         L.kvko_c0_bits.argtypes = [i32, i32, i32]
         L.kvko_c0_bits.restype = i64
         L.kvko_num_threads.restype = i32
+        L.kvko_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        L.kvko_bf16_to_f64.restype = f64
+        L.kvko_f32_to_bf16_rne.argtypes = [ctypes.c_float]
+        L.kvko_f32_to_bf16_rne.restype = ctypes.c_uint16
+        L.kvko_bf16_round.argtypes = [P, i64, P]
         _lib = L
     return _lib
 
@@ -195,6 +200,32 @@ def quantize_rows(c_kv: np.ndarray, k_rope: np.ndarray, d: int, b: int):
     v = token_vectors(c_kv, k_rope, d)
     scales, codes = quantize(v, b)
     return pack(codes, b), scales, codes
+
+
+def f32_to_bf16_rne(x: float) -> int:
+    """binary32 -> bfloat16 bit pattern, round to nearest, ties to even."""
+    return int(lib().kvko_f32_to_bf16_rne(float(np.float32(x))))
+
+
+def bf16_bits_to_f64(h: int) -> float:
+    return lib().kvko_bf16_to_f64(int(h))
+
+
+def bf16_rows(c_kv: np.ndarray, k_rope: np.ndarray, d: int):
+    """The uncompressed cache of one sequence: the token vectors [c[:d] || k^R] stored as
+    bfloat16 (round to nearest even).  Returns (bits uint16 [T, n], values float64 [T, n])."""
+    v = token_vectors(c_kv, k_rope, d)
+    bits = np.zeros(v.shape, dtype=np.uint16)
+    lib().kvko_bf16_round(_p(v), v.size, _p(bits))
+    return bits, bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def decode_sequence_bf16(q_lat, q_rope, values, d: int, sigma: float, tok=None):
+    """Attention of one sequence over its uncompressed (bf16) cache rows `values` [T, n]."""
+    T = values.shape[0]
+    if tok is None:
+        tok = np.arange(T, dtype=np.int32)
+    return attend(np.asarray(q_lat, dtype=np.float64)[:, :d], q_rope, values, tok, sigma)
 
 
 def decode_sequence(q_lat, q_rope, codes, scales, d: int, sigma: float, tok=None):

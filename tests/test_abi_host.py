@@ -65,8 +65,8 @@ def test_table_validation(kvk):
     # d not a multiple of 16, d > r, d < 16
     for dd in (24, 80, 0):
         assert _status(kvk, [0], [dd], [8], 64, 16, 1, 256, query_only=True) == 2
-    # b outside {2, 4, 8, 16}
-    for bb in (1, 3, 5, 32):
+    # b outside {2, 4, 8, 16} and the uncompressed bf16 anchor (0)
+    for bb in (1, 3, 5, 32, -1):
         assert _status(kvk, [0], [32], [bb], 64, 16, 1, 256, query_only=True) == 2
     # bad dims
     assert _status(kvk, [0], [32], [8], 60, 16, 1, 256, query_only=True) == 1
@@ -148,3 +148,25 @@ def test_planning_layout_cannot_launch(kvk):
         del torch
     finally:
         kvk.kvk_destroy(handle)
+
+
+def test_uncompressed_bf16_anchor_layout(kvk, oracle_mod):
+    """b = 0 keeps an anchor uncompressed in bf16: 16 bits per element and no scale in the
+    cost (the same as the oracle's cost model), 2 bytes per element in the row."""
+    anchor, d, b = [0, 0, 2, 3], [512, 0, 256, 128], [0, 0, 0, 4]
+    _, need, bits = kvk.kvk_create_layout(anchor, d, b, 512, 64, 2, 64, query_only=True)
+    assert bits == (512 + 64) * 16 + (256 + 64) * 16 + (128 + 64) * 4 + 16
+    assert bits == oracle_mod.bits_per_token(anchor, d, b, 64)
+    lay, _, _ = kvk.kvk_create_layout(anchor, d, b, 512, 64, 2, 64)
+    try:
+        assert kvk.kvk_get_layer_info(lay, 0)["row_bytes"] == (512 + 64) * 2
+        assert kvk.kvk_get_layer_info(lay, 2)["row_bytes"] == (256 + 64) * 2
+        assert kvk.kvk_get_layer_info(lay, 3)["row_bytes"] == (128 + 64) * 4 // 8
+        assert kvk.kvk_get_layer_info(lay, 1)["b"] == 0
+    finally:
+        kvk.kvk_destroy(lay)
+    # a 14B-shaped plan kept wholly uncompressed costs C_0 * 576 / 2048 (48 layers of
+    # 576 bf16 elements against 48 layers of 2 x 8 x 128 bf16 keys and values)
+    c0 = oracle_mod.c0_bits(48, 8, 128)
+    full = oracle_mod.bits_per_token(list(range(48)), [512] * 48, [0] * 48, 64)
+    assert full * 2048 == c0 * 576

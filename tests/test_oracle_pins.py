@@ -326,18 +326,6 @@ def test_full_width_16_bit_cache_matches_unquantised_attention(oracle_mod):
     np.testing.assert_allclose(lse, ref_lse, atol=1e-3)
 
 
-def test_inheriting_layer_reads_anchor_cache(oracle_mod):
-    """Depth axis: a layer that inherits uses its anchor's rows; same query -> same output."""
-    rng = np.random.default_rng(10)
-    c = rng.standard_normal((40, 64)).astype(np.float32)
-    kr = rng.standard_normal((40, 16)).astype(np.float32)
-    _, s, k = oracle_mod.quantize_rows(c, kr, 32, 8)
-    q_lat, q_rope = rng.standard_normal((4, 64)), rng.standard_normal((4, 16))
-    a = oracle_mod.decode_sequence(q_lat, q_rope, k, s, 32, 0.1)
-    b = oracle_mod.decode_sequence(q_lat, q_rope, k.copy(), s.copy(), 32, 0.1)
-    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
-
-
 # --------------------------------------------------------------------------
 # cost model
 # --------------------------------------------------------------------------
@@ -384,3 +372,73 @@ def test_workload_tables_meet_their_budgets(oracle_mod):
             assert bits == t["bits_per_token"]
             full = len(a) * ((512 + 64) * 16 + 16)
             assert bits <= t["budget_bits"] or (bits == full and t["budget_bits"] >= full)
+
+
+# --------------------------------------------------------------------------
+# the uncompressed (bfloat16) cache the compressed one is measured against
+# --------------------------------------------------------------------------
+
+def _bf16_value(h):
+    return float(np.array([int(h) << 16], dtype=np.uint32).view(np.float32)[0])
+
+
+def test_bf16_rounding_is_nearest_even_by_search(oracle_mod):
+    """binary32 -> bfloat16: no other bfloat16 value of the same sign is nearer to x (exact
+    binary64 arithmetic over the neighbouring patterns), and exact ties go to an even last
+    fraction bit.  Includes constructed ties, subnormals, and values next to the largest."""
+    rng = np.random.default_rng(21)
+    xs = list(rng.standard_normal(2000).astype(np.float32))
+    xs += list((rng.standard_normal(500) * 2.0 ** rng.integers(-140, 120, 500)).astype(np.float32))
+    for h in (0x3F80, 0x3F81, 0x0001, 0x0080, 0x7F7E, 0x7F7F, 0x4049):
+        lo, hi = _bf16_value(h), _bf16_value(h + 1)
+        xs.append(np.float32((lo + hi) / 2))         # exact tie
+        xs.append(np.nextafter(np.float32((lo + hi) / 2), np.float32(np.inf)))
+        xs.append(np.nextafter(np.float32((lo + hi) / 2), np.float32(-np.inf)))
+        xs.append(-np.float32((lo + hi) / 2))
+    for x in xs:
+        x = np.float32(x)
+        if not np.isfinite(x):
+            continue
+        h = oracle_mod.f32_to_bf16_rne(float(x))
+        y = _bf16_value(h)
+        if np.isinf(y):          # overflow: x is at least half an ulp beyond the largest
+            assert abs(float(x)) >= _bf16_value(0x7F7F) + 2.0 ** (127 - 8)
+            continue
+        e = abs(float(x) - y)
+        sign = h & 0x8000
+        for k in (-2, -1, 1, 2):
+            hk = ((h & 0x7FFF) + k)
+            if 0 <= hk < 0x7F80:
+                ek = abs(float(x) - _bf16_value(sign | hk))
+                assert e <= ek, (float(x), hex(h), k)
+                if e == ek:
+                    assert (h & 1) == 0, (float(x), hex(h))
+
+
+def test_bf16_rounding_matches_torch(oracle_mod):
+    """The same conversion as torch's round-to-nearest-even bfloat16 cast (an implementation
+    the oracle does not call) on a million values of mixed magnitude."""
+    rng = np.random.default_rng(22)
+    x = (rng.standard_normal(1 << 20) * 2.0 ** rng.integers(-130, 127, 1 << 20)).astype(np.float32)
+    x[:4] = [0.0, -0.0, 1.0, -3.0]
+    bits = np.zeros(x.shape, dtype=np.uint16)
+    oracle_mod.lib().kvko_bf16_round(x.ctypes.data, x.size, bits.ctypes.data)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bits, ref)
+
+
+def test_bf16_cache_attention_equals_attention_on_the_rounded_rows(oracle_mod):
+    """For bfloat16 inputs the uncompressed cache holds them exactly, so its attention is
+    plain MLA attention on the inputs (torch SDPA in float64)."""
+    rng = np.random.default_rng(23)
+    T, r, dR, H = 300, 64, 16, 6
+    c = torch.from_numpy(rng.standard_normal((T, r)).astype(np.float32)).to(torch.bfloat16)
+    kr = torch.from_numpy(rng.standard_normal((T, dR)).astype(np.float32)).to(torch.bfloat16)
+    ql, qr = rng.standard_normal((H, r)), rng.standard_normal((H, dR))
+    bits, vals = oracle_mod.bf16_rows(c.float().numpy(), kr.float().numpy(), r)
+    exact = np.concatenate([c.float().numpy(), kr.float().numpy()], 1).astype(np.float64)
+    assert np.array_equal(vals, exact)
+    out, lse = oracle_mod.decode_sequence_bf16(ql, qr, vals, r, 0.125)
+    ref, ref_lse = _sdpa(ql, qr, exact, r, 0.125)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
