@@ -131,13 +131,18 @@ const char* kvk_status_string(kvk_status s) {
   return "unknown status";
 }
 
-kvk_status kvk_create_layout(int n_layers, const int32_t* anchor, const int32_t* d,
-                             const int32_t* b, int r, int d_rope, int max_batch, int max_tokens,
-                             int64_t budget_bits_per_token, void* dev_arena, size_t arena_bytes,
-                             kvk_layout** out, size_t* arena_bytes_needed,
-                             int64_t* bits_per_token) {
+}  // extern "C"
+
+// Layout with one fp16 scale per `group` consecutive elements of every quantised anchor's
+// row (group = 0: one scale per token).
+static kvk_status create_layout_impl(int n_layers, const int32_t* anchor, const int32_t* d,
+                                     const int32_t* b, int r, int d_rope, int group,
+                                     int max_batch, int max_tokens, int64_t budget_bits_per_token,
+                                     void* dev_arena, size_t arena_bytes, kvk_layout** out,
+                                     size_t* arena_bytes_needed, int64_t* bits_per_token) {
   if (out) *out = nullptr;
   if (n_layers < 1 || n_layers > 65536 || !anchor || !d || !b) return KVK_ERR_INVALID_ARG;
+  if (group != 0 && group != 16 && group != 32 && group != 64) return KVK_ERR_INVALID_ARG;
   if (r < 16 || r % 16 != 0 || d_rope < 0 || d_rope % 8 != 0) return KVK_ERR_INVALID_ARG;
   if (max_batch < 1 || max_batch > 4096 || max_tokens < 1) return KVK_ERR_INVALID_ARG;
   if ((int64_t)max_batch * (int64_t)max_tokens >= (int64_t(1) << 31)) return KVK_ERR_INVALID_ARG;
@@ -153,8 +158,12 @@ kvk_status kvk_create_layout(int n_layers, const int32_t* anchor, const int32_t*
       if (b[l] != 2 && b[l] != 4 && b[l] != 8 && b[l] != 16 && b[l] != KVK_BITS_BF16)
         return KVK_ERR_BAD_TABLE;
       if (d[l] + d_rope > kvk::kMaxRowElems) return KVK_ERR_UNSUPPORTED;
-      bits += (b[l] == KVK_BITS_BF16) ? (int64_t)(d[l] + d_rope) * 16
-                                      : (int64_t)(d[l] + d_rope) * b[l] + 16;
+      const int n = d[l] + d_rope;
+      if (group && b[l] != KVK_BITS_BF16 && n % group != 0) return KVK_ERR_BAD_TABLE;
+      if (b[l] == KVK_BITS_BF16)
+        bits += (int64_t)n * 16;
+      else
+        bits += (int64_t)n * b[l] + (group ? (int64_t)16 * (n / group) : 16);
       last = l;
     } else {
       if (l == 0 || anchor[l] != last) return KVK_ERR_BAD_TABLE;
@@ -169,11 +178,13 @@ kvk_status kvk_create_layout(int n_layers, const int32_t* anchor, const int32_t*
   tmp.d_rope = d_rope;
   tmp.max_batch = max_batch;
   tmp.max_tokens = max_tokens;
+  tmp.group = group;
   tmp.anchor.assign(anchor, anchor + n_layers);
   tmp.d.assign(d, d + n_layers);
   tmp.b.assign(b, b + n_layers);
   tmp.slot.assign(n_layers, -1);
   size_t off = kvk::kArenaHeader;
+  int max_sg = 1;
   const size_t tokens = (size_t)max_batch * (size_t)max_tokens;
   for (int l = 0; l < n_layers; ++l) {
     if (anchor[l] == l) {
@@ -183,19 +194,22 @@ kvk_status kvk_create_layout(int n_layers, const int32_t* anchor, const int32_t*
       A.b = b[l];
       A.n = d[l] + d_rope;
       A.row_bytes = row_bytes_of(A.n, A.b == KVK_BITS_BF16 ? 16 : A.b);
+      A.sg = (group && A.b != KVK_BITS_BF16) ? A.n / group : 1;
+      max_sg = std::max(max_sg, A.sg);
       off = align_up(off, kAlign);
       A.codes_off = (int64_t)off;
       off += tokens * (size_t)A.row_bytes;
       off = align_up(off, kAlign);
       A.scales_off = (int64_t)off;
-      off += tokens * sizeof(__half);
+      off += tokens * (size_t)A.sg * sizeof(__half);
       tmp.anchors.push_back(A);
     }
     tmp.slot[l] = (int)tmp.anchors.size() - 1;
   }
-  // tail slack: the tensor-core decode reads each tile's token scales as a 144-byte window
-  // from the 16-byte boundary at or below the first one, up to 16 bytes past a scale plane
-  off = align_up(off, kAlign) + kAlign;
+  // tail slack: the tensor-core decode reads each tile's scales (64 tokens) as one window from
+  // the 16-byte boundary at or below the first, which can reach past the last scale plane by
+  // up to 64 tokens' scales and 32 bytes
+  off = align_up(off, kAlign) + align_up((size_t)64 * max_sg * sizeof(__half) + 32, kAlign);
   if (arena_bytes_needed) *arena_bytes_needed = off;
   if (budget_bits_per_token > 0 && bits > budget_bits_per_token) return KVK_ERR_BUDGET;
   if (!out) return KVK_OK;  // query mode
@@ -228,6 +242,30 @@ kvk_status kvk_create_layout(int n_layers, const int32_t* anchor, const int32_t*
   return KVK_OK;
 }
 
+extern "C" {
+
+kvk_status kvk_create_layout(int n_layers, const int32_t* anchor, const int32_t* d,
+                             const int32_t* b, int r, int d_rope, int max_batch, int max_tokens,
+                             int64_t budget_bits_per_token, void* dev_arena, size_t arena_bytes,
+                             kvk_layout** out, size_t* arena_bytes_needed,
+                             int64_t* bits_per_token) {
+  return create_layout_impl(n_layers, anchor, d, b, r, d_rope, 0, max_batch, max_tokens,
+                            budget_bits_per_token, dev_arena, arena_bytes, out,
+                            arena_bytes_needed, bits_per_token);
+}
+
+kvk_status kvk_create_layout_grouped(int n_layers, const int32_t* anchor, const int32_t* d,
+                                     const int32_t* b, int r, int d_rope, int scale_group,
+                                     int max_batch, int max_tokens,
+                                     int64_t budget_bits_per_token, void* dev_arena,
+                                     size_t arena_bytes, kvk_layout** out,
+                                     size_t* arena_bytes_needed, int64_t* bits_per_token) {
+  if (scale_group == 0) return KVK_ERR_INVALID_ARG;
+  return create_layout_impl(n_layers, anchor, d, b, r, d_rope, scale_group, max_batch,
+                            max_tokens, budget_bits_per_token, dev_arena, arena_bytes, out,
+                            arena_bytes_needed, bits_per_token);
+}
+
 void kvk_destroy(kvk_layout* L) { delete L; }
 
 kvk_status kvk_get_layer_info(const kvk_layout* L, int layer, kvk_layer_info* info) {
@@ -245,6 +283,8 @@ kvk_status kvk_get_layer_info(const kvk_layout* L, int layer, kvk_layer_info* in
   info->max_tokens = L->max_tokens;
   info->r = L->r;
   info->d_rope = L->d_rope;
+  info->scales_per_token = A.sg;
+  info->scale_group = A.sg > 1 ? L->group : 0;
   return KVK_OK;
 }
 
@@ -311,6 +351,7 @@ kvk_status kvk_quant_write_layers(kvk_layout* L, int n, const int32_t* layers,
     q.row_bytes = A.row_bytes;
     q.d = A.d;
     q.b = A.b;
+    q.group = kvk::anchor_group(L, A);
     q.c_kv = c_kv[k];
     q.c_ss = c_stride_seq[k];
     q.c_st = c_stride_tok[k];
@@ -353,7 +394,7 @@ kvk_status kvk_decode_workspace_bytes_keep(const kvk_layout* L, int layer, int b
   kvk_status st = kvk_decode_workspace_bytes(L, layer, batch, n_heads, &base);
   if (st != KVK_OK) return st;
   const AnchorDesc& A = L->anchors[L->slot[layer]];
-  *bytes = align_up(base, kAlign) + kvk::compact_workspace_bytes(batch, keep_stride, A.row_bytes);
+  *bytes = align_up(base, kAlign) + kvk::compact_workspace_bytes(batch, keep_stride, A.row_bytes, A.sg);
   return KVK_OK;
 }
 
@@ -431,10 +472,10 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
     const int Gt = kvk::decode_ctas(L, batch, KVK_PATH_TENSOR);
     keep_off = align_up(kvk::decode_workspace(batch, n_heads, A.d, Gt, nullptr, nullptr), kAlign);
     const bool room =
-        workspace_bytes >= keep_off + kvk::compact_workspace_bytes(batch, keep_stride, A.row_bytes);
+        workspace_bytes >= keep_off + kvk::compact_workspace_bytes(batch, keep_stride, A.row_bytes, A.sg);
     kvk::CompactArgs probe;
     if (room) kvk::compact_carve(static_cast<uint8_t*>(workspace) + keep_off, batch, keep_stride,
-                                 A.row_bytes, &probe);
+                                 A.row_bytes, A.sg, &probe);
     const bool ok = room && keep_stride > 0 &&
                     make_codes_tmap(&keep_tmap, probe.dst_codes, (int64_t)batch * keep_stride,
                                     A.row_bytes, A.b, kvk::kTcTileTokens);
@@ -471,6 +512,8 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
   a.lse = lse;
   a.flags = reinterpret_cast<uint32_t*>(L->arena);
   a.limit_ns = L->wait_limit_ns ? L->wait_limit_ns : kvk::kDefaultWaitLimitNs;
+  a.group = kvk::anchor_group(L, A);
+  a.sg = A.sg;
   int G = kvk::decode_ctas(L, batch, path);
   size_t need = kvk::decode_workspace(batch, n_heads, A.d, G, workspace, &a);
   if (workspace_bytes < need) return KVK_ERR_WORKSPACE;
@@ -491,7 +534,7 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
     c.keep_stride = keep_stride;
     c.flags = a.flags;
     kvk::compact_carve(static_cast<uint8_t*>(workspace) + keep_off, batch, keep_stride,
-                       A.row_bytes, &c);
+                       A.row_bytes, A.sg, &c);
     e = kvk::launch_compact(c, batch, st);
     // the decode proper: the dense copy as a cache of keep_stride rows per sequence
     a.codes = c.dst_codes;

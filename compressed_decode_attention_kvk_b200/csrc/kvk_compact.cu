@@ -89,22 +89,27 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(CompactArgs c)
     for (int u = 0; u < kCopyUnroll; ++u)
       if (e0 + u * kCompactThreads < nw) dst[to[u]] = v[u];
   }
-  for (int r = tid; r < total; r += kCompactThreads)
-    c.dst_scales[dst_seq + r] = c.scales[src_seq + s_tok[r]];
+  // the rows' scales: one per token, or sg per token in a group-scaled cache
+  for (int e = tid; e < total * c.sg; e += kCompactThreads) {
+    const int r = e / c.sg, j = e - r * c.sg;
+    c.dst_scales[(dst_seq + r) * c.sg + j] = c.scales[(src_seq + s_tok[r]) * c.sg + j];
+  }
 }
 
 }  // namespace
 
-size_t compact_workspace_bytes(int batch, int keep_stride, int row_bytes) {
+size_t compact_workspace_bytes(int batch, int keep_stride, int row_bytes, int sg) {
   size_t off = align_up_sz(sizeof(int32_t) * (size_t)batch, 256);
   off = align_up_sz(off + (size_t)batch * (size_t)keep_stride * (size_t)row_bytes, 256);
-  // fp16 scales, plus slack: the decode reads each tile's scales as one 144-byte window from
-  // the 16-byte boundary at or below the tile's first scale
-  off = align_up_sz(off + (size_t)batch * (size_t)keep_stride * 2 + 256, 256);
+  // fp16 scales (sg per token), plus slack: the decode reads each tile's scales as one window
+  // from the 16-byte boundary at or below the tile's first scale, up to 64 tokens' scales and
+  // 32 bytes past the last kept row
+  off = align_up_sz(off + (size_t)batch * (size_t)keep_stride * 2 * sg + 64 * 2 * sg + 32, 256);
   return off;
 }
 
-void compact_carve(void* base, int batch, int keep_stride, int row_bytes, CompactArgs* c) {
+void compact_carve(void* base, int batch, int keep_stride, int row_bytes, int sg, CompactArgs* c) {
+  c->sg = sg;
   uint8_t* p = static_cast<uint8_t*>(base);
   c->cnt = reinterpret_cast<int32_t*>(p);
   size_t off = align_up_sz(sizeof(int32_t) * (size_t)batch, 256);

@@ -109,7 +109,8 @@ __global__ void __launch_bounds__(kHG * 32) decode_fma_kernel(DecodeArgs a) {
         if (tid < TT) {
           int t = (tid < cnt) ? token_at(a, seq, p + tid, seq_len) : -1;
           tokidx[tid] = t;
-          ss[tid] = (t >= 0) ? __half2float(a.scales[seq_row0 + t]) : 0.0f;
+          // a group-scaled cache carries its scales per element (below): unit token scale
+          ss[tid] = (t >= 0) ? (a.group ? 1.0f : __half2float(a.scales[seq_row0 + t])) : 0.0f;
         }
         __syncthreads();
         for (int e = tid; e < TT * n; e += nt) {
@@ -123,6 +124,7 @@ __global__ void __launch_bounds__(kHG * 32) decode_fma_kernel(DecodeArgs a) {
             const uint32_t w = __ldg(row + (bit >> 5));
             const uint32_t u = (w >> (bit & 31)) & mask;
             v = bf16_rows ? __uint_as_float(u << 16) : (float)((int)u - zero_off);
+            if (a.group) v *= __half2float(a.scales[(seq_row0 + t) * a.sg + k / a.group]);
           }
           cs[i * ldc + k] = v;
         }

@@ -23,7 +23,7 @@
 //   warp 15    warms L2 with the queries of the CTA's later pieces
 // Launched with 128 registers per thread; the softmax warpgroup raises its budget to
 // kRegsSoftmax, the conversion warpgroups lower theirs to kRegsConvert and the last
-// warpgroup to kRegsIssue (4 x 32 x (192 + 2 x 120 + 56) = 62464 <= 65536).
+// warpgroup to kRegsIssue (4 x 32 x (192 + 2 x 120 + 80) = 65536).
 // Per tile:  S^T[64 tok x N1 heads]  = C[64 x n] . Q^T         (M=64, A in smem, TMEM f32)
 //            O^T[128 feat x N2 heads] += C^T[128 x 64] . P    (M=128 per 128 latent features,
 //                                                               A = C^T in TMEM)
@@ -65,7 +65,7 @@ constexpr int kMma2Warp = 14;  // output MMAs
 // above it raises it (setmaxnreg.inc), one below lowers it (.dec) -- never the other way,
 // which would be an illegal instruction -- and the budgets sum to no more than the launch.
 constexpr uint32_t kLaunchRegs = 65536 / kThreads;   // 128
-constexpr uint32_t kRegsSoftmax = 192, kRegsConvert = 120, kRegsIssue = 56;
+constexpr uint32_t kRegsSoftmax = 192, kRegsConvert = 120, kRegsIssue = 80;
 static_assert(128 * (kRegsSoftmax + 2 * kRegsConvert + kRegsIssue) <= 65536, "register split");
 // 16-bit rows (int16 codes, or the bf16 values of an uncompressed anchor) are converted in
 // place in the slot the tensor memory accelerator filled; narrower codes go through a raw ring
@@ -89,10 +89,10 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kSmemLimit = 232448;
 constexpr int kQC = 3;   // 16-byte chunks per lane per query row (rows of up to 768 features)
 constexpr int kQD = 1;   // query rows in flight per convert warp while staging
-// Token-scale ring: per tile a 144-byte window (the tile's 64 fp16 scales from the 16-byte
-// boundary at or below the first), loaded by the TMA warp with a plain bulk copy.
+// Scale ring: per tile one window of the tile's fp16 scales (64 tokens x sg scales, from the
+// 16-byte boundary at or below the first, rounded up to 16 bytes: 144 bytes for one scale per
+// token), loaded by the TMA warp with a plain bulk copy.
 constexpr int kScSlots = 4;
-constexpr uint32_t kScBytes = 144;
 // barriers besides the rings: s full/empty, P full/empty (2), C^T full/empty (2), q full/empty,
 // o empty, two MMA drains, q seen, appended, scale full/empty (kScSlots each)
 constexpr int kFixedBars = 2 + 4 + 4 + 7 + 2 * kScSlots;
@@ -103,15 +103,18 @@ struct TcParams {
   int NP, NPd;          // 128-feature groups per row, and those holding latent features
   int NQA, NK16;        // 64-feature query atoms, 16-feature K steps
   int PR, RR, raw_slot; // ring slots (f16 groups, packed groups) and packed-group bytes
+  int LR;               // 16-bit codes: slots of the low parts (code - f16(code)) of a group
+  uint32_t off_lo;
   uint32_t lbo_p;       // bytes between the 8-token core-matrix rows of P (16 N2 + 32)
   uint32_t p_bytes;     // one P buffer: 8 lbo_p
   uint32_t off_p, off_pairs, off_raw, off_bar, off_misc;
   uint32_t idesc1, idesc2;
   int qdtype;           // KVK_BF16 or KVK_F16
+  uint32_t off_sc, sc_bytes;   // scale windows: ring offset and bytes per window (0: none)
+  int grouped;          // scales per element group, applied by the convert warps
 };
 
 struct Misc {
-  alignas(16) uint8_t sc[kScSlots][kScBytes];   // token-scale windows
   uint32_t tmem_base;
   int abort;
   float qs_inv[2][64];   // per piece parity and head: 2^-e of the staged query row
@@ -203,6 +206,18 @@ __device__ __forceinline__ uint32_t cvt_code16(uint32_t w) {
   const __half2 ls = __hsub2(bits_h2(__byte_perm(w, 0x64u, 0x4240u)), __float2half2_rn(1024.f));
   return h2_bits(__hfma2(hs, __float2half2_rn(256.f), ls));
 }
+// The same codes split exactly into two f16 parts, hi = f16(code) (rounded to nearest) and
+// lo = code - hi: with hb, lb the code's bytes (exact in f16), t = (hb - 128) * 256 - hi is an
+// integer of magnitude <= 263 (so the fused multiply-add is exact), and lo = t + lb an integer
+// of magnitude <= 8 (f16 spacing is at most 16 below 2^15): q . code = q . hi + q . lo exactly.
+__device__ __forceinline__ void cvt_code16_split(uint32_t w, uint32_t& hi, uint32_t& lo) {
+  const __half2 hs = __hsub2(bits_h2(__byte_perm(w, 0x64u, 0x4341u)), __float2half2_rn(1152.f));
+  const __half2 ls = __hsub2(bits_h2(__byte_perm(w, 0x64u, 0x4240u)), __float2half2_rn(1024.f));
+  const __half2 h = __hfma2(hs, __float2half2_rn(256.f), ls);
+  const __half2 t = __hfma2(hs, __float2half2_rn(256.f), __hneg2(h));
+  hi = h2_bits(h);
+  lo = h2_bits(__hadd2(t, ls));
+}
 // two bf16 values -> f16x2, round to nearest: exact for values in the f16 normal range
 // (bf16 keeps 8 significant bits, f16 11); beyond +-65504 a value becomes +-inf
 __device__ __forceinline__ uint32_t cvt_bf16x2(uint32_t w) {
@@ -257,9 +272,12 @@ __device__ __forceinline__ void load_group(const uint8_t* rawslot, int lane, int
   }
 }
 
-template <int BITS>
+// SCALED: each row's f16 values are multiplied by that row's group scale sc[k] (both halves),
+// rounded once -- the dequantised value code * s of a group-scaled cache.
+template <int BITS, bool SCALED>
 __device__ __forceinline__ void store_group(const uint32_t (&w)[4][kPackedWords<BITS>],
-                                            uint8_t* pair, int lane, int fb) {
+                                            uint8_t* pair, int lane, int fb,
+                                            const __half2 (&sc)[4]) {
   const int g = (fb >> 3) + (lane & 1);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -286,6 +304,12 @@ __device__ __forceinline__ void store_group(const uint32_t (&w)[4][kPackedWords<
       o.y = cvt_small(u0, 0x4342u, bias);
       o.z = cvt_small(u1, 0x4140u, bias);
       o.w = cvt_small(u1, 0x4342u, bias);
+    }
+    if constexpr (SCALED) {
+      o.x = h2_bits(__hmul2(bits_h2(o.x), sc[k]));
+      o.y = h2_bits(__hmul2(bits_h2(o.y), sc[k]));
+      o.z = h2_bits(__hmul2(bits_h2(o.z), sc[k]));
+      o.w = h2_bits(__hmul2(bits_h2(o.w), sc[k]));
     }
     *reinterpret_cast<uint4*>(pair + (g >> 3) * kAtom + r * 128 + (((g & 7) ^ (r & 7)) << 4)) = o;
   }
@@ -318,13 +342,16 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   uint8_t* p_s = smem + P.off_p;
   uint8_t* pairs = smem + P.off_pairs;
   uint8_t* raw = smem + P.off_raw;
+  uint8_t* scw = smem + P.off_sc;         // [kScSlots] scale windows
+  uint8_t* los = smem + P.off_lo;         // [LR] low parts of 16-bit codes (f16, as pairs)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.off_bar);
   uint64_t* b_pfull = bars;               // [PR] group converted, visible to the tensor core
   uint64_t* b_pempty = b_pfull + P.PR;    // [PR] group released by the MMAs
   uint64_t* b_tfull = b_pempty + P.PR;    // [PR] 16-bit: TMA landed in the group slot
   uint64_t* b_rfull = b_tfull + P.PR;     // [RR] packed group landed
   uint64_t* b_rempty = b_rfull + P.RR;    // [RR] packed group consumed
-  uint64_t* b_sfull = b_rempty + P.RR;    // scores ready in TMEM
+  uint64_t* b_loempty = b_rempty + P.RR;  // [LR] 16-bit: low-part slot released by the MMAs
+  uint64_t* b_sfull = b_loempty + P.LR;   // scores ready in TMEM
   uint64_t* b_sempty = b_sfull + 1;       // scores read
   uint64_t* b_Pfull = b_sempty + 1;       // [2] P written
   uint64_t* b_Pempty = b_Pfull + 2;       // [2] output MMA of that P done
@@ -356,6 +383,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       mbar_init(&b_rfull[i], 1);
       mbar_init(&b_rempty[i], kConvWarps);
     }
+    for (int i = 0; i < P.LR; ++i) mbar_init(&b_loempty[i], 1);
     mbar_init(b_sfull, 1);
     mbar_init(b_sempty, 4);
     for (int i = 0; i < 2; ++i) {
@@ -373,7 +401,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     mbar_init(b_app, 1);
     for (int i = 0; i < kScSlots; ++i) {
       mbar_init(&b_scfull[i], 1);
-      mbar_init(&b_scempty[i], 4);
+      // released by the softmax warps (token scales) or the convert warps (group scales)
+      mbar_init(&b_scempty[i], P.grouped ? kConvWarps : 4);
     }
     m->abort = 0;
     fence_mbar_init();
@@ -429,11 +458,12 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           const int row0 = c.seq * a.max_tokens + c.pos;
           bool ok = true;
           if constexpr (BITS != 0) {   // this tile's scale window (the arena has tail slack)
-            const uintptr_t sp = reinterpret_cast<uintptr_t>(a.scales + row0);
+            const uintptr_t sp = reinterpret_cast<uintptr_t>(a.scales + (int64_t)row0 * a.sg);
             if (!(ok = mbar_wait(&b_scempty[sr.slot], sr.phase ^ 1u, abort, a.limit_ns))) break;
-            mbar_arrive_expect_tx(&b_scfull[sr.slot], kScBytes);
-            bulk_load_hint(m->sc[sr.slot], reinterpret_cast<const void*>(sp & ~uintptr_t(15)),
-                           kScBytes, &b_scfull[sr.slot], pol);
+            mbar_arrive_expect_tx(&b_scfull[sr.slot], P.sc_bytes);
+            bulk_load_hint(scw + sr.slot * P.sc_bytes,
+                           reinterpret_cast<const void*>(sp & ~uintptr_t(15)), P.sc_bytes,
+                           &b_scfull[sr.slot], pol);
             sr.next(kScSlots);
             ++nsc;
           }
@@ -479,7 +509,9 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       // (bits 0-13, address >> 4), so each operand adds its byte offset >> 4
       const uint64_t a0 = sdesc(smem_u32(pairs), 16u, 1024u, kLayoutSw128);
       const uint64_t b0 = sdesc(smem_u32(q_s), 16u, 1024u, kLayoutSw128);
+      const uint64_t l0 = sdesc(smem_u32(los), 16u, 1024u, kLayoutSw128);
       const uint32_t q_atom = (uint32_t)P.N1 * 128u;
+      Ring lr;   // low-part slots (16-bit codes)
       bool ok = true;
       while (g.valid && ok) {
         ok = mbar_wait(b_sempty, ((uint32_t)g.tile & 1u) ^ 1u, abort, a.limit_ns);
@@ -502,9 +534,23 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
               for (int ks = 0; k0 + ks < P.NK16; ++ks)
                 mma1_elect(tmem + kSCol, ad + 2u * ks, bd + 2u * ks, P.idesc1, (k0 + ks) > 0);
             }
+            if constexpr (BITS == 16) {
+              // the low parts of the same codes: S += (code - f16(code)) . Q, exact in f16
+              const uint64_t ld = l0 + ((lr.slot * kPair + t * kAtom) >> 4);
+              if (k0 + 4 <= P.NK16) {
+                mma4_elect(tmem + kSCol, ld, 2u, bd, 2u, P.idesc1, 1u);
+              } else {
+                for (int ks = 0; k0 + ks < P.NK16; ++ks)
+                  mma1_elect(tmem + kSCol, ld + 2u * ks, bd + 2u * ks, P.idesc1, 1u);
+              }
+            }
           }
           commit_elect(&b_pempty[s]);   // this group's share of the slot release
           rg.next(P.PR);
+          if constexpr (BITS == 16) {
+            commit_elect(&b_loempty[lr.slot]);
+            lr.next(P.LR);
+          }
         }
         if (!ok) break;
         commit_elect(b_sfull);
@@ -562,13 +608,15 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
             ok = write_token_two_pass<__nv_bfloat16>(
                      static_cast<const __nv_bfloat16*>(a.app_c) + (int64_t)i * a.app_c_ss,
                      static_cast<const __nv_bfloat16*>(a.app_kr) + (int64_t)i * a.app_kr_ss,
-                     a.d, a.d_rope, a.b, codes_w + r * a.row_bytes, a.row_bytes, scales_w + r) &&
+                     a.d, a.d_rope, a.b, a.group, codes_w + r * a.row_bytes, a.row_bytes,
+                     scales_w + r * a.sg) &&
                  ok;
           else
             ok = write_token_two_pass<float>(
                      static_cast<const float*>(a.app_c) + (int64_t)i * a.app_c_ss,
                      static_cast<const float*>(a.app_kr) + (int64_t)i * a.app_kr_ss, a.d,
-                     a.d_rope, a.b, codes_w + r * a.row_bytes, a.row_bytes, scales_w + r) &&
+                     a.d_rope, a.b, a.group, codes_w + r * a.row_bytes, a.row_bytes,
+                     scales_w + r * a.sg) &&
                  ok;
         }
         if (!ok && lane == 0) atomicOr(a.flags, KVK_FLAG_NONFINITE);
@@ -607,6 +655,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     const int cw = warp - kConvWarp0;
     const int cq = cw & 3, ch = cw >> 2, fb = 32 * cq + 16 * ch;
     Ring pr, rr;   // f16 group ring, packed group ring
+    Ring sr;       // scale windows (group-scaled cache only)
     int last_piece = -1;
     bool fail = false;
     const int cpr = P.NQA * 8;   // 16-byte chunks per staged query row
@@ -622,6 +671,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
                               ((cc ^ r8) << 4));
     }
     const uint32_t pairs_u = smem_u32(pairs);
+    const uint32_t los_u = smem_u32(los);
+    Ring lr;   // low-part slots of 16-bit codes
     // does this warp own features of group p (the last group may hold only one atom)?
     auto owns_group = [&](int p) { return (cq >> 1) < (((2 * p + 1) * 64 < a.n) ? 2 : 1); };
     Cursor c;
@@ -727,9 +778,25 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         auto step16 = [&](int p, uint32_t (&x)[16], uint32_t (&y)[16]) {
           const uint32_t s = pr.slot;
           const bool go = !fail && owns_group(p);
+          uint32_t xl[16];   // 16-bit codes: the low parts, for the score MMAs only
           if (go) {
+            if constexpr (BITS == 16) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = (BITS == 0) ? cvt_bf16x2(x[i]) : cvt_code16(x[i]);
+              for (int i = 0; i < 16; ++i) cvt_code16_split(x[i], x[i], xl[i]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) x[i] = cvt_bf16x2(x[i]);
+            }
+            if (BITS == 0 && c.cnt < kTile) {
+              // rows past the piece's end hold whatever the cache or scratch holds there (as
+              // bf16 possibly a NaN, and P = 0 times NaN is NaN): zero them.  Register 4tg + i
+              // holds tokens 16tg + 8(i%2) + 2(lane%4) + {0, 1}.
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int t0 = 16 * (i >> 2) + 8 * (i & 1) + 2 * (lane & 3);
+                x[i] &= (t0 < c.cnt ? 0x0000FFFFu : 0u) | (t0 + 1 < c.cnt ? 0xFFFF0000u : 0u);
+              }
+            }
           }
           if (p + 1 < P.NP) {
             Ring nx = pr;
@@ -737,12 +804,23 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
             fail = fail || !wait_warp(&b_tfull[nx.slot], nx.phase, abort, a.limit_ns);
             if (!fail && owns_group(p + 1)) load16(nx.slot, y);
           }
-          if (go) {
+          if constexpr (BITS == 16) {   // the low-part slot is free once its MMAs are done
+            fail = fail || !wait_warp(&b_loempty[lr.slot], lr.phase ^ 1u, abort, a.limit_ns);
+          }
+          if (go && !fail) {
             const uint32_t base = pairs_u + s * (uint32_t)kPair;
 #pragma unroll
             for (int tg = 0; tg < 4; ++tg) {
               const uint32_t d4[4] = {x[4 * tg], x[4 * tg + 1], x[4 * tg + 2], x[4 * tg + 3]};
               stsm_x4_trans(base + aoff[tg], d4);
+            }
+            if constexpr (BITS == 16) {
+              const uint32_t lbase = los_u + lr.slot * (uint32_t)kPair;
+#pragma unroll
+              for (int tg = 0; tg < 4; ++tg) {
+                const uint32_t d4[4] = {xl[4 * tg], xl[4 * tg + 1], xl[4 * tg + 2], xl[4 * tg + 3]};
+                stsm_x4_trans(lbase + aoff[tg], d4);
+              }
             }
           }
           fence_proxy_async_smem();
@@ -757,6 +835,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
             if (go && !fail) tmem_st16x256b_x4(ct_addr + 32u * p, x);
           }
           pr.next(P.PR);
+          if constexpr (BITS == 16) lr.next(P.LR);
         };
         fail = fail || !wait_warp(&b_tfull[pr.slot], pr.phase, abort, a.limit_ns);
         if (!fail && owns_group(0)) load16(pr.slot, xa);
@@ -770,6 +849,14 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         // this warp's 16 features are read back transposed into C^T.
         constexpr int NW = kPackedWords<BITS>;
         uint32_t wa[4][NW], wb[4][NW];
+        // group-scaled cache: this tile's scale window (rows past the piece's end get scale 0)
+        const __half* wsc = nullptr;
+        if (P.grouped) {
+          fail = fail || !wait_warp(&b_scfull[sr.slot], sr.phase, abort, a.limit_ns);
+          wsc = reinterpret_cast<const __half*>(scw + sr.slot * P.sc_bytes) +
+                ((reinterpret_cast<uintptr_t>(a.scales + ((int64_t)c.seq * a.max_tokens + c.pos) *
+                                                             a.sg) & 15u) >> 1);
+        }
         auto loadw = [&](uint32_t (&w)[4][NW]) {
           const uint32_t rs = rr.slot;
           fail = fail || !wait_warp(&b_rfull[rs], rr.phase, abort, a.limit_ns);
@@ -783,7 +870,23 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           uint8_t* pair = pairs + s * kPair;
           if (p + 1 < P.NP) loadw(wn);
           fail = fail || !wait_warp(&b_pempty[s], ph ^ 1u, abort, a.limit_ns);
-          if (!fail) store_group<BITS>(w, pair, lane, fb);
+          if (!fail) {
+            if (P.grouped) {
+              // scale index of this lane's eight features: (128 p + fb + 8 (lane % 2)) / G
+              const int j = (128 * p + fb + 8 * (lane & 1)) / a.group;
+              __half2 sc[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int r = conv_row(lane, k);
+                const __half sv = (r < c.cnt) ? wsc[r * a.sg + j] : __float2half(0.f);
+                sc[k] = __halves2half2(sv, sv);
+              }
+              store_group<BITS, true>(w, pair, lane, fb, sc);
+            } else {
+              const __half2 one[4] = {};
+              store_group<BITS, false>(w, pair, lane, fb, one);
+            }
+          }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && !fail) mbar_arrive(&b_pfull[s]);
@@ -816,6 +919,11 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         for (int p = 0; p < P.NP; p += 2) {
           stepw(p, wa, wb);
           if (p + 1 < P.NP) stepw(p + 1, wb, wa);
+        }
+        if (P.grouped) {   // the tile's scale window is no longer read by this warp
+          __syncwarp();
+          if (lane == 0 && !fail) mbar_arrive(&b_scempty[sr.slot]);
+          sr.next(kScSlots);
         }
       }
       tmem_wait_st();
@@ -861,12 +969,13 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     while (c.valid) {
       const int t = c.tile, sb = t & 1;
       float s_a = 0.f, s_b = 0.f;
-      if constexpr (BITS == 0) {   // uncompressed rows: every token's scale is 1
+      if (BITS == 0 || (!kInPlace<BITS> && P.grouped)) {
+        // uncompressed rows, or scales applied per group by the convert warps: unit token scale
         s_a = (ra < c.cnt) ? 1.f : 0.f;
         s_b = (rb < c.cnt) ? 1.f : 0.f;
       } else {
         fail = fail || !mbar_wait(&b_scfull[sr.slot], sr.phase, abort, a.limit_ns);
-        const __half* w = reinterpret_cast<const __half*>(m->sc[sr.slot]) +
+        const __half* w = reinterpret_cast<const __half*>(scw + sr.slot * P.sc_bytes) +
                           ((reinterpret_cast<uintptr_t>(a.scales + (int64_t)c.seq * a.max_tokens +
                                                         c.pos) & 15u) >> 1);
         if (ra < c.cnt) s_a = __half2float(w[ra]);
@@ -1112,7 +1221,8 @@ struct Plan {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-Plan make_plan(int d, int d_rope, int b, int H, int batch) {
+// sg: fp16 scales per token (group > 0: a group-scaled cache, scales applied in conversion)
+Plan make_plan(int d, int d_rope, int b, int H, int batch, int group, int sg) {
   Plan pl;
   memset(&pl, 0, sizeof(pl));
   TcParams& P = pl.p;
@@ -1132,15 +1242,25 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
   const size_t p_bytes = 2 * (size_t)P.p_bytes;
   const size_t misc_bytes = sizeof(Misc) + sizeof(int32_t) * (size_t)(batch + 1);
   const bool in_place = (b == 16 || b == KVK_BITS_BF16);
+  // group scales are applied while the packed codes are unpacked (b < 16): 16-bit codes
+  // converted in place, and uncompressed rows, take the CUDA-core kernel in such a layout
+  if (group && in_place) return pl;
   const int raw_slot = in_place ? 0 : 64 * 16 * b;
   P.raw_slot = raw_slot;
+  P.grouped = group ? 1 : 0;
+  // a tile's scale window: 64 tokens x sg scales from a 16-byte boundary, rounded up to 16
+  P.sc_bytes = (b == KVK_BITS_BF16) ? 0u : (uint32_t)align_up((size_t)64 * sg * 2 + 16, 16);
+  const size_t sc_ring = align_up((size_t)kScSlots * P.sc_bytes, 1024);
   // try the largest rings that fit
-  const size_t fixed = align_up(q_bytes, 1024) + align_up(p_bytes, 1024);
+  const size_t fixed = align_up(q_bytes, 1024) + align_up(p_bytes, 1024) + sc_ring;
+  // 16-bit codes: the low parts of two groups in flight
+  const int LR = (b == 16) ? 2 : 0;
+  P.LR = LR;
   auto total_for = [&](int PR, int RR) {
     size_t off = fixed;
-    off += (size_t)PR * kPair;
+    off += (size_t)(PR + LR) * kPair;
     off = align_up(off + (size_t)RR * raw_slot, 1024);
-    off = align_up(off + (size_t)(3 * PR + 2 * RR + kFixedBars) * 8, 16);
+    off = align_up(off + (size_t)(3 * PR + 2 * RR + LR + kFixedBars) * 8, 16);
     off += misc_bytes;
     return off + 1024;   // runtime alignment slack of the dynamic shared memory base
   };
@@ -1161,12 +1281,15 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
   P.RR = RR;
   size_t off = fixed;
   P.off_p = (uint32_t)align_up(q_bytes, 1024);
+  P.off_sc = P.off_p + (uint32_t)align_up(p_bytes, 1024);
   P.off_pairs = (uint32_t)fixed;
   off += (size_t)PR * kPair;
+  P.off_lo = (uint32_t)off;
+  off += (size_t)LR * kPair;
   P.off_raw = (uint32_t)off;
   off = align_up(off + (size_t)RR * raw_slot, 1024);
   P.off_bar = (uint32_t)off;
-  off = align_up(off + (size_t)(3 * PR + 2 * RR + kFixedBars) * 8, 16);
+  off = align_up(off + (size_t)(3 * PR + 2 * RR + LR + kFixedBars) * 8, 16);
   P.off_misc = (uint32_t)off;
   pl.smem = off + misc_bytes + 1024;
   P.idesc1 = sm100::idesc_f16(64, P.N1, false, false);
@@ -1237,13 +1360,13 @@ cudaError_t launch_bits(const TcParams& P, const CUtensorMap& tmap, size_t smem,
 bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H) {
   if (dtype != KVK_BF16 && dtype != KVK_F16) return false;
   if (!A.tmap_ok) return false;
-  const Plan pl = make_plan(A.d, L->d_rope, A.b, H, L->max_batch);
+  const Plan pl = make_plan(A.d, L->d_rope, A.b, H, L->max_batch, anchor_group(L, A), A.sg);
   return pl.ok && launch_regs_ok(A.b, pl.p.N2);
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tmap, int dtype,
                              cudaStream_t st) {
-  Plan pl = make_plan(a.d, a.d_rope, a.b, a.H, a.batch);
+  Plan pl = make_plan(a.d, a.d_rope, a.b, a.H, a.batch, a.group, a.sg);
   if (!pl.ok) return cudaErrorInvalidValue;
   pl.p.a = a;
   pl.p.qdtype = dtype;

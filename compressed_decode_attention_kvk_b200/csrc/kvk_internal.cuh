@@ -28,6 +28,7 @@ struct AnchorDesc {
   int b = 0;
   int n = 0;             // d + d_rope
   int row_bytes = 0;
+  int sg = 1;            // fp16 scales per token: n / G in a group-scaled layout, else 1
   int64_t codes_off = 0;
   int64_t scales_off = 0;
   bool tmap_ok = false;
@@ -42,6 +43,7 @@ struct kvk_layout {
   int d_rope = 0;
   int max_batch = 0;
   int max_tokens = 0;
+  int group = 0;                          // elements per scale (0: one scale per token)
   std::vector<int> anchor, d, b;
   std::vector<int> slot;                  // layer -> index into anchors (its anchor's)
   std::vector<kvk::AnchorDesc> anchors;
@@ -84,6 +86,8 @@ struct DecodeArgs {
   int split_x;               // cost of a piece in tokens (split_cost / split_token)
   uint32_t* flags;
   uint64_t limit_ns;         // time limit of one wait in the tensor-core kernel
+  int group, sg;             // group-scaled cache: elements per scale and scales per token
+                             // (group = 0, sg = 1: one scale per token)
   // fused append (kvk_mla_decode_append): before the decode reads it, the new token of
   // sequence i -- app_c[i * app_c_ss + k] (k < d) and app_kr[i * app_kr_ss + k] (k < d_rope),
   // dtype app_dtype -- is written at position seq_len_i - 1 of the cache.  app_c == nullptr:
@@ -101,6 +105,11 @@ size_t decode_workspace(int batch, int H, int d, int G, void* base, DecodeArgs* 
 int decode_ctas(const kvk_layout* L, int batch, int path);
 
 // launchers (return cudaGetLastError())
+// The scale group of an anchor's writes (0 = one scale per token): the layout's, except that
+// an uncompressed anchor always keeps one (unit) scale per token.
+inline int anchor_group(const kvk_layout* L, const AnchorDesc& A) {
+  return (A.b == KVK_BITS_BF16) ? 0 : L->group;
+}
 cudaError_t launch_quant_write(const kvk_layout* L, const AnchorDesc& A, const void* c_kv,
                                int dtype, int64_t c_ss, int64_t c_st, const void* k_rope,
                                int64_t kr_ss, int64_t kr_st, int batch, const int32_t* start_pos,
@@ -110,6 +119,7 @@ struct QuantLayer {
   uint8_t* codes;
   __half* scales;
   int row_bytes, d, b;
+  int group;   // elements per scale (0: one per token)
   const void* c_kv;
   int64_t c_ss, c_st;
   const void* k_rope;
@@ -146,13 +156,14 @@ struct CompactArgs {
   const int32_t* keep_idx;   // [batch][keep_stride]
   const int32_t* keep_len;
   int keep_stride;
+  int sg;                    // fp16 scales per token
   int32_t* cnt;              // [batch] valid kept entries per sequence (written)
   uint8_t* dst_codes;        // [batch * keep_stride][row_bytes]
   __half* dst_scales;        // [batch * keep_stride] (+ slack for the decode's scale windows)
   uint32_t* flags;
 };
-size_t compact_workspace_bytes(int batch, int keep_stride, int row_bytes);
-void compact_carve(void* base, int batch, int keep_stride, int row_bytes, CompactArgs* c);
+size_t compact_workspace_bytes(int batch, int keep_stride, int row_bytes, int sg);
+void compact_carve(void* base, int batch, int keep_stride, int row_bytes, int sg, CompactArgs* c);
 cudaError_t launch_compact(const CompactArgs& c, int batch, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
 

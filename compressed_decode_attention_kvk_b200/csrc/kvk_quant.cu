@@ -25,7 +25,8 @@ constexpr int kMaxRounds = kMaxRowElems / (8 * 32);  // groups of 8 per lane
 template <typename T>
 __device__ __forceinline__ void quant_token(
     int64_t tok, uint8_t* __restrict__ codes, __half* __restrict__ scales, int row_bytes, int d,
-    int d_rope, int b, int max_tokens, const T* __restrict__ c_kv, int64_t c_ss, int64_t c_st,
+    int d_rope, int b, int group, int max_tokens, const T* __restrict__ c_kv, int64_t c_ss,
+    int64_t c_st,
     const T* __restrict__ k_rope, int64_t kr_ss, int64_t kr_st, int batch,
     const int32_t* __restrict__ start_pos, int n_new, uint32_t* __restrict__ flags) {
   const int lane = threadIdx.x & 31;
@@ -65,6 +66,37 @@ __device__ __forceinline__ void quant_token(
   }
 
   uint8_t* row = codes + ((int64_t)seq * max_tokens + pos) * row_bytes;
+  if (group) {
+    // one scale per `group` elements: each group of G elements is quantised like a token
+    const int sg = n / group, lpg = group >> 3;   // scales per token, lanes per group
+    __half* srow = scales + ((int64_t)seq * max_tokens + pos) * sg;
+    bool bad = !finite;
+#pragma unroll
+    for (int r = 0; r < kMaxRounds; ++r) {
+      const int g = r * 32 + lane;
+      if (r * 32 >= groups) break;                        // warp-uniform
+      float ga = 0.0f;
+      if (g < groups) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ga = fmaxf(ga, fabsf(v[r][k]));
+      }
+      for (int o = 1; o < lpg; o <<= 1) ga = fmaxf(ga, __shfl_xor_sync(0xffffffffu, ga, o));
+      if (g >= groups) continue;
+      const __half s16 = quant_scale(ga, b);
+      const float s = __half2float(s16);
+      bad = bad || isinf(s);
+      if ((lane & (lpg - 1)) == 0) srow[(8 * g) / group] = s16;
+      uint32_t u[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) u[k] = quant_field(v[r][k], s, b);
+      store_fields8(row + (int64_t)g * b, u, b);
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    if (bad && lane == 0) atomicOr(flags, KVK_FLAG_NONFINITE);
+    const int used = groups * b;
+    if (lane < row_bytes - used) row[used + lane] = 0;
+    return;
+  }
   // uncompressed anchor: the bf16 of every element (round to nearest even) and scale 1
   const __half s16 = (b == KVK_BITS_BF16) ? __float2half(1.0f) : quant_scale(amax, b);
   const float s = __half2float(s16);
@@ -95,13 +127,13 @@ __device__ __forceinline__ void quant_token(
 template <typename T>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 quant_write_kernel(uint8_t* __restrict__ codes, __half* __restrict__ scales, int row_bytes,
-                   int d, int d_rope, int b, int max_tokens, const T* __restrict__ c_kv,
+                   int d, int d_rope, int b, int group, int max_tokens, const T* __restrict__ c_kv,
                    int64_t c_ss, int64_t c_st, const T* __restrict__ k_rope, int64_t kr_ss,
                    int64_t kr_st, int batch, const int32_t* __restrict__ start_pos, int n_new,
                    uint32_t* __restrict__ flags) {
   quant_token<T>((int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5), codes, scales,
-                 row_bytes, d, d_rope, b, max_tokens, c_kv, c_ss, c_st, k_rope, kr_ss, kr_st,
-                 batch, start_pos, n_new, flags);
+                 row_bytes, d, d_rope, b, group, max_tokens, c_kv, c_ss, c_st, k_rope, kr_ss,
+                 kr_st, batch, start_pos, n_new, flags);
 }
 
 // Several anchor layers in one launch: blockIdx.y picks the layer.
@@ -112,7 +144,7 @@ quant_write_layers_kernel(const __grid_constant__ QuantLayers Q, int d_rope, int
                           uint32_t* __restrict__ flags) {
   const QuantLayer& l = Q.l[blockIdx.y];
   quant_token<T>((int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5), l.codes, l.scales,
-                 l.row_bytes, l.d, d_rope, l.b, max_tokens, static_cast<const T*>(l.c_kv),
+                 l.row_bytes, l.d, d_rope, l.b, l.group, max_tokens, static_cast<const T*>(l.c_kv),
                  l.c_ss, l.c_st, static_cast<const T*>(l.k_rope), l.kr_ss, l.kr_st, batch,
                  start_pos, n_new, flags);
 }
@@ -121,7 +153,7 @@ quant_write_layers_kernel(const __grid_constant__ QuantLayers Q, int d_rope, int
 template <typename T>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 quant_append_kernel(uint8_t* __restrict__ codes, __half* __restrict__ scales, int row_bytes,
-                    int d, int d_rope, int b, int max_tokens, const T* __restrict__ c_new,
+                    int d, int d_rope, int b, int group, int max_tokens, const T* __restrict__ c_new,
                     int64_t c_ss, const T* __restrict__ kr_new, int64_t kr_ss, int batch,
                     const int32_t* __restrict__ seq_lens, uint32_t* __restrict__ flags) {
   const int i = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
@@ -129,8 +161,10 @@ quant_append_kernel(uint8_t* __restrict__ codes, __half* __restrict__ scales, in
   const int len = min(max(__ldg(seq_lens + i), 0), max_tokens);
   if (len == 0) return;
   const int64_t r = (int64_t)i * max_tokens + (len - 1);
+  const int sg = group ? (d + d_rope) / group : 1;
   if (!write_token_two_pass<T>(c_new + (int64_t)i * c_ss, kr_new + (int64_t)i * kr_ss, d,
-                               d_rope, b, codes + r * row_bytes, row_bytes, scales + r) &&
+                               d_rope, b, group, codes + r * row_bytes, row_bytes,
+                               scales + r * sg) &&
       (threadIdx.x & 31) == 0)
     atomicOr(flags, KVK_FLAG_NONFINITE);
 }
@@ -146,12 +180,12 @@ cudaError_t launch_quant_append(const kvk_layout* L, const AnchorDesc& A, const 
   dim3 grid((unsigned)((batch + kWarpsPerBlock - 1) / kWarpsPerBlock)), block(kWarpsPerBlock * 32);
   if (dtype == KVK_BF16)
     quant_append_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
-        codes, scales, A.row_bytes, A.d, L->d_rope, A.b, L->max_tokens,
+        codes, scales, A.row_bytes, A.d, L->d_rope, A.b, anchor_group(L, A), L->max_tokens,
         static_cast<const __nv_bfloat16*>(c_new), c_ss, static_cast<const __nv_bfloat16*>(kr_new),
         kr_ss, batch, seq_lens, flags);
   else
     quant_append_kernel<float><<<grid, block, 0, stream>>>(
-        codes, scales, A.row_bytes, A.d, L->d_rope, A.b, L->max_tokens,
+        codes, scales, A.row_bytes, A.d, L->d_rope, A.b, anchor_group(L, A), L->max_tokens,
         static_cast<const float*>(c_new), c_ss, static_cast<const float*>(kr_new), kr_ss, batch,
         seq_lens, flags);
   return cudaGetLastError();
@@ -170,12 +204,12 @@ cudaError_t launch_quant_write(const kvk_layout* L, const AnchorDesc& A, const v
   dim3 grid((unsigned)blocks), block(kWarpsPerBlock * 32);
   if (dtype == KVK_BF16) {
     quant_write_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
-        codes, scales, A.row_bytes, A.d, L->d_rope, A.b, L->max_tokens,
+        codes, scales, A.row_bytes, A.d, L->d_rope, A.b, anchor_group(L, A), L->max_tokens,
         static_cast<const __nv_bfloat16*>(c_kv), c_ss, c_st,
         static_cast<const __nv_bfloat16*>(k_rope), kr_ss, kr_st, batch, start_pos, n_new, flags);
   } else {
     quant_write_kernel<float><<<grid, block, 0, stream>>>(
-        codes, scales, A.row_bytes, A.d, L->d_rope, A.b, L->max_tokens,
+        codes, scales, A.row_bytes, A.d, L->d_rope, A.b, anchor_group(L, A), L->max_tokens,
         static_cast<const float*>(c_kv), c_ss, c_st, static_cast<const float*>(k_rope), kr_ss,
         kr_st, batch, start_pos, n_new, flags);
   }

@@ -90,52 +90,83 @@ __device__ __forceinline__ void store_bf16x8(uint8_t* dst, const float (&v)[8]) 
 __device__ __forceinline__ int group_bytes(int b) { return b == KVK_BITS_BF16 ? 16 : b; }
 
 // One warp writes one token: v = [c[0..d) || k^R[0..d_rope)] read from crow / krow, stored in
-// `row` (row_bytes, padding zeroed) with its scale in *scale.  Two passes over the inputs
-// (the max, then the fields), so a lane holds only eight values at a time; the arithmetic is
-// that of the single-pass write kernel.  Returns false (in every lane) if an input is not
-// finite or the scale overflows fp16 (the stored token is then unspecified).
+// `row` (row_bytes, padding zeroed) with its scale(s) at `scale` (one per token, or one per
+// `group` elements when group > 0).  Two passes over the inputs (the max, then the fields), so
+// a lane holds only eight values at a time; the arithmetic is that of the single-pass write
+// kernel.  Returns false (in every lane) if an input is not finite or a scale overflows fp16
+// (the stored token is then unspecified).
 template <typename T>
 __device__ __forceinline__ bool write_token_two_pass(const T* crow, const T* krow, int d,
-                                                     int d_rope, int b, uint8_t* row,
+                                                     int d_rope, int b, int group, uint8_t* row,
                                                      int row_bytes, __half* scale) {
   const int lane = threadIdx.x & 31;
   const int groups = (d + d_rope) >> 3, d_groups = d >> 3;
-  float amax = 0.0f;
-  bool finite = true;
-  for (int g = lane; g < groups; g += 32) {
-    float v[8];
-    if (g < d_groups) load8<T>(crow + 8 * g, v);
-    else load8<T>(krow + 8 * (g - d_groups), v);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      finite = finite && isfinite(v[k]);
-      amax = fmaxf(amax, fabsf(v[k]));
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  finite = __all_sync(0xffffffffu, finite);
-  __half s16 = __float2half(1.0f);
-  if (b != KVK_BITS_BF16) s16 = quant_scale(amax, b);
-  const float s = __half2float(s16);
-  if (lane == 0) *scale = s16;
   const int gb = group_bytes(b);
-  for (int g = lane; g < groups; g += 32) {
-    float v[8];
+  auto load = [&](int g, float (&v)[8]) {
     if (g < d_groups) load8<T>(crow + 8 * g, v);
     else load8<T>(krow + 8 * (g - d_groups), v);
-    if (b == KVK_BITS_BF16) {
-      store_bf16x8(row + (int64_t)g * gb, v);
-    } else {
-      uint32_t u[8];
+  };
+  bool ok = true;
+  if (group) {   // one scale per `group` elements: one pass, a round of 32 lanes at a time
+    const int lpg = group >> 3;
+    for (int g0 = 0; g0 < groups; g0 += 32) {
+      const int g = g0 + lane;
+      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float ga = 0.0f;
+      if (g < groups) {
+        load(g, v);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) u[k] = quant_field(v[k], s, b);
-      store_fields8(row + (int64_t)g * gb, u, b);
+        for (int k = 0; k < 8; ++k) {
+          ok = ok && isfinite(v[k]);
+          ga = fmaxf(ga, fabsf(v[k]));
+        }
+      }
+      for (int o = 1; o < lpg; o <<= 1) ga = fmaxf(ga, __shfl_xor_sync(0xffffffffu, ga, o));
+      if (g < groups) {
+        const __half s16 = quant_scale(ga, b);
+        const float s = __half2float(s16);
+        ok = ok && !isinf(s);
+        if ((lane & (lpg - 1)) == 0) scale[(8 * g) / group] = s16;
+        uint32_t u[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) u[k] = quant_field(v[k], s, b);
+        store_fields8(row + (int64_t)g * gb, u, b);
+      }
+    }
+  } else {
+    float amax = 0.0f;
+    for (int g = lane; g < groups; g += 32) {
+      float v[8];
+      load(g, v);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        ok = ok && isfinite(v[k]);
+        amax = fmaxf(amax, fabsf(v[k]));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    __half s16 = __float2half(1.0f);
+    if (b != KVK_BITS_BF16) s16 = quant_scale(amax, b);
+    const float s = __half2float(s16);
+    ok = ok && (b == KVK_BITS_BF16 || !isinf(s));
+    if (lane == 0) *scale = s16;
+    for (int g = lane; g < groups; g += 32) {
+      float v[8];
+      load(g, v);
+      if (b == KVK_BITS_BF16) {
+        store_bf16x8(row + (int64_t)g * gb, v);
+      } else {
+        uint32_t u[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) u[k] = quant_field(v[k], s, b);
+        store_fields8(row + (int64_t)g * gb, u, b);
+      }
     }
   }
   const int used = groups * gb;
   if (lane < row_bytes - used) row[used + lane] = 0;
-  return finite && (b == KVK_BITS_BF16 || !isinf(s));
+  return __all_sync(0xffffffffu, ok);
 }
 
 }  // namespace kvk

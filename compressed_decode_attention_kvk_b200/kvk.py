@@ -33,7 +33,8 @@ EXPORTED = ("kvk_create_layout", "kvk_destroy", "kvk_get_layer_info", "kvk_quant
             "kvk_decode_workspace_bytes", "kvk_mla_decode", "kvk_read_status",
             "kvk_set_decode_path", "kvk_set_decode_ctas", "kvk_decode_path_for",
             "kvk_status_string", "kvk_mla_decode_noalloc", "kvk_quant_write_layers",
-            "kvk_decode_workspace_bytes_keep", "kvk_set_wait_limit", "kvk_mla_decode_append")
+            "kvk_decode_workspace_bytes_keep", "kvk_set_wait_limit", "kvk_mla_decode_append",
+            "kvk_create_layout_grouped")
 
 # size of the library's built-in scratch array used by kvk_mla_decode_noalloc
 KVK_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -51,7 +52,8 @@ class LayerInfo(ctypes.Structure):
                 ("row_bytes", ctypes.c_int32), ("codes", ctypes.c_void_p),
                 ("scales", ctypes.c_void_p), ("codes_offset", ctypes.c_int64),
                 ("scales_offset", ctypes.c_int64), ("max_batch", ctypes.c_int32),
-                ("max_tokens", ctypes.c_int32), ("r", ctypes.c_int32), ("d_rope", ctypes.c_int32)]
+                ("max_tokens", ctypes.c_int32), ("r", ctypes.c_int32), ("d_rope", ctypes.c_int32),
+                ("scales_per_token", ctypes.c_int32), ("scale_group", ctypes.c_int32)]
 
 
 _LIB = None
@@ -66,6 +68,8 @@ def _lib_handle():
         L = ctypes.CDLL(LIB_PATH)
         P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
         L.kvk_create_layout.argtypes = [i32, P, P, P, i32, i32, i32, i32, i64, P, sz, P, P, P]
+        L.kvk_create_layout_grouped.argtypes = [i32, P, P, P, i32, i32, i32, i32, i32, i64, P,
+                                                sz, P, P, P]
         L.kvk_destroy.argtypes = [P]
         L.kvk_destroy.restype = None
         L.kvk_get_layer_info.argtypes = [P, i32, P]
@@ -126,8 +130,9 @@ def _need_cuda(t, name, dtypes=None):
 # ---------------------------------------------------------------------------
 
 def kvk_create_layout(anchor, d, b, r, d_rope, max_batch, max_tokens, budget_bits_per_token=0,
-                      arena=None, query_only=False):
-    """Returns (handle or None, arena_bytes_needed, bits_per_token)."""
+                      arena=None, query_only=False, scale_group=0):
+    """Returns (handle or None, arena_bytes_needed, bits_per_token).  scale_group > 0 calls
+    kvk_create_layout_grouped (one fp16 scale per scale_group elements)."""
     L = _lib_handle()
     n = len(anchor)
     need = ctypes.c_size_t(0)
@@ -135,12 +140,17 @@ def kvk_create_layout(anchor, d, b, r, d_rope, max_batch, max_tokens, budget_bit
     handle = ctypes.c_void_p()
     if arena is not None:
         _need_cuda(arena, "arena")
-    st = L.kvk_create_layout(n, _i32_array(anchor), _i32_array(d), _i32_array(b), r, d_rope,
-                             max_batch, max_tokens, int(budget_bits_per_token), _ptr(arena),
-                             0 if arena is None else arena.numel() * arena.element_size(),
-                             None if query_only else ctypes.byref(handle), ctypes.byref(need),
-                             ctypes.byref(bits))
-    _check("kvk_create_layout", st)
+    common = (_ptr(arena), 0 if arena is None else arena.numel() * arena.element_size(),
+              None if query_only else ctypes.byref(handle), ctypes.byref(need), ctypes.byref(bits))
+    if scale_group:
+        st = L.kvk_create_layout_grouped(n, _i32_array(anchor), _i32_array(d), _i32_array(b), r,
+                                         d_rope, scale_group, max_batch, max_tokens,
+                                         int(budget_bits_per_token), *common)
+        _check("kvk_create_layout_grouped", st)
+    else:
+        st = L.kvk_create_layout(n, _i32_array(anchor), _i32_array(d), _i32_array(b), r, d_rope,
+                                 max_batch, max_tokens, int(budget_bits_per_token), *common)
+        _check("kvk_create_layout", st)
     return (None if query_only else handle), need.value, bits.value
 
 
@@ -336,23 +346,28 @@ class Layout:
     one is passed in)."""
 
     def __init__(self, anchor, d, b, r, d_rope, max_batch, max_tokens, budget_bits_per_token=0,
-                 arena=None, device="cuda"):
+                 arena=None, device="cuda", scale_group=0):
         self.anchor, self.d, self.b = list(anchor), list(d), list(b)
         self.r, self.d_rope = r, d_rope
         self.max_batch, self.max_tokens = max_batch, max_tokens
+        self.scale_group = scale_group
         _, need, bits = kvk_create_layout(anchor, d, b, r, d_rope, max_batch, max_tokens,
-                                          budget_bits_per_token, query_only=True)
+                                          budget_bits_per_token, query_only=True,
+                                          scale_group=scale_group)
         self.arena_bytes, self.bits_per_token = need, bits
         if arena is None:
             arena = torch.empty(need, dtype=torch.uint8, device=device)
         self.arena = arena
         self.handle, _, _ = kvk_create_layout(anchor, d, b, r, d_rope, max_batch, max_tokens,
-                                              budget_bits_per_token, arena=arena)
+                                              budget_bits_per_token, arena=arena,
+                                              scale_group=scale_group)
 
     @staticmethod
-    def query(anchor, d, b, r, d_rope, max_batch, max_tokens, budget_bits_per_token=0):
+    def query(anchor, d, b, r, d_rope, max_batch, max_tokens, budget_bits_per_token=0,
+              scale_group=0):
         _, need, bits = kvk_create_layout(anchor, d, b, r, d_rope, max_batch, max_tokens,
-                                          budget_bits_per_token, query_only=True)
+                                          budget_bits_per_token, query_only=True,
+                                          scale_group=scale_group)
         return need, bits
 
     @property
@@ -363,15 +378,19 @@ class Layout:
         return kvk_get_layer_info(self.handle, layer)
 
     def cache_views(self, layer):
-        """(codes uint8 [max_batch, max_tokens, row_bytes], scales fp16 [max_batch, max_tokens])
-        views of the arena for the layer's anchor."""
+        """(codes uint8 [max_batch, max_tokens, row_bytes], scales fp16 [max_batch, max_tokens]
+        -- [max_batch, max_tokens, scales_per_token] for a group-scaled anchor) views of the
+        arena for the layer's anchor."""
         info = self.layer_info(layer)
         T = self.max_batch * self.max_tokens
-        co, so = info["codes_offset"], info["scales_offset"]
+        co, so, sg = info["codes_offset"], info["scales_offset"], info["scales_per_token"]
         codes = self.arena[co:co + T * info["row_bytes"]].view(self.max_batch, self.max_tokens,
                                                                info["row_bytes"])
-        scales = self.arena[so:so + 2 * T].view(torch.float16).view(self.max_batch,
-                                                                    self.max_tokens)
+        scales = self.arena[so:so + 2 * T * sg].view(torch.float16)
+        if sg == 1:
+            scales = scales.view(self.max_batch, self.max_tokens)
+        else:
+            scales = scales.view(self.max_batch, self.max_tokens, sg)
         return codes, scales
 
     def quant_write(self, layer, c_kv, k_rope, start_pos, stream=None):

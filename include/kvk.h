@@ -119,6 +119,31 @@ kvk_status kvk_create_layout(int n_layers, const int32_t* anchor, const int32_t*
                              kvk_layout** out, size_t* arena_bytes_needed,
                              int64_t* bits_per_token);
 
+/*
+ * kvk_create_layout_grouped -- kvk_create_layout with one fp16 scale per group of
+ * `scale_group` consecutive elements of each quantised anchor's row instead of one per token:
+ * the group-scale comparison point of the precision axis (a 4-bit cache with a scale per 32
+ * elements costs 4.5 bits per element, the figure behind the 152x composition of "Hardware
+ * Benchmarking (Apple M3 Ultra)"; KIVI-style grouping in "Main Results / Table 2").
+ *
+ *   scale_group  G in {16, 32, 64}; every quantised anchor needs (d + d_rope) % G == 0
+ *                (else KVK_ERR_BAD_TABLE); uncompressed anchors keep one unit scale per token
+ *   other arguments as kvk_create_layout, and
+ *     bits_per_token = sum over quantised anchors of ((d + d_rope) * b + 16 * (d + d_rope) / G)
+ *                      (+ (d + d_rope) * 16 for uncompressed anchors).
+ * Scale plane of such an anchor: [max_batch][max_tokens][(d + d_rope) / G] fp16, scale j of a
+ * token covering elements [j G, (j + 1) G).  Each group is quantised as kvk_quant_write
+ * quantises a token (its own absmax, scale rounded up, round-half-even codes), and decode
+ * dequantises each element with its group's scale.  Every other entry point takes such a
+ * layout unchanged.
+ */
+kvk_status kvk_create_layout_grouped(int n_layers, const int32_t* anchor, const int32_t* d,
+                                     const int32_t* b, int r, int d_rope, int scale_group,
+                                     int max_batch, int max_tokens,
+                                     int64_t budget_bits_per_token, void* dev_arena,
+                                     size_t arena_bytes, kvk_layout** out,
+                                     size_t* arena_bytes_needed, int64_t* bits_per_token);
+
 /* Frees the host-side handle only (never the arena).  NULL is ignored. */
 void kvk_destroy(kvk_layout* layout);
 
@@ -138,6 +163,8 @@ typedef struct {
     int32_t max_tokens;
     int32_t r;
     int32_t d_rope;
+    int32_t scales_per_token; /* fp16 scales per token in the scale plane (1, or (d+d_rope)/G) */
+    int32_t scale_group;      /* elements per scale G of a group-scaled anchor, 0: per token    */
 } kvk_layer_info;
 
 kvk_status kvk_get_layer_info(const kvk_layout* layout, int layer, kvk_layer_info* info);

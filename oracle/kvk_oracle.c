@@ -326,6 +326,26 @@ int64_t kvko_bits_per_token(int n_layers, const int32_t* anchor, const int32_t* 
     return s;
 }
 
+/* Bits per token of a plan whose anchors carry one fp16 scale per group of G
+ * consecutive elements of [c[:d] || k^R] instead of one per token (the group-scale
+ * comparison point: a b-bit cache with a scale per G elements costs b + 16/G bits
+ * per element, e.g. 4.5 at b = 4, G = 32): anchors pay (d+d_R)*b + 16*(d+d_R)/G;
+ * an uncompressed (b = 0) anchor pays (d+d_R)*16. */
+int64_t kvko_bits_per_token_grouped(int n_layers, const int32_t* anchor, const int32_t* d,
+                                    const int32_t* b, int d_R, int G)
+{
+    int64_t s = 0;
+    for (int l = 0; l < n_layers; ++l) {
+        if (anchor[l] != l) continue;
+        const int n = d[l] + d_R;
+        if (b[l] == 0)
+            s += (int64_t)n * 16;
+        else
+            s += (int64_t)n * b[l] + (int64_t)16 * (n / G);
+    }
+    return s;
+}
+
 /* Uncompressed bf16 non-MLA cost: C_0 = L * 2 * n_kv * d_h * 16. */
 int64_t kvko_c0_bits(int n_layers, int n_kv, int d_h)
 {

@@ -67,6 +67,8 @@ def lib():
         L.kvko_f32_to_bf16_rne.argtypes = [ctypes.c_float]
         L.kvko_f32_to_bf16_rne.restype = ctypes.c_uint16
         L.kvko_bf16_round.argtypes = [P, i64, P]
+        L.kvko_bits_per_token_grouped.argtypes = [i32, P, P, P, i32, i32]
+        L.kvko_bits_per_token_grouped.restype = i64
         _lib = L
     return _lib
 
@@ -174,6 +176,14 @@ def bits_per_token(anchor, d, b, d_R: int, with_scale: bool = True) -> int:
     return int(lib().kvko_bits_per_token(len(a), _p(a), _p(dd), _p(bb), d_R, 1 if with_scale else 0))
 
 
+def bits_per_token_grouped(anchor, d, b, d_R: int, G: int) -> int:
+    """Bits per token with one fp16 scale per G elements of each anchor's row."""
+    a = np.ascontiguousarray(np.asarray(anchor, dtype=np.int32))
+    dd = np.ascontiguousarray(np.asarray(d, dtype=np.int32))
+    bb = np.ascontiguousarray(np.asarray(b, dtype=np.int32))
+    return int(lib().kvko_bits_per_token_grouped(len(a), _p(a), _p(dd), _p(bb), d_R, G))
+
+
 def c0_bits(n_layers: int, n_kv: int, d_h: int) -> int:
     return int(lib().kvko_c0_bits(n_layers, n_kv, d_h))
 
@@ -226,6 +236,36 @@ def decode_sequence_bf16(q_lat, q_rope, values, d: int, sigma: float, tok=None):
     if tok is None:
         tok = np.arange(T, dtype=np.int32)
     return attend(np.asarray(q_lat, dtype=np.float64)[:, :d], q_rope, values, tok, sigma)
+
+
+def quantize_rows_grouped(c_kv: np.ndarray, k_rope: np.ndarray, d: int, b: int, G: int):
+    """Quantise one sequence's tokens with one scale per group of G consecutive elements of
+    [c[:d] || k^R]: the per-token quantiser applied to every group as if it were a token.
+
+    Returns (packed rows uint8 [T, row_bytes], scales uint16 [T, n / G], codes int32 [T, n]).
+    """
+    v = token_vectors(c_kv, k_rope, d)
+    T, n = v.shape
+    assert n % G == 0
+    scales, codes = quantize(v.reshape(T * (n // G), G), b)
+    codes = codes.reshape(T, n)
+    return pack(codes, b), scales.reshape(T, n // G), codes
+
+
+def dequant_grouped(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """c_hat = code * s of its group, exact in binary64; scales [T, n / G]."""
+    T, n = codes.shape
+    ng = scales.shape[1]
+    return dequant(codes.reshape(T * ng, n // ng), scales.reshape(T * ng)).reshape(T, n)
+
+
+def decode_sequence_grouped(q_lat, q_rope, codes, scales, d: int, sigma: float, tok=None):
+    """Attention of one sequence over a group-scaled cache (codes [T, n], scales [T, n/G])."""
+    rows_hat = dequant_grouped(codes, scales)
+    T = rows_hat.shape[0]
+    if tok is None:
+        tok = np.arange(T, dtype=np.int32)
+    return attend(np.asarray(q_lat, dtype=np.float64)[:, :d], q_rope, rows_hat, tok, sigma)
 
 
 def decode_sequence(q_lat, q_rope, codes, scales, d: int, sigma: float, tok=None):

@@ -442,3 +442,71 @@ def test_bf16_cache_attention_equals_attention_on_the_rounded_rows(oracle_mod):
     ref, ref_lse = _sdpa(ql, qr, exact, r, 0.125)
     np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# group scales: one fp16 scale per G consecutive elements instead of per token
+# --------------------------------------------------------------------------
+
+def test_grouped_cost_reproduces_the_m3_ultra_ratio(oracle_mod):
+    """"Hardware Benchmarking (M3 Ultra)": a 4-bit cache, MLA rank 128 and 12 groups of 4
+    layers compose to 152x.  With one fp16 scale per 32 elements the 4-bit cache costs 4.5
+    bits per element, and the grouped cost function gives C_0 / bits = 151.7 -> 152."""
+    g = _read_kv(os.path.join(GOLDEN, "cost_model_closed_forms.txt"))
+    anchor = [4 * (l // 4) for l in range(48)]
+    d = [128 if l % 4 == 0 else 0 for l in range(48)]
+    b = [4 if l % 4 == 0 else 0 for l in range(48)]
+    bits = oracle_mod.bits_per_token_grouped(anchor, d, b, 64, 32)
+    assert bits == 12 * (128 + 64) * 4 + 12 * 16 * (128 + 64) // 32
+    c0 = oracle_mod.c0_bits(48, 8, 128)
+    assert round(c0 / bits) == g["m3_ultra_ratio_rounded"]
+    # one group per row is the per-token cost
+    assert oracle_mod.bits_per_token_grouped([0], [128], [4], 64, 192) == \
+        oracle_mod.bits_per_token([0], [128], [4], 64)
+
+
+def test_grouped_quantiser_with_one_group_is_the_per_token_quantiser(oracle_mod):
+    rng = np.random.default_rng(31)
+    c = rng.standard_normal((40, 64)).astype(np.float32)
+    kr = rng.standard_normal((40, 16)).astype(np.float32)
+    for b in (2, 4, 8, 16):
+        rows, s, k = oracle_mod.quantize_rows(c, kr, 64, b)
+        rows_g, s_g, k_g = oracle_mod.quantize_rows_grouped(c, kr, 64, b, 80)
+        assert np.array_equal(rows, rows_g) and np.array_equal(k, k_g)
+        assert np.array_equal(s, s_g[:, 0])
+
+
+@pytest.mark.parametrize("b", [2, 4, 8])
+@pytest.mark.parametrize("G", [16, 32])
+def test_grouped_quantiser_against_brute_force_and_bounds(oracle_mod, b, G):
+    """Each group's scale is the smallest binary16 value not below max|v_group| / q, its codes
+    the brute-force nearest (ties to even) under that scale, and the dequantised error at
+    most half the group's scale (up to the binary32 rounding of v / s)."""
+    rng = np.random.default_rng(40 + b + G)
+    q = 2 ** (b - 1) - 1
+    T, d, dR = 12, 64, 32
+    c = rng.standard_normal((T, d)).astype(np.float32)
+    kr = rng.standard_normal((T, dR)).astype(np.float32)
+    c[2, :G] *= 1e3                   # one loud group: the others keep their own scale
+    c[3, G:2 * G] = 0.0               # an all-zero group
+    _, scales, codes = oracle_mod.quantize_rows_grouped(c, kr, d, b, G)
+    v = np.concatenate([c, kr], axis=1)
+    for t in range(T):
+        for j in range(v.shape[1] // G):
+            vg = v[t, j * G:(j + 1) * G]
+            A = float(np.max(np.abs(vg)))
+            s = oracle_mod.f16_bits_to_f64(int(scales[t, j]))
+            cg = codes[t, j * G:(j + 1) * G]
+            if A == 0.0:
+                assert s == 0.0 and not cg.any()
+                continue
+            want_s, _ = _smallest_f16_at_least(float(np.float32(A) / np.float32(q)))
+            assert s == want_s, (t, j)
+            assert np.array_equal(cg, _brute_codes(vg, s, q)), (t, j)
+            err = np.abs(vg.astype(np.float64) - cg * s)
+            assert np.all(err <= s / 2 + np.abs(vg.astype(np.float64)) * 2.0 ** -23)
+    # the loud group does not coarsen its neighbours
+    assert scales[2, 1] < scales[2, 0]
+    rows_hat = oracle_mod.dequant_grouped(codes, scales)
+    assert np.array_equal(rows_hat[:, :G], codes[:, :G] * np.array(
+        [oracle_mod.f16_bits_to_f64(int(x)) for x in scales[:, 0]])[:, None])
