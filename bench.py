@@ -44,6 +44,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="kvk", choices=["kvk", "reference"])
     p.add_argument("--workload", default="14b_4x")
+    p.add_argument("--budget", type=int, default=None,
+                   help="compression target of a budget-sweep workload (1, 2, 4, 8 or 16)")
     p.add_argument("--graph", action="store_true", help="replay the step as a CUDA graph")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -199,21 +201,26 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 class DecodeWorkload:
-    def __init__(self, name, device, pkg):
+    def __init__(self, name, device, pkg, budget=None, time_prefill=False):
         self.w = w = workloads.WORKLOADS[name]
-        self.t = t = workloads.table(name)
+        self.t = t = workloads.table(name, budget)
+        self.budget = budget if budget is not None else (w.budgets[0] if w.budgets else None)
         self.device = device
         self.pkg = pkg
         self.B, self.T, self.H = w.batch, w.tokens, w.n_heads
         self.lay = pkg.Layout(t["anchor"], t["d"], t["b"], w.r, w.d_rope, self.B, self.T,
-                              device=device)
+                              device=device, scale_group=w.scale_group)
         self.anchors = [l for l in range(w.n_layers) if t["anchor"][l] == l]
         zero = torch.zeros(self.B, dtype=torch.int32, device=device)
-        for l in self.anchors:            # prefill (not timed)
-            c = workloads.latent(w, l, self.B, self.T, device=device)
-            kr = workloads.rope_key(w, l, self.B, self.T, device=device)
-            self.lay.quant_write(l, c, kr, zero)
-            del c, kr
+        self.prefill = None
+        if time_prefill:
+            self.prefill = self._timed_prefill(zero)
+        else:
+            for l in self.anchors:            # prefill (not timed)
+                c = workloads.latent(w, l, self.B, self.T, device=device)
+                kr = workloads.rope_key(w, l, self.B, self.T, device=device)
+                self.lay.quant_write(l, c, kr, zero)
+                del c, kr
         torch.cuda.synchronize(device)
         # per-step inputs: one new token per anchor (written at the last position), queries
         self.app_pos = torch.full((self.B,), self.T - 1, dtype=torch.int32, device=device)
@@ -240,12 +247,16 @@ class DecodeWorkload:
         self.bytes_per_layer = []
         for l in range(w.n_layers):
             info = self.lay.layer_info(l)
-            # rows read (the kept ones with a keep list) and their scales, plus 4 B per index
-            self.bytes_per_layer.append(self.B * self.n_read * (info["row_bytes"] + 2) +
+            # rows read (the kept ones with a keep list) and their scales (none for an
+            # uncompressed anchor, one per group in a group-scaled cache), plus 4 B per index
+            sb = 0 if info["b"] == 0 else 2 * info["scales_per_token"]
+            self.bytes_per_layer.append(self.B * self.n_read * (info["row_bytes"] + sb) +
                                         (4 * self.B * w.keep if w.keep else 0))
         self.decode_bytes = sum(self.bytes_per_layer)
         mx = max(self.bytes_per_layer)
-        self.l2_note = ("inputs larger than L2 (per-layer cache > 126 MB)" if not w.keep else
+        self.l2_note = ("inputs larger than L2 (per-layer cache > 126 MB)" if mx > 126e6 and not w.keep else
+                        f"per-layer cache {mx / 1e6:.1f} MB < 126 MB L2: layers that inherit "
+                        "the previous layer's anchor may find it in L2" if not w.keep else
                         f"kept rows {mx / 1e6:.1f} MB per layer (< 126 MB L2), gathered from a "
                         f"{self.B * self.T * max(self.lay.layer_info(l)['row_bytes'] + 2 for l in range(w.n_layers)) / 1e6:.0f} MB "
                         "cache: a layer that inherits the previous layer's anchor may find them in L2")
@@ -255,6 +266,43 @@ class DecodeWorkload:
         if w.keep and self.lay.decode_path_for(0, self.q[0][0].dtype, self.H, True) == 1:
             per_layer = 3
         self.launches_per_step = 1 + per_layer * w.n_layers
+
+    def _timed_prefill(self, zero):
+        """The quantise-on-write of the whole prompt (batch x tokens) for every anchor layer,
+        one kvk_quant_write_layers launch per chunk of at most 64 anchors, inputs resident in
+        HBM; timed with CUDA events (best of 3).  Algorithmic bytes: the bf16 inputs read plus
+        the rows and scales written."""
+        from compressed_decode_attention_kvk_b200 import kvk
+        w = self.w
+        ins = {l: (workloads.latent(w, l, self.B, self.T, device=self.device),
+                   workloads.rope_key(w, l, self.B, self.T, device=self.device))
+               for l in self.anchors}
+        torch.cuda.synchronize(self.device)
+        nbytes = 0
+        for l in self.anchors:
+            info = self.lay.layer_info(l)
+            sb = 0 if info["b"] == 0 else 2 * info["scales_per_token"]
+            nbytes += self.B * self.T * ((info["d"] + w.d_rope) * 2 + info["row_bytes"] + sb)
+        best = None
+        for _ in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for k in range(0, len(self.anchors), 64):
+                ls = self.anchors[k:k + 64]
+                kvk.kvk_quant_write_layers(self.lay.handle, ls, [ins[l][0] for l in ls],
+                                           [ins[l][1] for l in ls], zero)
+            b.record()
+            torch.cuda.synchronize(self.device)
+            ms = a.elapsed_time(b)
+            best = ms if best is None else min(best, ms)
+        del ins
+        torch.cuda.empty_cache()
+        peak, kind = measured_peaks()
+        gbs = nbytes / (best * 1e-3) / 1e9
+        return {"ms": round(best, 4), "bytes": nbytes, "GBps": round(gbs, 1),
+                "frac": round(gbs / peak, 4), "peak": peak, "peak_kind": kind,
+                "tokens": self.B * self.T, "anchors": len(self.anchors),
+                "kernel": "quant_write_layers_kernel (the prompt's quantise-on-write)"}
 
     def step(self, events=None):
         from compressed_decode_attention_kvk_b200 import kvk
@@ -280,7 +328,8 @@ def run_kvk(args, rank, world, local, pg):
     barrier(pg)
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    wl = DecodeWorkload(args.workload, device, pkg)
+    wl = DecodeWorkload(args.workload, device, pkg, budget=args.budget,
+                        time_prefill=workloads.WORKLOADS[args.workload].prefill)
     L = wl.w.n_layers
 
     # ---- device-timed steps (inputs resident in HBM) -----------------------------------
@@ -359,11 +408,15 @@ def run_kvk(args, rank, world, local, pg):
             "dtype": "bf16", "data": "synthetic (seeded, generated on device)",
             "config": {"workload": args.workload, "layers": L, "heads": wl.H, "r": wl.w.r,
                        "d_rope": wl.w.d_rope, "batch": wl.B, "tokens": wl.T,
+                       "budget": wl.budget, "scale_group": wl.w.scale_group,
                        "bits_per_token": wl.lay.bits_per_token,
+                       "compression_vs_bf16_c0": round(
+                           2 * wl.w.n_kv * wl.w.d_h * 16 * L / wl.lay.bits_per_token, 3)
+                       if wl.w.n_kv else None,
                        "decode_bytes_per_step": wl.decode_bytes,
                        "l2": wl.l2_note,
                        "graph": bool(graph), "parallelism": f"replicas x{world}"},
-            "roofline": roof, "e2e": e2e, "cpu_baseline": cpu,
+            "roofline": roof, "e2e": e2e, "cpu_baseline": cpu, "prefill": wl.prefill,
             "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

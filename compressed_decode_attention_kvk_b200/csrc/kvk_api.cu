@@ -626,6 +626,29 @@ kvk_status kvk_set_decode_ctas(kvk_layout* L, int ctas) {
   return KVK_OK;
 }
 
+kvk_status kvk_absorb(const void* x, int x_dtype, int64_t x_stride_seq, int64_t x_stride_head,
+                      const void* w, int64_t w_stride_row, int64_t w_stride_head, void* y,
+                      int y_dtype, int64_t y_stride_seq, int64_t y_stride_head, int batch,
+                      int n_heads, int K, int n, kvk_stream_t stream) {
+  if (!x || !w || !y) return KVK_ERR_INVALID_ARG;
+  if ((x_dtype != KVK_BF16 && x_dtype != KVK_F32) || (y_dtype != KVK_BF16 && y_dtype != KVK_F32))
+    return KVK_ERR_INVALID_ARG;
+  if (batch < 1 || n_heads < 1 || n_heads > 65535 || K < 64 || K > 512 || K % 64 != 0 ||
+      n < 16 || n % 16 != 0 || n > 65535 * 128)
+    return KVK_ERR_INVALID_ARG;
+  if (x_stride_seq < 0 || x_stride_head < 0 || y_stride_seq < 0 || y_stride_head < 0 ||
+      w_stride_row < n || w_stride_head < (int64_t)K * w_stride_row)
+    return KVK_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y) || x_stride_seq % 8 || x_stride_head % 8 ||
+      w_stride_row % 8 || w_stride_head % 8 || y_stride_seq % 8 || y_stride_head % 8)
+    return KVK_ERR_ALIGNMENT;
+  cudaError_t e = kvk::launch_absorb(x, x_dtype == KVK_F32, x_stride_seq, x_stride_head, w,
+                                     w_stride_row, w_stride_head, y, y_dtype == KVK_F32,
+                                     y_stride_seq, y_stride_head, batch, n_heads, K, n, nullptr,
+                                     reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVK_OK : KVK_ERR_CUDA;
+}
+
 kvk_status kvk_set_wait_limit(kvk_layout* L, uint64_t ns) {
   if (!L) return KVK_ERR_INVALID_ARG;
   L->wait_limit_ns = ns;

@@ -56,7 +56,7 @@ using namespace sm100;
 constexpr int kThreads = 512;   // 16 warps = 4 warpgroups (warp 15 has no role)
 constexpr int kConvWarp0 = 4;
 constexpr int kConvWarps = 8;
-constexpr int kConvThreads = 32 * kConvWarps;
+constexpr int kTeamWarps = kConvWarps / 2;   // two conversion teams take alternate groups
 constexpr int kTmaWarp = 12;
 constexpr int kMmaWarp = 13;   // score MMAs; owns TMEM
 constexpr int kMma2Warp = 14;  // output MMAs
@@ -272,11 +272,14 @@ __device__ __forceinline__ void load_group(const uint8_t* rawslot, int lane, int
   }
 }
 
-// SCALED: each row's f16 values are multiplied by that row's group scale sc[k] (both halves),
-// rounded once -- the dequantised value code * s of a group-scaled cache.
+// SCALED: each row's f16 values are multiplied by that row's group scale sc[k] (both halves):
+// the dequantised value code * s of a group-scaled cache, split exactly into hi = f16(code * s)
+// (stored in `pair`) and lo = code * s - hi (stored at the same place in `lo_pair`; the fused
+// multiply-add is exact, the product of a b <= 8 bit code and an 11-bit scale having at most
+// 18 significant bits).
 template <int BITS, bool SCALED>
 __device__ __forceinline__ void store_group(const uint32_t (&w)[4][kPackedWords<BITS>],
-                                            uint8_t* pair, int lane, int fb,
+                                            uint8_t* pair, uint8_t* lo_pair, int lane, int fb,
                                             const __half2 (&sc)[4]) {
   const int g = (fb >> 3) + (lane & 1);
 #pragma unroll
@@ -305,13 +308,22 @@ __device__ __forceinline__ void store_group(const uint32_t (&w)[4][kPackedWords<
       o.z = cvt_small(u1, 0x4140u, bias);
       o.w = cvt_small(u1, 0x4342u, bias);
     }
+    const int at = (g >> 3) * kAtom + r * 128 + (((g & 7) ^ (r & 7)) << 4);
     if constexpr (SCALED) {
-      o.x = h2_bits(__hmul2(bits_h2(o.x), sc[k]));
-      o.y = h2_bits(__hmul2(bits_h2(o.y), sc[k]));
-      o.z = h2_bits(__hmul2(bits_h2(o.z), sc[k]));
-      o.w = h2_bits(__hmul2(bits_h2(o.w), sc[k]));
+      uint4 h, l;
+      h.x = h2_bits(__hmul2(bits_h2(o.x), sc[k]));
+      h.y = h2_bits(__hmul2(bits_h2(o.y), sc[k]));
+      h.z = h2_bits(__hmul2(bits_h2(o.z), sc[k]));
+      h.w = h2_bits(__hmul2(bits_h2(o.w), sc[k]));
+      l.x = h2_bits(__hfma2(bits_h2(o.x), sc[k], __hneg2(bits_h2(h.x))));
+      l.y = h2_bits(__hfma2(bits_h2(o.y), sc[k], __hneg2(bits_h2(h.y))));
+      l.z = h2_bits(__hfma2(bits_h2(o.z), sc[k], __hneg2(bits_h2(h.z))));
+      l.w = h2_bits(__hfma2(bits_h2(o.w), sc[k], __hneg2(bits_h2(h.w))));
+      *reinterpret_cast<uint4*>(pair + at) = h;
+      *reinterpret_cast<uint4*>(lo_pair + at) = l;
+    } else {
+      *reinterpret_cast<uint4*>(pair + at) = o;
     }
-    *reinterpret_cast<uint4*>(pair + (g >> 3) * kAtom + r * 128 + (((g & 7) ^ (r & 7)) << 4)) = o;
   }
 }
 
@@ -374,14 +386,14 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
 
   if (tid == 0) {
     for (int i = 0; i < P.PR; ++i) {
-      mbar_init(&b_pfull[i], kConvWarps);
+      mbar_init(&b_pfull[i], kTeamWarps);   // the team converting the group
       // score MMAs (commit), plus the convert warps where they read the slot after q_full
-      mbar_init(&b_pempty[i], kInPlace<BITS> ? 1 : 1 + kConvWarps);
+      mbar_init(&b_pempty[i], kInPlace<BITS> ? 1 : 1 + kTeamWarps);
       mbar_init(&b_tfull[i], 1);
     }
     for (int i = 0; i < P.RR; ++i) {
       mbar_init(&b_rfull[i], 1);
-      mbar_init(&b_rempty[i], kConvWarps);
+      mbar_init(&b_rempty[i], kTeamWarps);
     }
     for (int i = 0; i < P.LR; ++i) mbar_init(&b_loempty[i], 1);
     mbar_init(b_sfull, 1);
@@ -534,8 +546,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
               for (int ks = 0; k0 + ks < P.NK16; ++ks)
                 mma1_elect(tmem + kSCol, ad + 2u * ks, bd + 2u * ks, P.idesc1, (k0 + ks) > 0);
             }
-            if constexpr (BITS == 16) {
-              // the low parts of the same codes: S += (code - f16(code)) . Q, exact in f16
+            if (BITS == 16 || P.grouped) {
+              // the low parts of the same rows: S += (c - f16(c)) . Q, exact in f16
               const uint64_t ld = l0 + ((lr.slot * kPair + t * kAtom) >> 4);
               if (k0 + 4 <= P.NK16) {
                 mma4_elect(tmem + kSCol, ld, 2u, bd, 2u, P.idesc1, 1u);
@@ -547,7 +559,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           }
           commit_elect(&b_pempty[s]);   // this group's share of the slot release
           rg.next(P.PR);
-          if constexpr (BITS == 16) {
+          if (BITS == 16 || P.grouped) {
             commit_elect(&b_loempty[lr.slot]);
             lr.next(P.LR);
           }
@@ -645,36 +657,67 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   } else if (has_work && warp >= kConvWarp0) {
     regs_set<kRegsConvert>();
     // ------------------------------------------------------------------ convert
-    // Warp cw sits in TMEM lane quarter cq = cw % 4 and owns features fb .. fb+15 of every
-    // group, fb = 32 cq + 16 ch (ch = cw / 4): TMEM lanes fb .. fb+15 of C^T.  The groups of a
-    // tile are software-pipelined: the codes of group p+1 are loaded while group p is
-    // converted and stored, so each warp keeps two groups in flight.  The warps share no
-    // barrier among themselves (every hand-off is an mbarrier), so a warp that stops on a
-    // failed wait leaves its loop alone; it then arrives on nothing more, and everything
-    // downstream of the group it stopped at waits until it sees the abort word.
+    // Two teams of four warps take alternate groups (team cw / 4 converts the groups p with
+    // p % 2 == team), so two groups are in flight; in its team's groups warp cw owns the 32
+    // features 32 cq .. 32 cq + 31 (cq = cw % 4), which are its own TMEM lane quarter of C^T.
+    // The warps share no barrier among themselves (every hand-off is an mbarrier), so a warp
+    // that stops on a failed wait leaves its loop alone; it then arrives on nothing more, and
+    // everything downstream of the group it stopped at waits until it sees the abort word.
     const int cw = warp - kConvWarp0;
-    const int cq = cw & 3, ch = cw >> 2, fb = 32 * cq + 16 * ch;
+    const int cq = cw & 3, team = cw >> 2;
     Ring pr, rr;   // f16 group ring, packed group ring
     Ring sr;       // scale windows (group-scaled cache only)
     int last_piece = -1;
     bool fail = false;
     const int cpr = P.NQA * 8;   // 16-byte chunks per staged query row
-    // this lane's ldmatrix row address inside a group slot, per 16-token block tg: atom cq/2,
-    // 16-byte chunk 4(cq%2) + 2ch + (lane/8)/2 of token 16tg + 8((lane/8)%2) + lane%8
-    uint32_t aoff[4];
+    // this lane's ldmatrix row address inside a group slot, per 16-feature half h and 16-token
+    // block tg: atom cq/2, 16-byte chunk 4(cq%2) + 2h + (lane/8)/2 of token
+    // 16tg + 8((lane/8)%2) + lane%8
+    uint32_t aoff[2][4];
     {
       const int mi = lane >> 3, r8 = lane & 7;
-      const int cc = 4 * (cq & 1) + 2 * ch + (mi >> 1);
 #pragma unroll
-      for (int tg = 0; tg < 4; ++tg)
-        aoff[tg] = (uint32_t)((cq >> 1) * kAtom + (16 * tg + 8 * (mi & 1) + r8) * 128 +
-                              ((cc ^ r8) << 4));
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int tg = 0; tg < 4; ++tg)
+          aoff[h][tg] = (uint32_t)((cq >> 1) * kAtom + (16 * tg + 8 * (mi & 1) + r8) * 128 +
+                                   (((4 * (cq & 1) + 2 * h + (mi >> 1)) ^ r8) << 4));
     }
     const uint32_t pairs_u = smem_u32(pairs);
     const uint32_t los_u = smem_u32(los);
-    Ring lr;   // low-part slots of 16-bit codes
+    Ring lr;   // low-part slots
     // does this warp own features of group p (the last group may hold only one atom)?
     auto owns_group = [&](int p) { return (cq >> 1) < (((2 * p + 1) * 64 < a.n) ? 2 : 1); };
+    // ldmatrix (transposed) of this warp's 32 features x 64 tokens of a group slot
+    auto ldsm32 = [&](uint32_t base, uint32_t (&x)[32]) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int tg = 0; tg < 4; ++tg) {
+          uint32_t d4[4];
+          ldsm_x4_trans(base + aoff[h][tg], d4);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) x[16 * h + 4 * tg + i] = d4[i];
+        }
+    };
+    auto stsm32 = [&](uint32_t base, const uint32_t (&x)[32]) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int tg = 0; tg < 4; ++tg) {
+          const uint32_t d4[4] = {x[16 * h + 4 * tg], x[16 * h + 4 * tg + 1],
+                                  x[16 * h + 4 * tg + 2], x[16 * h + 4 * tg + 3]};
+          stsm_x4_trans(base + aoff[h][tg], d4);
+        }
+    };
+    // this warp's C^T: TMEM lanes 32 cq .. 32 cq + 31, columns of latent group p
+    auto tmem_st32 = [&](uint32_t col, const uint32_t (&x)[32]) {
+      const uint32_t* x0 = x;
+      tmem_st16x256b_x4(tmem + ((uint32_t)(32 * cq) << 16) + col,
+                        *reinterpret_cast<const uint32_t(*)[16]>(x0));
+      tmem_st16x256b_x4(tmem + ((uint32_t)(32 * cq + 16) << 16) + col,
+                        *reinterpret_cast<const uint32_t(*)[16]>(x0 + 16));
+    };
     Cursor c;
     cursor_start(c, seq0, off, a.batch, lo, hi);
     while (c.valid) {
@@ -756,99 +799,70 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         last_piece = c.piece;
       }
       const int ctb = c.tile & 1;   // C^T buffer of this tile
-      const uint32_t ct_addr = tmem + ((uint32_t)fb << 16) + kCtCol0 + 128u * ctb;
+      const uint32_t ct_col = kCtCol0 + 128u * ctb;
+      // the output MMAs of tile - 2 have finished reading this C^T buffer (waited before the
+      // team's first store of the tile)
+      auto wait_ct = [&]() {
+        fail = fail || !wait_warp(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u, abort,
+                                  a.limit_ns);
+        tc_fence_after();
+      };
+      const bool low_parts = (BITS == 16) || P.grouped;   // score MMAs add exact low parts
       if constexpr (kInPlace<BITS>) {
-        // In place, 16-bit codes (or bf16 values) -> f16, in one pass through registers: each 8x8 block
-        // (8 tokens x 8 features) is loaded transposed, converted element by element, stored
-        // back transposed (row-major again, for the score MMAs) and the same registers, now
-        // feature-major, go to C^T in TMEM (lanes fb .. fb+15 of latent group p).  The slot
-        // is not read after q_full, so only the score MMAs release it.
-        uint32_t xa[16], xb[16];
-        auto load16 = [&](uint32_t slot, uint32_t (&x)[16]) {
-          const uint32_t base = pairs_u + slot * (uint32_t)kPair;
+        // In place, 16-bit codes (or bf16 values) -> f16, in one pass through registers: each
+        // 8x8 block (8 tokens x 8 features) is loaded transposed, converted element by
+        // element, stored back transposed (row-major again, for the score MMAs) and the same
+        // registers, now feature-major, go to C^T in TMEM.  The slot is not read after q_full,
+        // so only the score MMAs release it.
+        for (int p = 0; p < P.NP; ++p) {
+          if ((p & 1) == team) {
+            const uint32_t s = pr.slot;
+            fail = fail || !wait_warp(&b_tfull[s], pr.phase, abort, a.limit_ns);
+            const bool go = !fail && owns_group(p);
+            uint32_t x[32], xl[32];
+            if (go) {
+              ldsm32(pairs_u + s * (uint32_t)kPair, x);
+              if constexpr (BITS == 16) {
 #pragma unroll
-          for (int tg = 0; tg < 4; ++tg) {
-            uint32_t d4[4];
-            ldsm_x4_trans(base + aoff[tg], d4);
+                for (int i = 0; i < 32; ++i) cvt_code16_split(x[i], x[i], xl[i]);
+              } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) x[4 * tg + i] = d4[i];
-          }
-        };
-        // group p is in x (loaded); convert it, load group p+1 into y, store and hand off x
-        auto step16 = [&](int p, uint32_t (&x)[16], uint32_t (&y)[16]) {
-          const uint32_t s = pr.slot;
-          const bool go = !fail && owns_group(p);
-          uint32_t xl[16];   // 16-bit codes: the low parts, for the score MMAs only
-          if (go) {
-            if constexpr (BITS == 16) {
+                for (int i = 0; i < 32; ++i) x[i] = cvt_bf16x2(x[i]);
+                if (c.cnt < kTile) {
+                  // rows past the piece's end hold whatever the cache or scratch holds there
+                  // (as bf16 possibly a NaN, and P = 0 times NaN is NaN): zero them.  Register
+                  // 16h + 4tg + i holds tokens 16tg + 8(i%2) + 2(lane%4) + {0, 1}.
 #pragma unroll
-              for (int i = 0; i < 16; ++i) cvt_code16_split(x[i], x[i], xl[i]);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) x[i] = cvt_bf16x2(x[i]);
-            }
-            if (BITS == 0 && c.cnt < kTile) {
-              // rows past the piece's end hold whatever the cache or scratch holds there (as
-              // bf16 possibly a NaN, and P = 0 times NaN is NaN): zero them.  Register 4tg + i
-              // holds tokens 16tg + 8(i%2) + 2(lane%4) + {0, 1}.
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const int t0 = 16 * (i >> 2) + 8 * (i & 1) + 2 * (lane & 3);
-                x[i] &= (t0 < c.cnt ? 0x0000FFFFu : 0u) | (t0 + 1 < c.cnt ? 0xFFFF0000u : 0u);
+                  for (int i = 0; i < 32; ++i) {
+                    const int t0 = 16 * ((i >> 2) & 3) + 8 * (i & 1) + 2 * (lane & 3);
+                    x[i] &= (t0 < c.cnt ? 0x0000FFFFu : 0u) | (t0 + 1 < c.cnt ? 0xFFFF0000u : 0u);
+                  }
+                }
               }
             }
-          }
-          if (p + 1 < P.NP) {
-            Ring nx = pr;
-            nx.next(P.PR);
-            fail = fail || !wait_warp(&b_tfull[nx.slot], nx.phase, abort, a.limit_ns);
-            if (!fail && owns_group(p + 1)) load16(nx.slot, y);
-          }
-          if constexpr (BITS == 16) {   // the low-part slot is free once its MMAs are done
-            fail = fail || !wait_warp(&b_loempty[lr.slot], lr.phase ^ 1u, abort, a.limit_ns);
-          }
-          if (go && !fail) {
-            const uint32_t base = pairs_u + s * (uint32_t)kPair;
-#pragma unroll
-            for (int tg = 0; tg < 4; ++tg) {
-              const uint32_t d4[4] = {x[4 * tg], x[4 * tg + 1], x[4 * tg + 2], x[4 * tg + 3]};
-              stsm_x4_trans(base + aoff[tg], d4);
+            if constexpr (BITS == 16)   // the low-part slot is free once its MMAs are done
+              fail = fail || !wait_warp(&b_loempty[lr.slot], lr.phase ^ 1u, abort, a.limit_ns);
+            if (go && !fail) {
+              stsm32(pairs_u + s * (uint32_t)kPair, x);
+              if constexpr (BITS == 16) stsm32(los_u + lr.slot * (uint32_t)kPair, xl);
             }
-            if constexpr (BITS == 16) {
-              const uint32_t lbase = los_u + lr.slot * (uint32_t)kPair;
-#pragma unroll
-              for (int tg = 0; tg < 4; ++tg) {
-                const uint32_t d4[4] = {xl[4 * tg], xl[4 * tg + 1], xl[4 * tg + 2], xl[4 * tg + 3]};
-                stsm_x4_trans(lbase + aoff[tg], d4);
-              }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && !fail) mbar_arrive(&b_pfull[s]);
+            if (p < P.NPd) {
+              if (p == team) wait_ct();
+              if (go && !fail) tmem_st32(ct_col + 32u * p, x);
             }
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && !fail) mbar_arrive(&b_pfull[s]);
-          if (p < P.NPd) {
-            if (p == 0) {   // the output MMAs of tile - 2 have finished reading this buffer
-              fail = fail || !wait_warp(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u,
-                                        abort, a.limit_ns);
-              tc_fence_after();
-            }
-            if (go && !fail) tmem_st16x256b_x4(ct_addr + 32u * p, x);
           }
           pr.next(P.PR);
           if constexpr (BITS == 16) lr.next(P.LR);
-        };
-        fail = fail || !wait_warp(&b_tfull[pr.slot], pr.phase, abort, a.limit_ns);
-        if (!fail && owns_group(0)) load16(pr.slot, xa);
-        for (int p = 0; p < P.NP; p += 2) {
-          step16(p, xa, xb);
-          if (p + 1 < P.NP) step16(p + 1, xb, xa);
         }
       } else {
-        // Packed codes: group p's words are loaded into registers (and its raw slot released)
-        // before group p-1 is converted; then each group is unpacked into its f16 slot, and
-        // this warp's 16 features are read back transposed into C^T.
+        // Packed codes: the team's group is read from the raw ring into registers (and the raw
+        // slot released), unpacked into its f16 slot -- with a group-scaled cache multiplied by
+        // the group scales and split into exact high and low parts -- and this warp's 32
+        // features are read back transposed into C^T.
         constexpr int NW = kPackedWords<BITS>;
-        uint32_t wa[4][NW], wb[4][NW];
         // group-scaled cache: this tile's scale window (rows past the piece's end get scale 0)
         const __half* wsc = nullptr;
         if (P.grouped) {
@@ -857,68 +871,59 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
                 ((reinterpret_cast<uintptr_t>(a.scales + ((int64_t)c.seq * a.max_tokens + c.pos) *
                                                              a.sg) & 15u) >> 1);
         }
-        auto loadw = [&](uint32_t (&w)[4][NW]) {
-          const uint32_t rs = rr.slot;
-          fail = fail || !wait_warp(&b_rfull[rs], rr.phase, abort, a.limit_ns);
-          if (!fail) load_group<BITS>(raw + rs * P.raw_slot, lane, fb, w);
-          __syncwarp();
-          if (lane == 0 && !fail) mbar_arrive(&b_rempty[rs]);
-          rr.next(P.RR);
-        };
-        auto stepw = [&](int p, uint32_t (&w)[4][NW], uint32_t (&wn)[4][NW]) {
-          const uint32_t s = pr.slot, ph = pr.phase;
-          uint8_t* pair = pairs + s * kPair;
-          if (p + 1 < P.NP) loadw(wn);
-          fail = fail || !wait_warp(&b_pempty[s], ph ^ 1u, abort, a.limit_ns);
-          if (!fail) {
-            if (P.grouped) {
-              // scale index of this lane's eight features: (128 p + fb + 8 (lane % 2)) / G
-              const int j = (128 * p + fb + 8 * (lane & 1)) / a.group;
-              __half2 sc[4];
+        for (int p = 0; p < P.NP; ++p) {
+          if ((p & 1) == team) {
+            const uint32_t s = pr.slot, ph = pr.phase, rs = rr.slot;
+            uint8_t* pair = pairs + s * kPair;
+            uint32_t w[2][4][NW];
+            fail = fail || !wait_warp(&b_rfull[rs], rr.phase, abort, a.limit_ns);
+            if (!fail) {
+              load_group<BITS>(raw + rs * P.raw_slot, lane, 32 * cq, w[0]);
+              load_group<BITS>(raw + rs * P.raw_slot, lane, 32 * cq + 16, w[1]);
+            }
+            __syncwarp();
+            if (lane == 0 && !fail) mbar_arrive(&b_rempty[rs]);
+            fail = fail || !wait_warp(&b_pempty[s], ph ^ 1u, abort, a.limit_ns);
+            if (P.grouped)   // the low-part slot is free once its MMAs are done
+              fail = fail || !wait_warp(&b_loempty[lr.slot], lr.phase ^ 1u, abort, a.limit_ns);
+            if (!fail) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const int r = conv_row(lane, k);
-                const __half sv = (r < c.cnt) ? wsc[r * a.sg + j] : __float2half(0.f);
-                sc[k] = __halves2half2(sv, sv);
+              for (int h = 0; h < 2; ++h) {
+                const int fb = 32 * cq + 16 * h;
+                if (P.grouped) {
+                  // scale index of this lane's eight features: (128 p + fb + 8 (lane % 2)) / G
+                  const int j = (128 * p + fb + 8 * (lane & 1)) / a.group;
+                  __half2 sc[4];
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) {
+                    const int r = conv_row(lane, k);
+                    const __half sv = (r < c.cnt) ? wsc[r * a.sg + j] : __float2half(0.f);
+                    sc[k] = __halves2half2(sv, sv);
+                  }
+                  store_group<BITS, true>(w[h], pair, los + lr.slot * kPair, lane, fb, sc);
+                } else {
+                  const __half2 one[4] = {};
+                  store_group<BITS, false>(w[h], pair, nullptr, lane, fb, one);
+                }
               }
-              store_group<BITS, true>(w, pair, lane, fb, sc);
-            } else {
-              const __half2 one[4] = {};
-              store_group<BITS, false>(w, pair, lane, fb, one);
             }
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && !fail) mbar_arrive(&b_pfull[s]);
-          if (p < P.NPd) {
-            // transpose this warp's 16 features x 64 tokens into C^T (TMEM lanes fb .. fb+15
-            // of latent group p): four 16-token blocks
-            if (p == 0) {   // the output MMAs of tile - 2 have finished reading this buffer
-              fail = fail || !wait_warp(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u,
-                                        abort, a.limit_ns);
-              tc_fence_after();
-            }
-            if (!fail && owns_group(p)) {
-              const uint32_t base = smem_u32(pair);
-              uint32_t x[16];
-#pragma unroll
-              for (int tg = 0; tg < 4; ++tg) {
-                uint32_t d4[4];
-                ldsm_x4_trans(base + aoff[tg], d4);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) x[4 * tg + i] = d4[i];
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && !fail) mbar_arrive(&b_pfull[s]);
+            if (p < P.NPd) {
+              if (p == team) wait_ct();
+              if (!fail && owns_group(p)) {
+                uint32_t x[32];
+                ldsm32(smem_u32(pair), x);
+                tmem_st32(ct_col + 32u * p, x);
               }
-              tmem_st16x256b_x4(ct_addr + 32u * p, x);
             }
+            __syncwarp();
+            if (lane == 0 && !fail) mbar_arrive(&b_pempty[s]);   // this warp is done with the slot
           }
-          __syncwarp();
-          if (lane == 0 && !fail) mbar_arrive(&b_pempty[s]);   // this warp is done with the slot
           pr.next(P.PR);
-        };
-        loadw(wa);
-        for (int p = 0; p < P.NP; p += 2) {
-          stepw(p, wa, wb);
-          if (p + 1 < P.NP) stepw(p + 1, wb, wa);
+          rr.next(P.RR);
+          if (P.grouped) lr.next(P.LR);
         }
         if (P.grouped) {   // the tile's scale window is no longer read by this warp
           __syncwarp();
@@ -926,6 +931,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           sr.next(kScSlots);
         }
       }
+      (void)low_parts;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -1253,8 +1259,8 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch, int group, int sg) {
   const size_t sc_ring = align_up((size_t)kScSlots * P.sc_bytes, 1024);
   // try the largest rings that fit
   const size_t fixed = align_up(q_bytes, 1024) + align_up(p_bytes, 1024) + sc_ring;
-  // 16-bit codes: the low parts of two groups in flight
-  const int LR = (b == 16) ? 2 : 0;
+  // 16-bit codes and group-scaled rows: the low parts of two groups in flight
+  const int LR = (b == 16 || group) ? 2 : 0;
   P.LR = LR;
   auto total_for = [&](int PR, int RR) {
     size_t off = fixed;

@@ -167,6 +167,13 @@ void compact_carve(void* base, int batch, int keep_stride, int row_bytes, int sg
 cudaError_t launch_compact(const CompactArgs& c, int batch, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
 
+// Absorbed projections (kvk_absorb.cu): y[b, h, j] = sum_k x[b, h, k] w[h, k, j].
+size_t absorb_smem_bytes(int K, int x_f32);
+cudaError_t launch_absorb(const void* x, int x_f32, int64_t x_ss, int64_t x_sh, const void* w,
+                          int64_t w_sk, int64_t w_sh, void* y, int y_f32, int64_t y_ss,
+                          int64_t y_sh, int batch, int heads, int K, int n, uint32_t* flags,
+                          cudaStream_t st);
+
 // Work split of the flattened tokens over G CTAs.  Sequence i occupies the cost range
 // [off[i] + X i, off[i+1] + X (i+1)): X units standing for the fixed cost of a piece (query
 // staging, partial write-back), then one unit per token; C = N + X batch in all.  CTA c owns

@@ -125,6 +125,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, 
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
+// 3D tile load global -> shared (coordinates innermost first), completion on an mbarrier
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, int y, int z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
 // Bulk copy (no tensor map) of `bytes` (multiple of 16) from global to shared memory; both
 // addresses 16-byte aligned; completion counted on an mbarrier (this CTA only).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,

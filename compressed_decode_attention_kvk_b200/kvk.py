@@ -34,7 +34,7 @@ EXPORTED = ("kvk_create_layout", "kvk_destroy", "kvk_get_layer_info", "kvk_quant
             "kvk_set_decode_path", "kvk_set_decode_ctas", "kvk_decode_path_for",
             "kvk_status_string", "kvk_mla_decode_noalloc", "kvk_quant_write_layers",
             "kvk_decode_workspace_bytes_keep", "kvk_set_wait_limit", "kvk_mla_decode_append",
-            "kvk_create_layout_grouped")
+            "kvk_create_layout_grouped", "kvk_absorb")
 
 # size of the library's built-in scratch array used by kvk_mla_decode_noalloc
 KVK_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -70,6 +70,8 @@ def _lib_handle():
         L.kvk_create_layout.argtypes = [i32, P, P, P, i32, i32, i32, i32, i64, P, sz, P, P, P]
         L.kvk_create_layout_grouped.argtypes = [i32, P, P, P, i32, i32, i32, i32, i32, i64, P,
                                                 sz, P, P, P]
+        L.kvk_absorb.argtypes = [P, i32, i64, i64, P, i64, i64, P, i32, i64, i64, i32, i32, i32,
+                                 i32, P]
         L.kvk_destroy.argtypes = [P]
         L.kvk_destroy.restype = None
         L.kvk_get_layer_info.argtypes = [P, i32, P]
@@ -305,6 +307,26 @@ def kvk_mla_decode_noalloc(handle, layer, q_lat, q_rope, seq_lens, softmax_scale
         _ptr(keep_idx), _ptr(keep_len), 0 if keep_idx is None else keep_idx.stride(0),
         float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream))
     _check("kvk_mla_decode_noalloc", st)
+
+
+def kvk_absorb(x, w, y, stream=None):
+    """y[b, h, j] = sum_k x[b, h, k] * w[h, k, j] on the tensor cores.  x [B, H, K] (bf16 or
+    fp32, last dim contiguous), w [H, K, >= n] bf16 (rows contiguous), y [B, H, n] (bf16 or
+    fp32, last dim contiguous); n = y.shape[2]."""
+    _need_cuda(x, "x", (torch.bfloat16, torch.float32))
+    _need_cuda(w, "w", (torch.bfloat16,))
+    _need_cuda(y, "y", (torch.bfloat16, torch.float32))
+    if x.stride(2) != 1 or w.stride(2) != 1 or y.stride(2) != 1:
+        raise ValueError("x, w and y need a contiguous last dim")
+    B, H, K = x.shape
+    n = y.shape[2]
+    if tuple(y.shape[:2]) != (B, H) or w.shape[0] != H or w.shape[1] < K or w.shape[2] < n:
+        raise ValueError("shapes of x [B, H, K], w [H, >=K, >=n] and y [B, H, n] do not match")
+    st = _lib_handle().kvk_absorb(_ptr(x), _DTYPE[x.dtype], x.stride(0), x.stride(1), _ptr(w),
+                                  w.stride(1), w.stride(0), _ptr(y), _DTYPE[y.dtype], y.stride(0),
+                                  y.stride(1), B, H, K, n, _stream(stream))
+    _check("kvk_absorb", st)
+    return y
 
 
 def kvk_read_status(handle, clear=False, stream=None) -> int:

@@ -338,6 +338,32 @@ kvk_status kvk_mla_decode_noalloc(kvk_layout* layout, int layer, const void* q_l
                                   float softmax_scale, float* out, float* lse,
                                   kvk_stream_t stream);
 
+/*
+ * kvk_absorb -- the absorbed MLA projections on either side of the decode, on the tensor
+ * cores ("Three Non-Eviction Compression Axes", item 2: only the first d latent coordinates
+ * a layer keeps are produced or consumed):
+ *     y[b][h][j] = sum_{k < K} x[b][h][k] * w[h][k][j]      for b < batch, h < n_heads, j < n
+ * Query side: x = q_nope (bf16, K = the head dim), w = W_UK restricted to its first d columns,
+ * y = q_lat (bf16, n = d) for kvk_mla_decode.  Output side: x = the decode output (fp32, K = d),
+ * w = W_UV restricted to its first d rows, y = the heads' values (fp32, n = the value dim).
+ *
+ *   x       device, x_dtype KVK_BF16 or KVK_F32, element (b, h, k) at
+ *           x[b * x_stride_seq + h * x_stride_head + k]; an fp32 x enters the tensor cores
+ *           as two bf16 parts (hi = bf16(x), lo = bf16(x - hi)), about 16 significant bits
+ *   w       device bf16, element (h, k, j) at w[h * w_stride_head + k * w_stride_row + j]
+ *           (w_stride_row >= n, w_stride_head >= K * w_stride_row)
+ *   y       device, y_dtype KVK_BF16 (rounded to nearest even) or KVK_F32, element (b, h, j) at
+ *           y[b * y_stride_seq + h * y_stride_head + j]; written completely
+ *   K       64 <= K <= 512, K % 64 == 0;  n >= 16, n % 16 == 0;  1 <= n_heads <= 65535
+ *   All strides are in elements and multiples of 8; pointers 16-byte aligned
+ *   (KVK_ERR_ALIGNMENT otherwise).  Accumulation is fp32.  No layout is involved; a wait that
+ *   runs out (2 s) leaves y unspecified.
+ */
+kvk_status kvk_absorb(const void* x, int x_dtype, int64_t x_stride_seq, int64_t x_stride_head,
+                      const void* w, int64_t w_stride_row, int64_t w_stride_head, void* y,
+                      int y_dtype, int64_t y_stride_seq, int64_t y_stride_head, int batch,
+                      int n_heads, int K, int n, kvk_stream_t stream);
+
 /* Copy the sticky device flags to *flags (synchronises the stream); clear != 0 resets them
  * to zero afterwards. */
 kvk_status kvk_read_status(kvk_layout* layout, uint32_t* flags, int clear, kvk_stream_t stream);

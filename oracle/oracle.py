@@ -268,6 +268,15 @@ def decode_sequence_grouped(q_lat, q_rope, codes, scales, d: int, sigma: float, 
     return attend(np.asarray(q_lat, dtype=np.float64)[:, :d], q_rope, rows_hat, tok, sigma)
 
 
+def absorb(x: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """The absorbed MLA projection (the query into the latent space with W_UK, the output out
+    of it with W_UV; "Three Non-Eviction Compression Axes", item 2): y[b, h, j] =
+    sum_k x[b, h, k] w[h, k, j], in binary64 (a matrix product per head)."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    return np.einsum("bhk,hkj->bhj", x, w)
+
+
 def decode_sequence(q_lat, q_rope, codes, scales, d: int, sigma: float, tok=None):
     """Attention of one sequence over its anchor's quantised cache.
 

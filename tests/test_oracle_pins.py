@@ -365,7 +365,7 @@ def test_workload_tables_meet_their_budgets(oracle_mod):
         for l in range(len(a)):
             if a[l] == l:
                 last = l
-                assert t["d"][l] > 0 and t["b"][l] in (2, 4, 8, 16)
+                assert t["d"][l] > 0 and t["b"][l] in (0, 2, 4, 8, 16)
             assert a[l] == last
         if "budget_bits" in t:
             bits = oracle_mod.bits_per_token(a, t["d"], t["b"], 64)
@@ -510,3 +510,31 @@ def test_grouped_quantiser_against_brute_force_and_bounds(oracle_mod, b, G):
     rows_hat = oracle_mod.dequant_grouped(codes, scales)
     assert np.array_equal(rows_hat[:, :G], codes[:, :G] * np.array(
         [oracle_mod.f16_bits_to_f64(int(x)) for x in scales[:, 0]])[:, None])
+
+
+# --------------------------------------------------------------------------
+# absorbed projections
+# --------------------------------------------------------------------------
+
+def test_absorb_against_brute_force_and_identity(oracle_mod):
+    """y[b, h, j] = sum_k x[b, h, k] w[h, k, j]: a brute-force loop on a tiny case, the
+    identity weight (y = x's first n coordinates), and a per-head weight that picks one head."""
+    rng = np.random.default_rng(51)
+    B, H, K, n = 2, 3, 5, 4
+    x = rng.standard_normal((B, H, K))
+    w = rng.standard_normal((H, K, n))
+    y = oracle_mod.absorb(x, w)
+    for b in range(B):
+        for h in range(H):
+            for j in range(n):
+                s = 0.0
+                for k in range(K):
+                    s += x[b, h, k] * w[h, k, j]
+                assert abs(y[b, h, j] - s) <= 1e-12 * max(1.0, abs(s))
+    eye = np.broadcast_to(np.eye(K, 3), (H, K, 3))
+    assert np.array_equal(oracle_mod.absorb(x, eye), x[:, :, :3])
+    sel = np.zeros((H, K, n))
+    sel[1, 2, :] = 1.0
+    y2 = oracle_mod.absorb(x, sel)
+    assert not y2[:, 0].any() and not y2[:, 2].any()
+    assert np.array_equal(y2[:, 1], np.repeat(x[:, 1, 2:3], n, axis=1))

@@ -14,6 +14,13 @@ shapes, 32 sequences x 8k tokens, the 1/8 eviction keep ratio, the budget sweep)
                 latent channel j scaled by std_j ~ U(0.5, 2) (per layer)
 * ``14b_evict`` as 14b with batch 16, 32768 tokens, sorted keep list of 4096 per sequence
 * ``14b_sweep`` as 14b with batch 8, 8192-token prefill, budgets 1x..16x, Student-t(3) latents
+
+Two fixed plans of the 14B shape (batch 32, 8192 tokens, latents as ``14b_4x``) bracket them:
+
+* ``14b_bf16``  every layer an uncompressed bf16 anchor with the full rank (d = 512): the MLA
+                cache the compression is measured against (C_0 / bits = 3.56)
+* ``14b_g32``   the composition of the M3 Ultra benchmark: 12 anchors (one per 4 layers) of
+                rank 128 at 4 bits with one fp16 scale per 32 elements (C_0 / bits = 151.7)
 """
 from __future__ import annotations
 
@@ -46,6 +53,7 @@ class Workload:
     b_set: tuple = ()
     seed: int = 0
     prefill: bool = False
+    scale_group: int = 0       # elements per fp16 scale (0: one scale per token)
     extra: dict = field(default_factory=dict)
 
 
@@ -59,6 +67,10 @@ WORKLOADS = {
     "14b_evict": Workload("14b_evict", 48, 40, 512, 64, 16, 32768, "bf16", "normal", n_kv=8,
                           d_h=128, keep=4096, budgets=(4,), d_set=(128, 256, 384, 512),
                           b_set=(4, 8, 16), seed=32),
+    "14b_bf16": Workload("14b_bf16", 48, 40, 512, 64, 32, 8192, "bf16", "channel_std", n_kv=8,
+                         d_h=128, seed=14),
+    "14b_g32": Workload("14b_g32", 48, 40, 512, 64, 32, 8192, "bf16", "channel_std", n_kv=8,
+                        d_h=128, seed=14, scale_group=32),
     "14b_sweep": Workload("14b_sweep", 48, 40, 512, 64, 8, 8192, "bf16", "student_t3", n_kv=8,
                           d_h=128, budgets=(1, 2, 4, 8, 16), d_set=(128, 256, 384, 512),
                           b_set=(2, 4, 8, 16), seed=16, prefill=True),
@@ -72,10 +84,20 @@ TINY_TABLES = {
 }
 
 
+# Fixed plans of the 14B shape (b = 0: an uncompressed bf16 anchor).
+FIXED_TABLES = {
+    "14b_bf16": {"anchor": list(range(48)), "d": [512] * 48, "b": [0] * 48},
+    "14b_g32": {"anchor": [4 * (l // 4) for l in range(48)],
+                "d": [128 if l % 4 == 0 else 0 for l in range(48)],
+                "b": [4 if l % 4 == 0 else 0 for l in range(48)]},
+}
+
+
 def load_tables() -> dict:
     with open(TABLES_PATH) as f:
         t = json.load(f)
     t.update({k: dict(v) for k, v in TINY_TABLES.items()})
+    t.update({k: dict(v) for k, v in FIXED_TABLES.items()})
     return t
 
 
