@@ -78,6 +78,23 @@ bool make_codes_tmap(CUtensorMap* m, void* base, int64_t rows, int row_bytes, in
   return r == CUDA_SUCCESS;
 }
 
+// One part of the query (latent or rope) as a 3D tensor [batch][H][elems] of 16-bit elements
+// with the caller's strides (in elements); box = 64 features x rows heads, 128-byte swizzle,
+// so that a box lands as one UMMA K-major atom.  Heads >= H and features >= elems read zero.
+bool make_query_tmap(CUtensorMap* m, const void* base, int64_t elems, int H, int batch,
+                     int64_t stride_head, int64_t stride_seq, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || elems < 1) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)elems, (cuuint64_t)H, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)stride_head * 2, (cuuint64_t)stride_seq * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 namespace kvk {
@@ -485,6 +502,23 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
     }
   }
 
+  // The tensor-core kernel copies each piece's query rows with TMA: tensor maps over the
+  // caller's query tensors, built per call (their addresses and strides are the call's).
+  CUtensorMap qmap_l, qmap_r;
+  memset(&qmap_r, 0, sizeof(qmap_r));
+  if (path == KVK_PATH_TENSOR) {
+    const int rows = kvk::tc_query_rows(n_heads);
+    bool ok = make_query_tmap(&qmap_l, q_lat, A.d, n_heads, batch, q_lat_stride_head,
+                              q_lat_stride_seq, rows);
+    if (ok && L->d_rope > 0)
+      ok = make_query_tmap(&qmap_r, q_rope, L->d_rope, n_heads, batch, q_rope_stride_head,
+                           q_rope_stride_seq, rows);
+    if (!ok) {
+      if (L->path == KVK_PATH_TENSOR) return KVK_ERR_UNSUPPORTED;
+      path = KVK_PATH_CUDA_CORE;
+    }
+  }
+
   kvk::DecodeArgs a;
   memset(&a, 0, sizeof(a));
   a.codes = L->arena + A.codes_off;
@@ -544,7 +578,7 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
     a.keep_idx = nullptr;
     a.keep_len = nullptr;
     a.keep_stride = 0;
-    if (e == cudaSuccess) e = kvk::launch_decode_tc(a, keep_tmap, dtype, st);
+    if (e == cudaSuccess) e = kvk::launch_decode_tc(a, keep_tmap, qmap_l, qmap_r, dtype, st);
   } else if (path == KVK_PATH_TENSOR) {
     if (app) {   // the decode kernel writes the new tokens itself
       a.app_c = app->c;
@@ -553,7 +587,7 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
       a.app_kr_ss = app->kr_ss;
       a.app_dtype = app->dtype;
     }
-    e = kvk::launch_decode_tc(a, A.tmap_tile, dtype, st);
+    e = kvk::launch_decode_tc(a, A.tmap_tile, qmap_l, qmap_r, dtype, st);
   } else {
     if (app)
       e = kvk::launch_quant_append(L, A, app->c, app->dtype, app->c_ss, app->kr, app->kr_ss,

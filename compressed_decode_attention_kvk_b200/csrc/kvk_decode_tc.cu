@@ -13,33 +13,37 @@
 //   warps 0-3  softmax: read S from TMEM, per-token scale, lazy online softmax, write P
 //              (f16) to shared memory, rescale O in TMEM when a max grows, write partials
 //   warps 4-11 convert: packed b-bit codes -> f16 operand tiles (UMMA 128-byte-swizzled,
-//              K-major) and their transpose into TMEM; staged query (power-of-two scaled).
-//              Two warps per SM sub-partition, 16 features of every 128-feature group each.
+//              K-major) and their transpose into TMEM.  Two teams of four warps take
+//              alternate 128-feature groups; in a group, warp w owns 32 features (its TMEM
+//              lane quarter of C^T).
 //   warp 12    TMA producer: 128-feature groups of 64 packed rows into a ring, and each
-//              tile's token scales; the stream is read once, so it carries an evict-first
-//              L2 policy
+//              tile's scales; the stream is read once, so it carries an evict-first L2 policy
 //   warp 13    score-MMA issuer (one thread) and TMEM owner
 //   warp 14    output-MMA issuer (one thread)
-//   warp 15    warms L2 with the queries of the CTA's later pieces
+//   warp 15    query warp: each piece's query rows by TMA, scaled to f16 in place; the fused
+//              append's new tokens; warms L2 with the queries of later pieces
 // Launched with 128 registers per thread; the softmax warpgroup raises its budget to
 // kRegsSoftmax, the conversion warpgroups lower theirs to kRegsConvert and the last
 // warpgroup to kRegsIssue (4 x 32 x (192 + 2 x 120 + 80) = 65536).
-// Per tile:  S^T[64 tok x N1 heads]  = C[64 x n] . Q^T         (M=64, A in smem, TMEM f32)
+// Per tile:  S^T[64 tok x N heads]   = C[64 x n] . Q^T         (A in smem, TMEM f32)
 //            O^T[128 feat x N2 heads] += C^T[128 x 64] . P    (M=128 per 128 latent features,
 //                                                               A = C^T in TMEM)
-// Heads sit on N, so 40 heads cost N = 40 / 48, never M = 128.  The convert warps turn each
-// 128-feature group into f16 in place (UMMA 128-byte swizzled, K-major: the score MMA's A)
-// and put their 16 features of it, transposed, into TMEM (tcgen05.st), so a ring slot is free
-// as soon as the score MMA has read it; the output MMA reads C^T from TMEM.  For 16-bit
-// codes both happen in one register pass (ldmatrix.trans, convert, stmatrix.trans back, the
-// same registers to TMEM); narrower codes are unpacked from a raw ring first and then
-// transposed with ldmatrix.trans.
-// The transpose fragment orders the 16 tokens of each K step as 0,1,8,9,2,3,10,11,4,5,12,13,
-// 6,7,14,15; the softmax warps write P's K rows in that same order.
-// Dequantisation: codes of b <= 8 bits are exact in f16; 16-bit codes are rounded to f16
-// (relative 2^-12).  The per-token scale s_t multiplies the S row and is folded into P as
-// p * s_t / S_run, with S_run a running power of two >= every scale seen so far (when it
-// grows, O is rescaled by the exact ratio).
+// Heads sit on N, so 40 heads cost N = 40 / 48, never M = 128.  Scores are exact for every
+// format: codes of b <= 8 bits and bf16 values are exact in f16; a 16-bit code c is split into
+// hi = f16(c) and lo = c - hi (both exact), and a group-scaled value c * s likewise.  Those
+// two parts form a stacked A operand: per 16-token block, the 16 rows of high parts and the 16
+// rows of low parts, so one M = 128 MMA per K step yields both partial scores, the high ones
+// of tokens 16q .. 16q + 15 in TMEM lanes 32q .. 32q + 15 and the low ones in lanes
+// 32q + 16 .. 32q + 31, which the softmax adds.  Otherwise the score MMA is M = 64.
+// The convert warps turn each group into f16 (in place for 16-bit rows, from a raw ring for
+// packed codes) and put their 32 features of it, transposed, into TMEM (tcgen05.st), so a ring
+// slot is free as soon as the score MMA has read it; the output MMA reads C^T from TMEM.  The
+// transpose fragment orders the 16 tokens of each K step as 0,1,8,9,2,3,10,11,4,5,12,13,6,7,
+// 14,15; the softmax warps write P's K rows in that same order.  C^T holds f16(code) (for 16-bit
+// codes rounded, relative 2^-12 on the output, inside its tolerance).
+// The per-token scale s_t multiplies the S row and is folded into P as p * s_t / S_run, with
+// S_run a running power of two >= every scale seen so far (when it grows, O is rescaled by the
+// exact ratio).
 // Every wait is bounded in time; on expiry the kernel records KVK_FLAG_TIMEOUT, drains its
 // own TMA loads and MMAs, frees TMEM and exits.
 #include <string.h>
@@ -60,6 +64,7 @@ constexpr int kTeamWarps = kConvWarps / 2;   // two conversion teams take altern
 constexpr int kTmaWarp = 12;
 constexpr int kMmaWarp = 13;   // score MMAs; owns TMEM
 constexpr int kMma2Warp = 14;  // output MMAs
+constexpr int kQueryWarp = 15; // query staging, fused append
 // Register budgets.  The block is launched with kLaunchRegs per thread (the host checks that
 // ptxas allocated exactly that before choosing this kernel); a warpgroup whose budget is
 // above it raises it (setmaxnreg.inc), one below lowers it (.dec) -- never the other way,
@@ -78,7 +83,6 @@ __device__ __forceinline__ void regs_set() {
 }
 constexpr int kTile = kTcTileTokens;   // 64
 constexpr int kAtom = 8192;            // 64 rows x 128 bytes (64 f16 features)
-constexpr int kPair = 2 * kAtom;       // 128 features
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol = 0;          // scores S^T, one buffer (N1 <= 64 columns)
 constexpr uint32_t kCtCol0 = 64;       // C^T double buffer: 64 + 128 b, latent group p at + 32 p
@@ -87,24 +91,26 @@ constexpr uint32_t kOCol0 = 320;       // O^T group p at 320 + N2 p
 constexpr uint64_t kDrainLimitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kSmemLimit = 232448;
-constexpr int kQC = 3;   // 16-byte chunks per lane per query row (rows of up to 768 features)
-constexpr int kQD = 1;   // query rows in flight per convert warp while staging
+// 16-byte chunks per lane of a half warp per staged query row (rows of up to 768 features)
+constexpr int kQL = 6;   // (a bound on the row: 16 kQL chunks of 8 features)
 // Scale ring: per tile one window of the tile's fp16 scales (64 tokens x sg scales, from the
 // 16-byte boundary at or below the first, rounded up to 16 bytes: 144 bytes for one scale per
 // token), loaded by the TMA warp with a plain bulk copy.
 constexpr int kScSlots = 4;
 // barriers besides the rings: s full/empty, P full/empty (2), C^T full/empty (2), q full/empty,
-// o empty, two MMA drains, q seen, appended, scale full/empty (kScSlots each)
-constexpr int kFixedBars = 2 + 4 + 4 + 7 + 2 * kScSlots;
+// o empty, two MMA drains, q seen, appended, q landed, scale full/empty (kScSlots each)
+constexpr int kFixedBars = 2 + 4 + 4 + 8 + 2 * kScSlots;
 
 struct TcParams {
   DecodeArgs a;
-  int N1, N2;           // N of the score MMA (heads rounded to 8) and of the output MMA (16)
+  int N1, N2;           // staged query rows (heads rounded to 8); N of the output MMA (to 16)
   int NP, NPd;          // 128-feature groups per row, and those holding latent features
   int NQA, NK16;        // 64-feature query atoms, 16-feature K steps
   int PR, RR, raw_slot; // ring slots (f16 groups, packed groups) and packed-group bytes
-  int LR;               // 16-bit codes: slots of the low parts (code - f16(code)) of a group
-  uint32_t off_lo;
+  int stacked;          // score A = exact high + low parts (16-bit codes, group scales): M = 128
+  uint32_t atom_bytes;  // one 64-feature atom of a group slot (8 KB, 16 KB stacked)
+  uint32_t slot_bytes;  // one group slot: 2 atoms
+  uint32_t rbs;         // bytes per 16-token block of an atom (2048, 4096 stacked)
   uint32_t lbo_p;       // bytes between the 8-token core-matrix rows of P (16 N2 + 32)
   uint32_t p_bytes;     // one P buffer: 8 lbo_p
   uint32_t off_p, off_pairs, off_raw, off_bar, off_misc;
@@ -199,14 +205,8 @@ __device__ __forceinline__ bool wait_warp(uint64_t* b, uint32_t parity, uint32_t
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-// two 16-bit offset-binary codes -> f16x2 of (u - 32768), rounded once:
-// code = (hi - 128) * 256 + lo with both parts exact in f16, fused multiply-add
-__device__ __forceinline__ uint32_t cvt_code16(uint32_t w) {
-  const __half2 hs = __hsub2(bits_h2(__byte_perm(w, 0x64u, 0x4341u)), __float2half2_rn(1152.f));
-  const __half2 ls = __hsub2(bits_h2(__byte_perm(w, 0x64u, 0x4240u)), __float2half2_rn(1024.f));
-  return h2_bits(__hfma2(hs, __float2half2_rn(256.f), ls));
-}
-// The same codes split exactly into two f16 parts, hi = f16(code) (rounded to nearest) and
+// Two 16-bit offset-binary codes, each split exactly into two f16 parts, hi = f16(code)
+// (rounded to nearest) and
 // lo = code - hi: with hb, lb the code's bytes (exact in f16), t = (hb - 128) * 256 - hi is an
 // integer of magnitude <= 263 (so the fused multiply-add is exact), and lo = t + lb an integer
 // of magnitude <= 8 (f16 spacing is at most 16 below 2^15): q . code = q . hi + q . lo exactly.
@@ -231,6 +231,17 @@ __device__ __forceinline__ uint32_t spread2(uint32_t x) {  // 4 x 2-bit fields -
   x = (x | (x << 12)) & 0x000F000Fu;
   x = (x | (x << 6)) & 0x03030303u;
   return x;
+}
+
+// Byte offset of token row r (0..63) of 64-feature atom a inside a group slot.  A plain slot
+// holds each atom's 64 rows contiguously (rbs = 2048: 16 rows of 128 bytes per block); a
+// stacked slot interleaves, per 16-token block, the 16 rows of high parts with the 16 rows of
+// low parts of the same tokens (rbs = 4096, low block at + kLoOff), so that one M = 128 score
+// MMA reads A rows [hi 0-15, lo 0-15, hi 16-31, lo 16-31, ...] and TMEM lane quarter q receives
+// the high and the low scores of tokens 16q .. 16q + 15.
+constexpr uint32_t kLoOff = 2048;
+__device__ __forceinline__ uint32_t slot_addr(int a, int r, uint32_t atom_bytes, uint32_t rbs) {
+  return (uint32_t)a * atom_bytes + (uint32_t)(r >> 4) * rbs + (uint32_t)(r & 15) * 128u;
 }
 
 // Row handled by `lane` in pass k of a convert warp (two lanes per row, one 16-byte chunk
@@ -274,13 +285,15 @@ __device__ __forceinline__ void load_group(const uint8_t* rawslot, int lane, int
 
 // SCALED: each row's f16 values are multiplied by that row's group scale sc[k] (both halves):
 // the dequantised value code * s of a group-scaled cache, split exactly into hi = f16(code * s)
-// (stored in `pair`) and lo = code * s - hi (stored at the same place in `lo_pair`; the fused
-// multiply-add is exact, the product of a b <= 8 bit code and an 11-bit scale having at most
-// 18 significant bits).
+// (stored at the row's place) and lo = code * s - hi (stored kLoOff bytes further, in the
+// stacked slot's low-part block of the same 16 tokens; the fused multiply-add is exact, the
+// product of a b <= 8 bit code and an 11-bit scale having at most 18 significant bits).
+// Token row r of atom a sits at a * atom_bytes + (r / 16) * rbs + (r % 16) * 128 (slot_addr).
 template <int BITS, bool SCALED>
 __device__ __forceinline__ void store_group(const uint32_t (&w)[4][kPackedWords<BITS>],
-                                            uint8_t* pair, uint8_t* lo_pair, int lane, int fb,
-                                            const __half2 (&sc)[4]) {
+                                            uint8_t* pair, int lane, int fb,
+                                            const __half2 (&sc)[4], uint32_t atom_bytes,
+                                            uint32_t rbs) {
   const int g = (fb >> 3) + (lane & 1);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -308,7 +321,7 @@ __device__ __forceinline__ void store_group(const uint32_t (&w)[4][kPackedWords<
       o.z = cvt_small(u1, 0x4140u, bias);
       o.w = cvt_small(u1, 0x4342u, bias);
     }
-    const int at = (g >> 3) * kAtom + r * 128 + (((g & 7) ^ (r & 7)) << 4);
+    const uint32_t at = slot_addr(g >> 3, r, atom_bytes, rbs) + (((g & 7) ^ (r & 7)) << 4);
     if constexpr (SCALED) {
       uint4 h, l;
       h.x = h2_bits(__hmul2(bits_h2(o.x), sc[k]));
@@ -320,7 +333,7 @@ __device__ __forceinline__ void store_group(const uint32_t (&w)[4][kPackedWords<
       l.z = h2_bits(__hfma2(bits_h2(o.z), sc[k], __hneg2(bits_h2(h.z))));
       l.w = h2_bits(__hfma2(bits_h2(o.w), sc[k], __hneg2(bits_h2(h.w))));
       *reinterpret_cast<uint4*>(pair + at) = h;
-      *reinterpret_cast<uint4*>(lo_pair + at) = l;
+      *reinterpret_cast<uint4*>(pair + at + kLoOff) = l;
     } else {
       *reinterpret_cast<uint4*>(pair + at) = o;
     }
@@ -344,7 +357,8 @@ __device__ __forceinline__ void load8_bits(const uint4 u, int dtype, float (&v)[
 
 template <int BITS, int NH>
 __global__ void __launch_bounds__(kThreads, 1)
-decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUtensorMap tmap) {
+decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUtensorMap tmap,
+                 const __grid_constant__ CUtensorMap qmap_l, const __grid_constant__ CUtensorMap qmap_r) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array by an offset so that every
   // pointer below stays in the shared state space (plain LDS / STS, not generic accesses)
@@ -355,15 +369,13 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   uint8_t* pairs = smem + P.off_pairs;
   uint8_t* raw = smem + P.off_raw;
   uint8_t* scw = smem + P.off_sc;         // [kScSlots] scale windows
-  uint8_t* los = smem + P.off_lo;         // [LR] low parts of 16-bit codes (f16, as pairs)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.off_bar);
   uint64_t* b_pfull = bars;               // [PR] group converted, visible to the tensor core
   uint64_t* b_pempty = b_pfull + P.PR;    // [PR] group released by the MMAs
   uint64_t* b_tfull = b_pempty + P.PR;    // [PR] 16-bit: TMA landed in the group slot
   uint64_t* b_rfull = b_tfull + P.PR;     // [RR] packed group landed
   uint64_t* b_rempty = b_rfull + P.RR;    // [RR] packed group consumed
-  uint64_t* b_loempty = b_rempty + P.RR;  // [LR] 16-bit: low-part slot released by the MMAs
-  uint64_t* b_sfull = b_loempty + P.LR;   // scores ready in TMEM
+  uint64_t* b_sfull = b_rempty + P.RR;    // scores ready in TMEM
   uint64_t* b_sempty = b_sfull + 1;       // scores read
   uint64_t* b_Pfull = b_sempty + 1;       // [2] P written
   uint64_t* b_Pempty = b_Pfull + 2;       // [2] output MMA of that P done
@@ -376,7 +388,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   uint64_t* b_final2 = b_final + 1;       // output-MMA drain
   uint64_t* b_qseen = b_final2 + 1;       // softmax has taken the piece's query scale
   uint64_t* b_app = b_qseen + 1;          // fused append: new tokens written
-  uint64_t* b_scfull = b_app + 1;         // [kScSlots] scale window landed
+  uint64_t* b_qload = b_app + 1;          // a piece's query rows landed (TMA)
+  uint64_t* b_scfull = b_qload + 1;       // [kScSlots] scale window landed
   uint64_t* b_scempty = b_scfull + kScSlots;   // [kScSlots] scale window read (last)
   Misc* m = reinterpret_cast<Misc*>(smem + P.off_misc);
   int32_t* off = reinterpret_cast<int32_t*>(m + 1);
@@ -395,7 +408,6 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       mbar_init(&b_rfull[i], 1);
       mbar_init(&b_rempty[i], kTeamWarps);
     }
-    for (int i = 0; i < P.LR; ++i) mbar_init(&b_loempty[i], 1);
     mbar_init(b_sfull, 1);
     mbar_init(b_sempty, 4);
     for (int i = 0; i < 2; ++i) {
@@ -411,6 +423,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     mbar_init(b_final2, 1);
     mbar_init(b_qseen, 4);
     mbar_init(b_app, 1);
+    mbar_init(b_qload, 1);
     for (int i = 0; i < kScSlots; ++i) {
       mbar_init(&b_scfull[i], 1);
       // released by the softmax warps (token scales) or the convert warps (group scales)
@@ -424,6 +437,10 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     tmem_relinquish();
   }
   if (warp == kTmaWarp && lane == 0) tma_prefetch_desc(&tmap);
+  if (warp == kQueryWarp && lane == 0) {
+    tma_prefetch_desc(&qmap_l);
+    if (a.d_rope > 0) tma_prefetch_desc(&qmap_r);
+  }
   block_seq_offsets(a, off, m->scan_tmp);   // contains __syncthreads
   if (blockIdx.x == 0)
     for (int i = tid; i <= a.batch; i += kThreads) a.seq_off[i] = off[i];
@@ -458,9 +475,9 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         uint32_t cnt = 0;
         Ring rg;
         const int slots = kInPlace<BITS> ? P.PR : P.RR;
-        // hold the first cache loads until the first query is staged: its loads then do not
-        // queue behind every CTA's ring fill
-        mbar_wait(b_qfull, 0u, abort, a.limit_ns);
+        // hold the first cache loads until the first query rows have landed: their loads then
+        // do not queue behind every CTA's ring fill
+        mbar_wait(b_qload, 0u, abort, a.limit_ns);
         // a fused append writes this CTA's new tokens first (the spare warp)
         if (a.app_c) mbar_wait(b_app, 0u, abort, a.limit_ns);
         Ring sr;   // scale ring
@@ -483,11 +500,13 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
             const uint32_t s = rg.slot, ph = rg.phase;
             if (kInPlace<BITS>) {
               if (!(ok = mbar_wait(&b_pempty[s], ph ^ 1u, abort, a.limit_ns))) break;
+              // each atom's 64 rows land contiguously at the start of the atom's place (a
+              // stacked slot's convert warps then move them into the interleaved layout)
               const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
               mbar_arrive_expect_tx(&b_tfull[s], nat * kAtom);
               for (int t = 0; t < nat; ++t)
-                tma_load_2d_hint(pairs + s * kPair + t * kAtom, &tmap, (2 * p + t) * 128, row0,
-                                 &b_tfull[s], pol);
+                tma_load_2d_hint(pairs + s * P.slot_bytes + t * P.atom_bytes, &tmap,
+                                 (2 * p + t) * 128, row0, &b_tfull[s], pol);
             } else {
               if (!(ok = mbar_wait(&b_rempty[s], ph ^ 1u, abort, a.limit_ns))) break;
               mbar_arrive_expect_tx(&b_rfull[s], P.raw_slot);
@@ -519,11 +538,13 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       Ring rg;
       // descriptors of slot 0 / atom 0; every other operand differs only in its start address
       // (bits 0-13, address >> 4), so each operand adds its byte offset >> 4
+      // A: M = 64 rows of one atom, or (stacked) M = 128 rows, the atom's interleaved high- and
+      // low-part blocks; B: the staged query atom (N = heads rounded to 8, or to 16 when
+      // stacked: rows past N1 are read from the next atom, or from the P buffers after the
+      // last one, and give score columns of heads >= H, which the softmax ignores)
       const uint64_t a0 = sdesc(smem_u32(pairs), 16u, 1024u, kLayoutSw128);
       const uint64_t b0 = sdesc(smem_u32(q_s), 16u, 1024u, kLayoutSw128);
-      const uint64_t l0 = sdesc(smem_u32(los), 16u, 1024u, kLayoutSw128);
       const uint32_t q_atom = (uint32_t)P.N1 * 128u;
-      Ring lr;   // low-part slots (16-bit codes)
       bool ok = true;
       while (g.valid && ok) {
         ok = mbar_wait(b_sempty, ((uint32_t)g.tile & 1u) ^ 1u, abort, a.limit_ns);
@@ -537,7 +558,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           for (int t = 0; t < 2; ++t) {
             const int atom = 2 * p + t;
             if (atom * 64 >= a.n) break;
-            const uint64_t ad = a0 + ((s * kPair + t * kAtom) >> 4);
+            const uint64_t ad = a0 + ((s * P.slot_bytes + t * P.atom_bytes) >> 4);
             const uint64_t bd = b0 + ((atom * q_atom) >> 4);
             const int k0 = atom * 4;
             if (k0 + 4 <= P.NK16) {
@@ -546,23 +567,9 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
               for (int ks = 0; k0 + ks < P.NK16; ++ks)
                 mma1_elect(tmem + kSCol, ad + 2u * ks, bd + 2u * ks, P.idesc1, (k0 + ks) > 0);
             }
-            if (BITS == 16 || P.grouped) {
-              // the low parts of the same rows: S += (c - f16(c)) . Q, exact in f16
-              const uint64_t ld = l0 + ((lr.slot * kPair + t * kAtom) >> 4);
-              if (k0 + 4 <= P.NK16) {
-                mma4_elect(tmem + kSCol, ld, 2u, bd, 2u, P.idesc1, 1u);
-              } else {
-                for (int ks = 0; k0 + ks < P.NK16; ++ks)
-                  mma1_elect(tmem + kSCol, ld + 2u * ks, bd + 2u * ks, P.idesc1, 1u);
-              }
-            }
           }
           commit_elect(&b_pempty[s]);   // this group's share of the slot release
           rg.next(P.PR);
-          if (BITS == 16 || P.grouped) {
-            commit_elect(&b_loempty[lr.slot]);
-            lr.next(P.LR);
-          }
         }
         if (!ok) break;
         commit_elect(b_sfull);
@@ -603,10 +610,32 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       if (lane == 0) wait_noabort(b_final2, 0);
       __syncwarp();
     } else {
-      // ------------------------------------------------------------------ spare warp
+      // ------------------------------------------------------------------ query warp
+      // Loads each piece's query rows [N1][n] with TMA into the 64-feature atoms of the score
+      // MMAs' B (heads >= H and features past each part zero-filled); the convert warps then
+      // scale and convert them in place.
+      const int lat_atoms = a.d / 64;
+      const uint32_t q_atom = (uint32_t)P.N1 * 128u;
+      auto issue_q = [&](int seq) {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(b_qload, (uint32_t)P.NQA * q_atom);
+          for (int at = 0; at < P.NQA; ++at) {
+            if (at < lat_atoms) tma_load_3d(q_s + at * q_atom, &qmap_l, 64 * at, 0, seq, b_qload);
+            else tma_load_3d(q_s + at * q_atom, &qmap_r, 64 * (at - lat_atoms), 0, seq, b_qload);
+          }
+        }
+        __syncwarp();
+      };
+      Cursor c;
+      cursor_start(c, seq0, off, a.batch, lo, hi);
+      uint32_t nq = 0;   // query loads issued
+      if (c.valid) {
+        issue_q(c.seq);
+        ++nq;
+      }
       // Fused append: the new token of every sequence whose last position this CTA owns is
       // quantised (the write kernel's arithmetic) and stored before the TMA warp issues any
-      // load; the proxy fence makes those generic stores visible to its async-proxy reads.
+      // cache load; the proxy fence makes those generic stores visible to its async-proxy reads.
       if (a.app_c) {
         uint8_t* codes_w = const_cast<uint8_t*>(a.codes);
         __half* scales_w = const_cast<__half*>(a.scales);
@@ -636,29 +665,48 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         __syncwarp();
         if (lane == 0) mbar_arrive(b_app);
       }
-      // Warm L2 with the queries of the sequences after the first that this CTA touches
-      // (the convert warps stage the first one at once).
-      Cursor c;
-      cursor_start(c, seq0, off, a.batch, lo, hi);
-      const int lat_lines = (2 * a.d + 127) / 128, rope_lines = (2 * a.d_rope + 127) / 128;
-      const int lines = lat_lines + rope_lines;
-      while (c.valid) {
-        ++c.seq;
-        if (!(c.valid = find_piece(c, off, a.batch, lo, hi))) break;
-        const uint8_t* ql = static_cast<const uint8_t*>(a.q_lat) + 2 * ((int64_t)c.seq * a.ql_ss);
-        const uint8_t* qr = static_cast<const uint8_t*>(a.q_rope) + 2 * ((int64_t)c.seq * a.qr_ss);
-        for (int i = lane; i < a.H * lines; i += 32) {
-          const int h = i / lines, k = i - h * lines;
-          if (k < lat_lines) prefetch_l2(ql + 2 * ((int64_t)h * a.ql_sh) + 128 * k);
-          else prefetch_l2(qr + 2 * ((int64_t)h * a.qr_sh) + 128 * (k - lat_lines));
+      // Warm L2 with the queries of the later pieces (their TMA loads then hit L2).
+      {
+        Cursor w = c;
+        const int lat_lines = (2 * a.d + 127) / 128, rope_lines = (2 * a.d_rope + 127) / 128;
+        const int lines = lat_lines + rope_lines;
+        while (w.valid) {
+          ++w.seq;
+          if (!(w.valid = find_piece(w, off, a.batch, lo, hi))) break;
+          const uint8_t* ql = static_cast<const uint8_t*>(a.q_lat) + 2 * ((int64_t)w.seq * a.ql_ss);
+          const uint8_t* qr =
+              static_cast<const uint8_t*>(a.q_rope) + 2 * ((int64_t)w.seq * a.qr_ss);
+          for (int i = lane; i < a.H * lines; i += 32) {
+            const int h = i / lines, k = i - h * lines;
+            if (k < lat_lines) prefetch_l2(ql + 2 * ((int64_t)h * a.ql_sh) + 128 * k);
+            else prefetch_l2(qr + 2 * ((int64_t)h * a.qr_sh) + 128 * (k - lat_lines));
+          }
         }
       }
+      // Later pieces: the rows of piece k are loaded once piece k-1's score MMAs are done
+      // with the atoms and the softmax warps have taken its scales; the convert warps scale
+      // them when they reach the piece.
+      bool fail = false;
+      for (int piece = 1; !fail; ++piece) {
+        ++c.seq;
+        if (!(c.valid = find_piece(c, off, a.batch, lo, hi))) break;
+        fail = !wait_warp(b_qempty, ((uint32_t)piece & 1u) ^ 1u, abort, a.limit_ns) ||
+               !wait_warp(b_qseen, ((uint32_t)piece - 1u) & 1u, abort, a.limit_ns);
+        if (!fail) {
+          issue_q(c.seq);
+          ++nq;
+        }
+      }
+      // the last query load this warp issued has landed before the block exits (after an
+      // abort it may still be in flight)
+      if (nq > 0 && lane == 0) wait_noabort(b_qload, (nq - 1) & 1u);
+      __syncwarp();
     }
   } else if (has_work && warp >= kConvWarp0) {
     regs_set<kRegsConvert>();
     // ------------------------------------------------------------------ convert
-    // Two teams of four warps take alternate groups (team cw / 4 converts the groups p with
-    // p % 2 == team), so two groups are in flight; in its team's groups warp cw owns the 32
+    // Two teams of four warps take alternate groups (team cw / 4 converts the CTA's groups with
+    // the team's parity), so two groups are in flight; in its team's groups warp cw owns the 32
     // features 32 cq .. 32 cq + 31 (cq = cw % 4), which are its own TMEM lane quarter of C^T.
     // The warps share no barrier among themselves (every hand-off is an mbarrier), so a warp
     // that stops on a failed wait leaves its loop alone; it then arrives on nothing more, and
@@ -667,35 +715,39 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     const int cq = cw & 3, team = cw >> 2;
     Ring pr, rr;   // f16 group ring, packed group ring
     Ring sr;       // scale windows (group-scaled cache only)
-    int last_piece = -1;
     bool fail = false;
-    const int cpr = P.NQA * 8;   // 16-byte chunks per staged query row
     // this lane's ldmatrix row address inside a group slot, per 16-feature half h and 16-token
     // block tg: atom cq/2, 16-byte chunk 4(cq%2) + 2h + (lane/8)/2 of token
-    // 16tg + 8((lane/8)%2) + lane%8
-    uint32_t aoff[2][4];
+    // 16tg + 8((lane/8)%2) + lane%8, in the slot's layout (aoff; the low part of a stacked
+    // slot at + kLoOff) and, for 16-bit rows, where TMA put it (roff: the atom's 64 rows
+    // contiguous from the atom's start; the same as aoff in a plain slot).  Both keep the
+    // 128-byte swizzle phase (token % 8), so a warp's cells stay in its own 16-byte columns:
+    // it reads all of them (ldmatrix) before it writes any, and no other warp touches them.
+    uint32_t aoff[2][4], roff[2][4];
     {
       const int mi = lane >> 3, r8 = lane & 7;
 #pragma unroll
       for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int tg = 0; tg < 4; ++tg)
-          aoff[h][tg] = (uint32_t)((cq >> 1) * kAtom + (16 * tg + 8 * (mi & 1) + r8) * 128 +
-                                   (((4 * (cq & 1) + 2 * h + (mi >> 1)) ^ r8) << 4));
+        for (int tg = 0; tg < 4; ++tg) {
+          const int tok = 16 * tg + 8 * (mi & 1) + r8;
+          const uint32_t col = (uint32_t)(((4 * (cq & 1) + 2 * h + (mi >> 1)) ^ r8) << 4);
+          aoff[h][tg] = slot_addr(cq >> 1, tok, P.atom_bytes, P.rbs) + col;
+          roff[h][tg] = (uint32_t)(cq >> 1) * P.atom_bytes + (uint32_t)tok * 128u + col;
+        }
     }
     const uint32_t pairs_u = smem_u32(pairs);
-    const uint32_t los_u = smem_u32(los);
-    Ring lr;   // low-part slots
     // does this warp own features of group p (the last group may hold only one atom)?
     auto owns_group = [&](int p) { return (cq >> 1) < (((2 * p + 1) * 64 < a.n) ? 2 : 1); };
-    // ldmatrix (transposed) of this warp's 32 features x 64 tokens of a group slot
-    auto ldsm32 = [&](uint32_t base, uint32_t (&x)[32]) {
+    // ldmatrix (transposed) of this warp's 32 features x 64 tokens of a group slot, in the
+    // slot layout (off = aoff) or as TMA left them (off = roff)
+    auto ldsm32 = [&](uint32_t base, const uint32_t (&off)[2][4], uint32_t (&x)[32]) {
 #pragma unroll
       for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int tg = 0; tg < 4; ++tg) {
           uint32_t d4[4];
-          ldsm_x4_trans(base + aoff[h][tg], d4);
+          ldsm_x4_trans(base + off[h][tg], d4);
 #pragma unroll
           for (int i = 0; i < 4; ++i) x[16 * h + 4 * tg + i] = d4[i];
         }
@@ -720,108 +772,90 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     };
     Cursor c;
     cursor_start(c, seq0, off, a.batch, lo, hi);
+    const uint32_t q_atom = (uint32_t)P.N1 * 128u;
+    const int cpr = P.NQA * 8;   // 16-byte chunks per staged query row
+    const int hs = lane >> 4, l16 = lane & 15;
     while (c.valid) {
       if (fail || abort_read(abort)) break;
-      if (c.piece != last_piece) {
-        // Stage this sequence's query as f16 rows [N1][n], scaled by 2^e so that max |q|
-        // lands in [2^14, 2^15) (exact for bf16 inputs in range); rows >= H and features
-        // >= n are zero.  Wait until the previous piece's scores no longer read it and the
-        // softmax warps have taken the previous piece's scale (bounds q_full to one phase
-        // ahead of its slowest waiter).
-        fail = fail || !wait_warp(b_qempty, ((uint32_t)c.piece & 1u) ^ 1u, abort, a.limit_ns);
-        if (c.piece > 0)
-          fail = fail || !wait_warp(b_qseen, ((uint32_t)c.piece - 1u) & 1u, abort, a.limit_ns);
-        const uint8_t* qlat = static_cast<const uint8_t*>(a.q_lat) + 2 * ((int64_t)c.seq * a.ql_ss);
-        const uint8_t* qrope =
-            static_cast<const uint8_t*>(a.q_rope) + 2 * ((int64_t)c.seq * a.qr_ss);
-        // One pass: warp cw stages heads cw, cw + 8, ...; lane l holds chunks l, l + 32, ... of
-        // a row, the warp reduces the row's max |q|, and the row is written scaled by 2^e_h
-        // (max |q_h| in [2^14, 2^15), exact for bf16 inputs in range).  Rows >= H and chunks
-        // >= n are zero.  The loop body is one row (a small code footprint: this code runs
-        // once per piece and would otherwise be fetched cold); the loads of the next kQD rows
-        // are in flight while a row is processed.
-        auto load_row = [&](int h, uint4 (&v)[kQC]) {
-#pragma unroll
-          for (int j = 0; j < kQC; ++j) {
-            const int f0 = 8 * (lane + 32 * j);
-            v[j] = make_uint4(0u, 0u, 0u, 0u);
-            if (h < a.H && f0 < a.n)
-              v[j] = *reinterpret_cast<const uint4*>(
-                  (f0 < a.d) ? qlat + 2 * ((int64_t)h * a.ql_sh + f0)
-                             : qrope + 2 * ((int64_t)h * a.qr_sh + (f0 - a.d)));
-          }
-        };
-        uint4 v[kQD + 1][kQC];
-#pragma unroll
-        for (int i = 0; i < kQD; ++i)
-          if (cw + kConvWarps * i < P.N1) load_row(cw + kConvWarps * i, v[i]);
+      if (c.first) {
+        // Stage the piece's query once its rows have landed: row h scaled by 2^e_h so that
+        // max |q_h| lands in [2^14, 2^15) (exact for bf16 inputs in range) and rounded to f16
+        // in place; the softmax warps apply 2^-e_h.  Each warp takes row pairs 2 cw + 16 i
+        // (one row per half warp; lane l16 holds the row's 16-byte chunks l16, l16 + 16, ...).
+        fail = fail || !wait_warp(b_qload, (uint32_t)c.piece & 1u, abort, a.limit_ns);
+        if (fail) break;
 #pragma unroll 1
-        for (int h = cw; h < P.N1; h += kConvWarps) {
-          if (h + kConvWarps * kQD < P.N1) load_row(h + kConvWarps * kQD, v[kQD]);
-          float f[kQC][8];
+        for (int hb = 2 * cw; hb < P.N1; hb += 2 * kConvWarps) {
+          // compact loops: this code runs once per piece, so it is mostly fetched cold
+          const int h = hb + hs;
+          const uint32_t rbase = smem_u32(q_s) + (uint32_t)h * 128u;
           float mx = 0.f;
+#pragma unroll 1
+          for (int fc = l16; fc < cpr; fc += 16) {
+            float f[8];
+            load8_bits(lds128(rbase + (fc >> 3) * q_atom + (((fc & 7) ^ (h & 7)) << 4)), P.qdtype,
+                       f);
 #pragma unroll
-          for (int j = 0; j < kQC; ++j) {
-            load8_bits(v[0][j], P.qdtype, f[j]);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[j][e]));
+            for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
           }
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
           // e = 14 - floor(log2 max |q|) from the exponent field (a subnormal max counts as
           // 2^-126), at most 126 so that 2^e and 2^-e are normal floats
           int e = 0;
           if (mx > 0.f && isfinite(mx))
             e = min(14 - (max((__float_as_int(mx) >> 23) & 0xff, 1) - 127), 126);
           const float qscale = __int_as_float((127 + e) << 23);
-          if (lane == 0) m->qs_inv[c.piece & 1][h] = __int_as_float((127 - e) << 23);
-#pragma unroll
-          for (int j = 0; j < kQC; ++j) {
-            const int fc = lane + 32 * j;
-            if (fc >= cpr) break;
+          if (l16 == 0) m->qs_inv[c.piece & 1][h] = __int_as_float((127 - e) << 23);
+#pragma unroll 1
+          for (int fc = l16; fc < cpr; fc += 16) {
+            const uint32_t addr = rbase + (fc >> 3) * q_atom + (((fc & 7) ^ (h & 7)) << 4);
+            float f[8];
+            load8_bits(lds128(addr), P.qdtype, f);
             uint4 o;
-            o.x = h2_bits(__floats2half2_rn(f[j][0] * qscale, f[j][1] * qscale));
-            o.y = h2_bits(__floats2half2_rn(f[j][2] * qscale, f[j][3] * qscale));
-            o.z = h2_bits(__floats2half2_rn(f[j][4] * qscale, f[j][5] * qscale));
-            o.w = h2_bits(__floats2half2_rn(f[j][6] * qscale, f[j][7] * qscale));
-            const int at = fc >> 3, jj = fc & 7;
-            *reinterpret_cast<uint4*>(q_s + at * (P.N1 * 128) + h * 128 + ((jj ^ (h & 7)) << 4)) = o;
+            o.x = h2_bits(__floats2half2_rn(f[0] * qscale, f[1] * qscale));
+            o.y = h2_bits(__floats2half2_rn(f[2] * qscale, f[3] * qscale));
+            o.z = h2_bits(__floats2half2_rn(f[4] * qscale, f[5] * qscale));
+            o.w = h2_bits(__floats2half2_rn(f[6] * qscale, f[7] * qscale));
+            sts128(addr, o);
           }
-#pragma unroll
-          for (int i = 0; i < kQD; ++i)
-#pragma unroll
-            for (int j = 0; j < kQC; ++j) v[i][j] = v[i + 1][j];
         }
-        // q_full counts one arrival per convert warp, each after its own rows are written
-        fence_proxy_async_smem();
+        fence_proxy_async_smem();   // the generic writes, visible to the score MMAs
         __syncwarp();
-        if (lane == 0 && !fail) mbar_arrive(b_qfull);
-        last_piece = c.piece;
+        if (lane == 0) mbar_arrive(b_qfull);
       }
       const int ctb = c.tile & 1;   // C^T buffer of this tile
       const uint32_t ct_col = kCtCol0 + 128u * ctb;
       // the output MMAs of tile - 2 have finished reading this C^T buffer (waited before the
-      // team's first store of the tile)
+      // team's first store of the tile, and by every warp before it arrives on the buffer's
+      // full barrier: a team that stores no C^T -- the one converting only the rope group when
+      // d <= 128 -- would otherwise run two tiles ahead and arrive twice in one phase)
+      bool ct_waited = false;
+      // the teams take alternate groups of the CTA's whole group sequence (with an odd number
+      // of groups per tile, each team's share alternates between tiles)
+      const int gbase = c.tile * P.NP;
       auto wait_ct = [&]() {
         fail = fail || !wait_warp(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u, abort,
                                   a.limit_ns);
         tc_fence_after();
+        ct_waited = true;
       };
-      const bool low_parts = (BITS == 16) || P.grouped;   // score MMAs add exact low parts
       if constexpr (kInPlace<BITS>) {
         // In place, 16-bit codes (or bf16 values) -> f16, in one pass through registers: each
         // 8x8 block (8 tokens x 8 features) is loaded transposed, converted element by
-        // element, stored back transposed (row-major again, for the score MMAs) and the same
-        // registers, now feature-major, go to C^T in TMEM.  The slot is not read after q_full,
-        // so only the score MMAs release it.
+        // element, stored back transposed (row-major again, for the score MMAs; 16-bit codes
+        // as exact high and low parts in the stacked slot) and the same registers, now
+        // feature-major, go to C^T in TMEM.  The slot is not read after p_full, so only the
+        // score MMAs release it.
         for (int p = 0; p < P.NP; ++p) {
-          if ((p & 1) == team) {
+          if (((p + gbase) & 1) == team) {
             const uint32_t s = pr.slot;
             fail = fail || !wait_warp(&b_tfull[s], pr.phase, abort, a.limit_ns);
             const bool go = !fail && owns_group(p);
+            const uint32_t sbase = pairs_u + s * P.slot_bytes;
             uint32_t x[32], xl[32];
             if (go) {
-              ldsm32(pairs_u + s * (uint32_t)kPair, x);
+              ldsm32(sbase, roff, x);
               if constexpr (BITS == 16) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) cvt_code16_split(x[i], x[i], xl[i]);
@@ -840,22 +874,19 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
                 }
               }
             }
-            if constexpr (BITS == 16)   // the low-part slot is free once its MMAs are done
-              fail = fail || !wait_warp(&b_loempty[lr.slot], lr.phase ^ 1u, abort, a.limit_ns);
             if (go && !fail) {
-              stsm32(pairs_u + s * (uint32_t)kPair, x);
-              if constexpr (BITS == 16) stsm32(los_u + lr.slot * (uint32_t)kPair, xl);
+              stsm32(sbase, x);
+              if constexpr (BITS == 16) stsm32(sbase + kLoOff, xl);
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0 && !fail) mbar_arrive(&b_pfull[s]);
             if (p < P.NPd) {
-              if (p == team) wait_ct();
+              if (!ct_waited) wait_ct();
               if (go && !fail) tmem_st32(ct_col + 32u * p, x);
             }
           }
           pr.next(P.PR);
-          if constexpr (BITS == 16) lr.next(P.LR);
         }
       } else {
         // Packed codes: the team's group is read from the raw ring into registers (and the raw
@@ -872,9 +903,9 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
                                                              a.sg) & 15u) >> 1);
         }
         for (int p = 0; p < P.NP; ++p) {
-          if ((p & 1) == team) {
+          if (((p + gbase) & 1) == team) {
             const uint32_t s = pr.slot, ph = pr.phase, rs = rr.slot;
-            uint8_t* pair = pairs + s * kPair;
+            uint8_t* pair = pairs + s * P.slot_bytes;
             uint32_t w[2][4][NW];
             fail = fail || !wait_warp(&b_rfull[rs], rr.phase, abort, a.limit_ns);
             if (!fail) {
@@ -884,8 +915,6 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
             __syncwarp();
             if (lane == 0 && !fail) mbar_arrive(&b_rempty[rs]);
             fail = fail || !wait_warp(&b_pempty[s], ph ^ 1u, abort, a.limit_ns);
-            if (P.grouped)   // the low-part slot is free once its MMAs are done
-              fail = fail || !wait_warp(&b_loempty[lr.slot], lr.phase ^ 1u, abort, a.limit_ns);
             if (!fail) {
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
@@ -900,10 +929,10 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
                     const __half sv = (r < c.cnt) ? wsc[r * a.sg + j] : __float2half(0.f);
                     sc[k] = __halves2half2(sv, sv);
                   }
-                  store_group<BITS, true>(w[h], pair, los + lr.slot * kPair, lane, fb, sc);
+                  store_group<BITS, true>(w[h], pair, lane, fb, sc, P.atom_bytes, P.rbs);
                 } else {
                   const __half2 one[4] = {};
-                  store_group<BITS, false>(w[h], pair, nullptr, lane, fb, one);
+                  store_group<BITS, false>(w[h], pair, lane, fb, one, P.atom_bytes, P.rbs);
                 }
               }
             }
@@ -911,10 +940,10 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
             __syncwarp();
             if (lane == 0 && !fail) mbar_arrive(&b_pfull[s]);
             if (p < P.NPd) {
-              if (p == team) wait_ct();
+              if (!ct_waited) wait_ct();
               if (!fail && owns_group(p)) {
                 uint32_t x[32];
-                ldsm32(smem_u32(pair), x);
+                ldsm32(smem_u32(pair), aoff, x);
                 tmem_st32(ct_col + 32u * p, x);
               }
             }
@@ -923,7 +952,6 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           }
           pr.next(P.PR);
           rr.next(P.RR);
-          if (P.grouped) lr.next(P.LR);
         }
         if (P.grouped) {   // the tile's scale window is no longer read by this warp
           __syncwarp();
@@ -931,7 +959,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           sr.next(kScSlots);
         }
       }
-      (void)low_parts;
+      if (!ct_waited) wait_ct();
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -942,15 +970,26 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   } else if (has_work) {
     regs_set<kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax
-    // TMEM holds S^T with tokens on lanes: the M = 64 layout puts rows 16q .. 16q+15 in
-    // lanes 32q .. 32q+15.  Loaded with the 16x256b shape, thread t of warp q holds rows
-    // ra = 16q + t/4 and rb = ra + 8, heads 8j + 2(t%4) + {0, 1} of every 8-head block j.
-    // The four warps leave the loop only together (named_or agreement every tile).
-    constexpr int NB = NH / 8;
+    // Thread layout: lane t of warp q holds token r = 16q + t % 16 of the tile and the HH = NH/2
+    // heads h0 .. h0 + HH - 1, h0 = HH (t / 16).  S^T is read with the 32x32b shape (thread t
+    // <-> TMEM lane 32q + t, every column):
+    //  - M = 64 score MMA: rows 16q .. 16q + 15 sit in lanes 32q .. 32q + 15 and lanes 16-31 of
+    //    the quarter hold nothing, so thread t >= 16 takes its heads of token 16q + t - 16 from
+    //    lane t - 16;
+    //  - stacked M = 128 score MMA: lane 32q + t (t < 16) holds the high-part scores of token
+    //    16q + t and lane 32q + 16 + t its low-part scores, and each thread adds the other
+    //    lane's partial scores of its heads.
+    // One shuffle per head either way.  The four warps leave the loop only together (named_or
+    // agreement every tile).
+    constexpr int HH = NH / 2;
+    constexpr int NHB = HH / 8;   // 8-head blocks of a thread
     const int q = warp;
     const uint32_t lb = tmem + ((uint32_t)(32 * q) << 16);
-    const int ra = 16 * q + (lane >> 2), rb = ra + 8;
-    const int hc = 2 * (lane & 3);
+    const int hf = lane >> 4;
+    const int u = lane & 15;
+    const int r = 16 * q + u;     // this thread's token in the tile
+    const int h0 = HH * hf;       // this thread's first head
+    const bool stacked = P.stacked != 0;
     bool fail = false;
 
     // S_run: running power of two >= every token scale seen so far (P = p * s / S_run keeps
@@ -958,34 +997,32 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     // rescales O by S_old / S_new, exactly (powers of two), together with any max update.
     float srun = 0.f, inv_srun = 0.f;
 
-    float l[2 * NB];    // partial weight sums of this thread's heads
-    float mr[2 * NB];   // reference max of this thread's heads (log2 units)
-    float qh[2 * NB];   // 2^-e_h of this thread's heads 8j + hc + {0, 1} in the current piece
+    float l[HH];    // partial weight sums of this thread's heads (its token)
+    float mr[HH];   // reference max of this thread's heads (log2 units)
+    float qh[HH];   // 2^-e_h of this thread's heads in the current piece
     int pt = 0;
     Cursor c;
     cursor_start(c, seq0, off, a.batch, lo, hi);
     const float coef0 = a.sigma * kLog2e;
-    // K slot of this thread's rows in P: the transposed C^T holds, in the 16 K slots of each
-    // step, tokens 0,1,8,9,2,3,10,11,4,5,12,13,6,7,14,15 of the step's 16 tokens
-    const int ka = 16 * q + 4 * (lane >> 3) + ((lane >> 2) & 1), kb = ka + 2;
-    // Token scales of rows ra / rb come from the tile's scale window in shared memory
-    // (bulk-copied by the TMA warp at least a tile ahead): no global loads in this role, so
-    // the proxy fence after each P write has nothing outstanding to wait for.
+    // K slot of token r in P: the transposed C^T holds, in the 16 K slots of each step, tokens
+    // 0,1,8,9,2,3,10,11,4,5,12,13,6,7,14,15 of the step's 16 tokens
+    const int kslot = 16 * q + 4 * ((u & 7) >> 1) + 2 * (u >> 3) + (u & 1);
+    // Token scales come from the tile's scale window in shared memory (bulk-copied by the TMA
+    // warp at least a tile ahead): no global loads in this role, so the proxy fence after each
+    // P write has nothing outstanding to wait for.
     Ring sr;
     while (c.valid) {
       const int t = c.tile, sb = t & 1;
-      float s_a = 0.f, s_b = 0.f;
+      float s_r = 0.f;
       if (BITS == 0 || (!kInPlace<BITS> && P.grouped)) {
         // uncompressed rows, or scales applied per group by the convert warps: unit token scale
-        s_a = (ra < c.cnt) ? 1.f : 0.f;
-        s_b = (rb < c.cnt) ? 1.f : 0.f;
+        s_r = (r < c.cnt) ? 1.f : 0.f;
       } else {
         fail = fail || !mbar_wait(&b_scfull[sr.slot], sr.phase, abort, a.limit_ns);
         const __half* w = reinterpret_cast<const __half*>(scw + sr.slot * P.sc_bytes) +
                           ((reinterpret_cast<uintptr_t>(a.scales + (int64_t)c.seq * a.max_tokens +
                                                         c.pos) & 15u) >> 1);
-        if (ra < c.cnt) s_a = __half2float(w[ra]);
-        if (rb < c.cnt) s_b = __half2float(w[rb]);
+        if (r < c.cnt) s_r = __half2float(w[r]);
         __syncwarp();
         if (lane == 0 && !fail) mbar_arrive(&b_scempty[sr.slot]);
         sr.next(kScSlots);
@@ -993,80 +1030,68 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       if (c.first) {
         fail = fail || !mbar_wait(b_qfull, (uint32_t)c.piece & 1u, abort, a.limit_ns);
 #pragma unroll
-        for (int j = 0; j < NB; ++j)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) qh[2 * j + e] = m->qs_inv[c.piece & 1][8 * j + hc + e];
+        for (int j = 0; j < HH; ++j) qh[j] = m->qs_inv[c.piece & 1][h0 + j];
         __syncwarp();
         if (lane == 0 && !fail) mbar_arrive(b_qseen);
 #pragma unroll
-        for (int i = 0; i < 2 * NB; ++i) {
-          l[i] = 0.f;
-          mr[i] = -INFINITY;
+        for (int j = 0; j < HH; ++j) {
+          l[j] = 0.f;
+          mr[j] = -INFINITY;
         }
         pt = 0;
       }
-      const bool va = ra < c.cnt, vb = rb < c.cnt;
-      const float ca = coef0 * s_a, cbf = coef0 * s_b;
+      const bool vr = r < c.cnt;
+      const float cr = coef0 * s_r;
       fail = fail || !mbar_wait(b_sfull, (uint32_t)t & 1u, abort, a.limit_ns);
       tc_fence_after();
-      float x[4 * NB];
-      if constexpr (NB == 8) {
-        float v[32];
-        tmem_ld16x256b_x8(lb + kSCol, v);
+      float x[HH];
+      // columns j and HH + j of the thread's lane, in kSplit rounds (fewer live registers at
+      // 64 heads)
+      constexpr int kSplit = (NH == 64) ? 2 : 1;
+      constexpr int CH = HH / kSplit;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = v[i];
-      } else if constexpr (NB == 6) {   // columns 0-31 and 32-47
-        float v[16], w[8];
-        tmem_ld16x256b_x4(lb + kSCol, v);
-        tmem_ld16x256b_x2(lb + kSCol + 32u, w);
+      for (int sp = 0; sp < kSplit; ++sp) {
+        float v[2 * CH];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = v[i];
+        for (int k = 0; k < CH / 8; ++k) {
+          tmem_ld8(lb + kSCol + (uint32_t)(sp * CH + 8 * k), *reinterpret_cast<float(*)[8]>(v + 8 * k));
+          tmem_ld8(lb + kSCol + (uint32_t)(HH + sp * CH + 8 * k),
+                   *reinterpret_cast<float(*)[8]>(v + CH + 8 * k));
+        }
+        tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 8; ++i) x[16 + i] = w[i];
-      } else if constexpr (NB == 4) {
-        float v[16];
-        tmem_ld16x256b_x4(lb + kSCol, v);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = v[i];
-      } else {
-        float v[8];
-        tmem_ld16x256b_x2(lb + kSCol, v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = v[i];
+        for (int j = 0; j < CH; ++j) {
+          const float send = (stacked && hf) ? v[j] : v[CH + j];
+          const float y = __shfl_xor_sync(0xffffffffu, send, 16);
+          const float own = hf ? v[CH + j] : v[j];
+          x[sp * CH + j] = stacked ? own + y : (hf ? y : own);
+        }
       }
-      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0 && !fail) mbar_arrive(b_sempty);
-      bool mine = (pt == 0) || s_a > srun || s_b > srun;
+      bool mine = (pt == 0) || s_r > srun;
 #pragma unroll
-      for (int j = 0; j < NB; ++j) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const bool hv = (8 * j + hc + e) < a.H;
-          x[4 * j + e] = (va && hv) ? x[4 * j + e] * qh[2 * j + e] * ca : -INFINITY;
-          x[4 * j + 2 + e] = (vb && hv) ? x[4 * j + 2 + e] * qh[2 * j + e] * cbf : -INFINITY;
-          mine = mine || (x[4 * j + e] > mr[2 * j + e] + 8.f) ||
-                 (x[4 * j + 2 + e] > mr[2 * j + e] + 8.f);
-        }
+      for (int j = 0; j < HH; ++j) {
+        const bool hv = (h0 + j) < a.H;
+        x[j] = (vr && hv) ? x[j] * qh[j] * cr : -INFINITY;
+        mine = mine || (x[j] > mr[j] + 8.f);
       }
       // lazy running max: recompute (and rescale) only when a score exceeds the reference
       // by more than 2^8, so P stays within f16 range without touching O every tile
       if (named_or(1, 128, mine || fail || abort_read(abort))) {
         if (named_or(1, 128, fail || abort_read(abort))) break;
 #pragma unroll
-        for (int j = 0; j < NB; ++j) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            float v = fmaxf(x[4 * j + e], x[4 * j + 2 + e]);
-            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-            if (lane < 4) m->red[q][8 * j + 2 * lane + e] = v;
-          }
+        for (int j = 0; j < HH; ++j) {   // tile max per head over the warp's 16 tokens
+          float v = x[j];
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+          if (u == 0) m->red[q][h0 + j] = v;
         }
         {
-          float sm = fmaxf(s_a, s_b);
+          float sm = s_r;
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, o));
           if (lane == 0) m->sred[q] = sm;
@@ -1094,16 +1119,10 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         }
         named_sync(1, 128);
 #pragma unroll
-        for (int j = 0; j < NB; ++j) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) mr[2 * j + e] = m->m_ref[8 * j + hc + e];
-        }
+        for (int j = 0; j < HH; ++j) mr[j] = m->m_ref[h0 + j];
         if (pt > 0) {
 #pragma unroll
-          for (int j = 0; j < NB; ++j) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) l[2 * j + e] *= m->alpha[8 * j + hc + e];
-          }
+          for (int j = 0; j < HH; ++j) l[j] *= m->alpha[h0 + j];
           // rescale O once the previous tile's output MMAs are done
           const int tp = t - 1;
           fail = fail ||
@@ -1127,29 +1146,31 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       }
 
       // P tile (MN-major core matrices, no swizzle): K slot k, heads 8j..8j+7 at
-      // (k/8) lbo_p + 128 j + (k%8) 16; this thread's word for heads 8j + hc + {0, 1} is at
-      // + 4 (lane % 4).  lbo_p = 16 N2 + 32 puts the two core rows a warp writes in
-      // disjoint banks.
+      // (k/8) lbo_p + 128 j + (k%8) 16; a thread writes its token's HH heads as NHB 16-byte
+      // rows.  lbo_p = 16 N2 + 32 puts the eight rows of each 8-lane phase in distinct banks.
       fail = fail || !mbar_wait(&b_Pempty[sb], ((uint32_t)(t >> 1) & 1u) ^ 1u, abort, a.limit_ns);
       {
-        const float wa = s_a * inv_srun, wb = s_b * inv_srun;
-        uint8_t* pbuf = p_s + sb * P.p_bytes + 4 * (lane & 3);
-        uint8_t* pa = pbuf + (ka >> 3) * P.lbo_p + (ka & 7) * 16;
-        uint8_t* pbp = pbuf + (kb >> 3) * P.lbo_p + (kb & 7) * 16;
+        const float wr = s_r * inv_srun;
+        uint8_t* prow = p_s + sb * P.p_bytes + (kslot >> 3) * P.lbo_p + (kslot & 7) * 16 +
+                        128 * (h0 >> 3);
 #pragma unroll
-        for (int j = 0; j < NB; ++j) {
-          float ea[2], eb[2];
+        for (int b8 = 0; b8 < NHB; ++b8) {
+          float e[8];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
+          for (int k = 0; k < 8; ++k) {
+            const int j = 8 * b8 + k;
             // a head whose reference is still -inf has only -inf scores so far (any finite
             // score takes the slow path), so a finite stand-in gives 2^-inf = 0 without NaN
-            const float m0 = (mr[2 * j + e] == -INFINITY) ? 0.f : mr[2 * j + e];
-            ea[e] = ex2_approx(x[4 * j + e] - m0);
-            eb[e] = ex2_approx(x[4 * j + 2 + e] - m0);
-            l[2 * j + e] += ea[e] + eb[e];
+            const float m0 = (mr[j] == -INFINITY) ? 0.f : mr[j];
+            e[k] = ex2_approx(x[j] - m0);
+            l[j] += e[k];
           }
-          *reinterpret_cast<uint32_t*>(pa + 128 * j) = h2_bits(__floats2half2_rn(ea[0] * wa, ea[1] * wa));
-          *reinterpret_cast<uint32_t*>(pbp + 128 * j) = h2_bits(__floats2half2_rn(eb[0] * wb, eb[1] * wb));
+          uint4 o;
+          o.x = h2_bits(__floats2half2_rn(e[0] * wr, e[1] * wr));
+          o.y = h2_bits(__floats2half2_rn(e[2] * wr, e[3] * wr));
+          o.z = h2_bits(__floats2half2_rn(e[4] * wr, e[5] * wr));
+          o.w = h2_bits(__floats2half2_rn(e[6] * wr, e[7] * wr));
+          *reinterpret_cast<uint4*>(prow + 128 * b8) = o;
         }
       }
       fence_proxy_async_smem();
@@ -1162,15 +1183,13 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         fail = fail || !mbar_wait(&b_Pempty[sb], (uint32_t)(t >> 1) & 1u, abort, a.limit_ns);
         tc_fence_after();
 #pragma unroll
-        for (int j = 0; j < NB; ++j) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            float v = l[2 * j + e];
-            v += __shfl_xor_sync(0xffffffffu, v, 4);
-            v += __shfl_xor_sync(0xffffffffu, v, 8);
-            v += __shfl_xor_sync(0xffffffffu, v, 16);
-            if (lane < 4) m->red[q][8 * j + 2 * lane + e] = v;
-          }
+        for (int j = 0; j < HH; ++j) {
+          float v = l[j];
+          v += __shfl_xor_sync(0xffffffffu, v, 1);
+          v += __shfl_xor_sync(0xffffffffu, v, 2);
+          v += __shfl_xor_sync(0xffffffffu, v, 4);
+          v += __shfl_xor_sync(0xffffffffu, v, 8);
+          if (u == 0) m->red[q][h0 + j] = v;
         }
         named_sync(1, 128);
         const int64_t slot = (int64_t)blockIdx.x + c.seq;
@@ -1233,24 +1252,31 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch, int group, int sg) {
   memset(&pl, 0, sizeof(pl));
   TcParams& P = pl.p;
   const int n = d + d_rope;
-  P.N1 = (H + 7) / 8 * 8;
+  const bool in_place = (b == 16 || b == KVK_BITS_BF16);
+  // group scales are applied while the packed codes are unpacked (b < 16): 16-bit codes
+  // converted in place, and uncompressed rows, take the CUDA-core kernel in such a layout
+  if (group && in_place) return pl;
+  // exact scores from high and low parts: 16-bit codes and group-scaled caches
+  const bool stacked = (b == 16) || group;
+  P.stacked = stacked ? 1 : 0;
+  P.N1 = tc_query_rows(H);
   P.N2 = (H + 15) / 16 * 16;
   P.NP = (n + 127) / 128;
   P.NPd = (d + 127) / 128;
   P.NQA = (n + 63) / 64;
   P.NK16 = (n + 15) / 16;
-  // TMEM: S^T (N1 <= 64 columns), two C^T buffers of 4 x 32 columns, O^T NPd x N2 columns
+  // TMEM: S^T (N2 <= 64 columns), two C^T buffers of 4 x 32 columns, O^T NPd x N2 columns
   if (H < 1 || P.N2 > 64 || P.NPd > 4 || kOCol0 + (uint32_t)(P.NPd * P.N2) > kTmemCols) return pl;
-  if (P.NQA * 8 > 32 * kQC) return pl;   // staged query rows of up to 768 features
+  if (P.NQA * 8 > 16 * kQL) return pl;   // staged query rows of up to 768 features
+  if (d % 64) return pl;                  // latent query atoms copied whole by TMA
   const size_t q_bytes = (size_t)P.NQA * P.N1 * 128;
   P.lbo_p = (uint32_t)P.N2 * 16u + 32u;
   P.p_bytes = 8u * P.lbo_p;
   const size_t p_bytes = 2 * (size_t)P.p_bytes;
   const size_t misc_bytes = sizeof(Misc) + sizeof(int32_t) * (size_t)(batch + 1);
-  const bool in_place = (b == 16 || b == KVK_BITS_BF16);
-  // group scales are applied while the packed codes are unpacked (b < 16): 16-bit codes
-  // converted in place, and uncompressed rows, take the CUDA-core kernel in such a layout
-  if (group && in_place) return pl;
+  P.atom_bytes = stacked ? 2u * kAtom : (uint32_t)kAtom;
+  P.slot_bytes = 2u * P.atom_bytes;
+  P.rbs = stacked ? 2u * kLoOff : kLoOff;
   const int raw_slot = in_place ? 0 : 64 * 16 * b;
   P.raw_slot = raw_slot;
   P.grouped = group ? 1 : 0;
@@ -1259,46 +1285,52 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch, int group, int sg) {
   const size_t sc_ring = align_up((size_t)kScSlots * P.sc_bytes, 1024);
   // try the largest rings that fit
   const size_t fixed = align_up(q_bytes, 1024) + align_up(p_bytes, 1024) + sc_ring;
-  // 16-bit codes and group-scaled rows: the low parts of two groups in flight
-  const int LR = (b == 16 || group) ? 2 : 0;
-  P.LR = LR;
   auto total_for = [&](int PR, int RR) {
     size_t off = fixed;
-    off += (size_t)(PR + LR) * kPair;
+    off += (size_t)PR * P.slot_bytes;
     off = align_up(off + (size_t)RR * raw_slot, 1024);
-    off = align_up(off + (size_t)(3 * PR + 2 * RR + LR + kFixedBars) * 8, 16);
+    off = align_up(off + (size_t)(3 * PR + 2 * RR + kFixedBars) * 8, 16);
     off += misc_bytes;
     return off + 1024;   // runtime alignment slack of the dynamic shared memory base
   };
   int PR = 0, RR = 0;
   if (in_place) {
+    // the TMA lands in the f16 slots: at least a tile's groups
     for (PR = 3 * P.NP; PR >= P.NP; --PR)
       if (total_for(PR, 0) <= (size_t)kSmemLimit) break;
+    if (PR < P.NP) return pl;
   } else {
+    // packed codes land in the raw ring; the f16 slots only span conversion to score MMA, so
+    // fewer than a tile's groups still flow (a group's slot is that of the group PR earlier,
+    // released by its score MMAs, which never wait for a later group)
     const int want = P.NP + (P.NP + 1) / 2;
-    for (PR = want; PR >= P.NP; --PR) {
+    bool fit = false;
+    for (PR = want; PR >= 2 && !fit; --PR) {
       for (RR = 4 * P.NP; RR >= 2; --RR)
-        if (total_for(PR, RR) <= (size_t)kSmemLimit) break;
-      if (RR >= 2 && total_for(PR, RR) <= (size_t)kSmemLimit) break;
+        if (total_for(PR, RR) <= (size_t)kSmemLimit) {
+          fit = true;
+          break;
+        }
+      if (fit) break;
     }
+    if (!fit) return pl;
   }
-  if (PR < P.NP || (!in_place && RR < 2)) return pl;
   P.PR = PR;
   P.RR = RR;
   size_t off = fixed;
   P.off_p = (uint32_t)align_up(q_bytes, 1024);
   P.off_sc = P.off_p + (uint32_t)align_up(p_bytes, 1024);
   P.off_pairs = (uint32_t)fixed;
-  off += (size_t)PR * kPair;
-  P.off_lo = (uint32_t)off;
-  off += (size_t)LR * kPair;
+  off += (size_t)PR * P.slot_bytes;
   P.off_raw = (uint32_t)off;
   off = align_up(off + (size_t)RR * raw_slot, 1024);
   P.off_bar = (uint32_t)off;
-  off = align_up(off + (size_t)(3 * PR + 2 * RR + LR + kFixedBars) * 8, 16);
+  off = align_up(off + (size_t)(3 * PR + 2 * RR + kFixedBars) * 8, 16);
   P.off_misc = (uint32_t)off;
   pl.smem = off + misc_bytes + 1024;
-  P.idesc1 = sm100::idesc_f16(64, P.N1, false, false);
+  // score MMA: M = 64 tokens x N1 heads, or stacked M = 128 (high and low rows) x N2 heads
+  P.idesc1 = stacked ? sm100::idesc_f16(128, P.N2, false, false)
+                     : sm100::idesc_f16(64, P.N1, false, false);
   P.idesc2 = sm100::idesc_f16(128, P.N2, false, true);   // A = C^T from TMEM, B = P MN-major
   pl.ok = pl.smem <= (size_t)kSmemLimit;
   return pl;
@@ -1338,25 +1370,31 @@ bool launch_regs_ok(int b, int N2) {
   return r == (int)kLaunchRegs;
 }
 
+struct Maps {
+  const CUtensorMap& codes;
+  const CUtensorMap& ql;
+  const CUtensorMap& qr;
+};
+
 template <int BITS, int NH>
-cudaError_t launch_bits_nh(const TcParams& P, const CUtensorMap& tmap, size_t smem, int grid,
+cudaError_t launch_bits_nh(const TcParams& P, const Maps& mp, size_t smem, int grid,
                            cudaStream_t st) {
   auto k = decode_tc_kernel<BITS, NH>;
   if (instance_regs<BITS, NH>() != (int)kLaunchRegs) return cudaErrorNotSupported;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<grid, kThreads, smem, st>>>(P, tmap);
+  k<<<grid, kThreads, smem, st>>>(P, mp.codes, mp.ql, mp.qr);
   return cudaGetLastError();
 }
 
 template <int BITS>
-cudaError_t launch_bits(const TcParams& P, const CUtensorMap& tmap, size_t smem, int grid,
+cudaError_t launch_bits(const TcParams& P, const Maps& mp, size_t smem, int grid,
                         cudaStream_t st) {
   switch (P.N2) {
-    case 16: return launch_bits_nh<BITS, 16>(P, tmap, smem, grid, st);
-    case 32: return launch_bits_nh<BITS, 32>(P, tmap, smem, grid, st);
-    case 48: return launch_bits_nh<BITS, 48>(P, tmap, smem, grid, st);
-    case 64: return launch_bits_nh<BITS, 64>(P, tmap, smem, grid, st);
+    case 16: return launch_bits_nh<BITS, 16>(P, mp, smem, grid, st);
+    case 32: return launch_bits_nh<BITS, 32>(P, mp, smem, grid, st);
+    case 48: return launch_bits_nh<BITS, 48>(P, mp, smem, grid, st);
+    case 64: return launch_bits_nh<BITS, 64>(P, mp, smem, grid, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -1370,18 +1408,19 @@ bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H) {
   return pl.ok && launch_regs_ok(A.b, pl.p.N2);
 }
 
-cudaError_t launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tmap, int dtype,
-                             cudaStream_t st) {
+cudaError_t launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tmap, const CUtensorMap& qmap_l,
+                             const CUtensorMap& qmap_r, int dtype, cudaStream_t st) {
   Plan pl = make_plan(a.d, a.d_rope, a.b, a.H, a.batch, a.group, a.sg);
   if (!pl.ok) return cudaErrorInvalidValue;
   pl.p.a = a;
   pl.p.qdtype = dtype;
+  const Maps mp{tmap, qmap_l, qmap_r};
   switch (a.b) {
-    case 16: return launch_bits<16>(pl.p, tmap, pl.smem, a.G, st);
-    case KVK_BITS_BF16: return launch_bits<KVK_BITS_BF16>(pl.p, tmap, pl.smem, a.G, st);
-    case 8: return launch_bits<8>(pl.p, tmap, pl.smem, a.G, st);
-    case 4: return launch_bits<4>(pl.p, tmap, pl.smem, a.G, st);
-    case 2: return launch_bits<2>(pl.p, tmap, pl.smem, a.G, st);
+    case 16: return launch_bits<16>(pl.p, mp, pl.smem, a.G, st);
+    case KVK_BITS_BF16: return launch_bits<KVK_BITS_BF16>(pl.p, mp, pl.smem, a.G, st);
+    case 8: return launch_bits<8>(pl.p, mp, pl.smem, a.G, st);
+    case 4: return launch_bits<4>(pl.p, mp, pl.smem, a.G, st);
+    case 2: return launch_bits<2>(pl.p, mp, pl.smem, a.G, st);
   }
   return cudaErrorInvalidValue;
 }

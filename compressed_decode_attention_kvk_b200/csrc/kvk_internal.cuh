@@ -16,6 +16,8 @@ namespace kvk {
 constexpr int kMaxRowElems = 2048;      // d + d_rope handled by the write kernel
 constexpr size_t kArenaHeader = 256;    // status flags live in the first bytes of the arena
 constexpr int kTcTileTokens = 64;       // tokens per tile of the tensor-core decode
+// staged query rows of the tensor-core decode: heads rounded up to 8
+inline int tc_query_rows(int H) { return (H + 7) / 8 * 8; }
 // Work-split cost of one piece on the tensor-core decode, in tokens: query staging and the
 // pipeline refill at a sequence boundary take about as long as 2.5 tiles.
 constexpr int kTcPieceCost = 160;
@@ -139,8 +141,10 @@ cudaError_t launch_quant_append(const kvk_layout* L, const AnchorDesc& A, const 
                                 int batch, const int32_t* seq_lens, cudaStream_t stream);
 cudaError_t launch_decode_fma(const DecodeArgs& a, int dtype, cudaStream_t stream);
 // tmap: the codes plane the kernel streams (the anchor's, or a compacted keep-list copy)
-cudaError_t launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tmap, int dtype,
-                             cudaStream_t stream);
+// qmap_l / qmap_r: the query's latent and rope parts as 3D tensors [batch][H][d or d_rope] of
+// 16-bit elements, boxes of 64 features x tc_query_rows(H) heads (128-byte swizzle)
+cudaError_t launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tmap, const CUtensorMap& qmap_l,
+                             const CUtensorMap& qmap_r, int dtype, cudaStream_t st);
 bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H);
 
 inline size_t align_up_sz(size_t x, size_t a) { return (x + a - 1) / a * a; }
