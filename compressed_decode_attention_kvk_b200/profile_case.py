@@ -13,6 +13,11 @@ larger than the 126 MB L2.
 --op write times the quantise-on-write of the whole cache instead (a prefill of batch x
 tokens tokens): algorithmic bytes per call = batch * tokens * ((d + d_rope) * 2 read from
 the bf16 inputs + row_bytes + 2 written).
+
+--op absorb times the two absorbed projections of a decode step on the tensor cores
+(kvk_absorb): the query side q_lat[b, h] = q_nope[b, h] . W_UK[h] (K = --nope, n = r) and the
+output side o[b, h] = out_lat[b, h] . W_UV[h] (K = r, n = --nope), bf16 weights, fp32
+activations; algorithmic bytes = weights + activations read + outputs written.
 """
 from __future__ import annotations
 
@@ -36,7 +41,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--path", default="auto", choices=["auto", "tensor", "cuda_core"])
     ap.add_argument("--ctas", type=int, default=0)
-    ap.add_argument("--op", default="decode", choices=["decode", "write"])
+    ap.add_argument("--op", default="decode", choices=["decode", "write", "absorb"])
+    ap.add_argument("--nope", type=int, default=128, help="per-head no-RoPE width (absorb)")
     args = ap.parse_args()
 
     from . import build as kb
@@ -45,6 +51,31 @@ def main():
 
     dev = torch.device("cuda")
     B, T, H = args.batch, args.tokens, args.heads
+    if args.op == "absorb":
+        g = torch.Generator(device=dev)
+        g.manual_seed(2)
+        res = []
+        for name, K, n in (("q_side", args.nope, args.r), ("o_side", args.r, args.nope)):
+            x = torch.randn(B, H, K, generator=g, device=dev)
+            w = (torch.randn(H, K, n, generator=g, device=dev) / math.sqrt(K)).to(torch.bfloat16)
+            y = torch.empty(B, H, n, device=dev)
+            for _ in range(args.warmup):
+                kvk.kvk_absorb(x, w, y)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(args.iters):
+                kvk.kvk_absorb(x, w, y)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / args.iters
+            nbytes = H * K * n * 2 + B * H * (K + n) * 4
+            flops = 2 * B * H * K * n
+            res.append({"side": name, "K": K, "n": n, "ms_per_call": round(ms, 5),
+                        "bytes_per_call": nbytes, "GBps": round(nbytes / ms / 1e6, 1),
+                        "TFLOPs": round(flops / ms / 1e9, 3)})
+        print(json.dumps({"op": "absorb", "batch": B, "heads": H, "results": res}))
+        return
     lay = kvk.Layout([0], [args.d], [args.b], args.r, args.d_rope, B, T, device=dev)
     lay.set_decode_path({"auto": 0, "tensor": 1, "cuda_core": 2}[args.path])
     lay.set_decode_ctas(args.ctas)
