@@ -8,9 +8,38 @@
 // combines, for sequence i, the slots c + i of every CTA c whose range meets it.
 #pragma once
 
+#include <utility>
+
 #include "kvk_internal.cuh"
 
 namespace kvk {
+
+// Programmatic dependent launch.  The decode kernels and the merge are launched with
+// programmatic stream serialisation: a kernel may start while the one before it in the
+// stream finishes, and griddep_wait() returns once that kernel has completed and its memory
+// is visible (at once when it was launched the ordinary way).  griddep_trigger() lets the
+// next kernel launch before this one completes.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// cudaLaunchKernelEx with programmatic stream serialisation
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Clamped token count of sequence i without raising flags.
 __device__ __forceinline__ int seq_tokens_quiet(const DecodeArgs& a, int i, bool* bad) {

@@ -397,6 +397,13 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+  // Launched as a programmatic dependent: let the merge launch now (its blocks take SMs as
+  // this kernel's blocks exit, and it waits for this grid to complete), then wait until the
+  // kernel before this one has completed before reading any input or the workspace.  (The
+  // grid is at most one block per SM, so every block of this grid is resident.)
+  griddep_trigger();
+  griddep_wait();
+
   if (tid == 0) {
     for (int i = 0; i < P.PR; ++i) {
       mbar_init(&b_pfull[i], kTeamWarps);   // the team converting the group
@@ -1383,8 +1390,8 @@ cudaError_t launch_bits_nh(const TcParams& P, const Maps& mp, size_t smem, int g
   if (instance_regs<BITS, NH>() != (int)kLaunchRegs) return cudaErrorNotSupported;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<grid, kThreads, smem, st>>>(P, mp.codes, mp.ql, mp.qr);
-  return cudaGetLastError();
+  e = launch_pdl(k, dim3(grid), dim3(kThreads), smem, st, P, mp.codes, mp.ql, mp.qr);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int BITS>

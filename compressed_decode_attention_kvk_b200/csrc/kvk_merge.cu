@@ -41,6 +41,7 @@ __device__ __forceinline__ float block_reduce(float v, float* red) {
 __global__ void __launch_bounds__(kMergeThreads, 4) merge_kernel(DecodeArgs a) {
   __shared__ float w_s[kChunk];
   __shared__ float red[kMergeThreads / 32];
+  griddep_wait();   // the decode's partials are complete and visible
   const int i = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
   const int64_t C = a.seq_off[a.batch] + (int64_t)a.split_x * a.batch;
   const int64_t s0 = a.seq_off[i], s1 = a.seq_off[i + 1];
@@ -167,8 +168,9 @@ __global__ void __launch_bounds__(kMergeThreads, 4) merge_kernel(DecodeArgs a) {
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t st) {
   if (a.H > 65535) return cudaErrorInvalidValue;
   dim3 grid(a.batch, a.H), block(kMergeThreads);
-  merge_kernel<<<grid, block, 0, st>>>(a);
-  return cudaGetLastError();
+  // a programmatic dependent of the decode: its blocks start as the decode's finish
+  cudaError_t e = launch_pdl(merge_kernel, grid, block, 0, st, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace kvk
