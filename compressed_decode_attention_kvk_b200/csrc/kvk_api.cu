@@ -555,6 +555,13 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSuccess;
+  // Tensor-core launch over a codes plane: packed b <= 8 codes with token scales take the
+  // kernel specialised for them, everything else the general one.
+  const bool packed = kvk::tc_packed_supported(L, A, dtype, n_heads);
+  auto launch_tc = [&](const CUtensorMap& codes_map) {
+    return packed ? kvk::launch_decode_tc_packed(a, codes_map, dtype, st)
+                  : kvk::launch_decode_tc(a, codes_map, qmap_l, qmap_r, dtype, st);
+  };
   if (path == KVK_PATH_TENSOR && keep) {
     kvk::CompactArgs c;
     memset(&c, 0, sizeof(c));
@@ -578,7 +585,7 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
     a.keep_idx = nullptr;
     a.keep_len = nullptr;
     a.keep_stride = 0;
-    if (e == cudaSuccess) e = kvk::launch_decode_tc(a, keep_tmap, qmap_l, qmap_r, dtype, st);
+    if (e == cudaSuccess) e = launch_tc(keep_tmap);
   } else if (path == KVK_PATH_TENSOR) {
     if (app) {   // the decode kernel writes the new tokens itself
       a.app_c = app->c;
@@ -587,7 +594,7 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
       a.app_kr_ss = app->kr_ss;
       a.app_dtype = app->dtype;
     }
-    e = kvk::launch_decode_tc(a, A.tmap_tile, qmap_l, qmap_r, dtype, st);
+    e = launch_tc(A.tmap_tile);
   } else {
     if (app)
       e = kvk::launch_quant_append(L, A, app->c, app->dtype, app->c_ss, app->kr, app->kr_ss,

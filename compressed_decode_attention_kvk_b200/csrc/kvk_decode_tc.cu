@@ -398,11 +398,12 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // Launched as a programmatic dependent: let the merge launch now (its blocks take SMs as
-  // this kernel's blocks exit, and it waits for this grid to complete), then wait until the
-  // kernel before this one has completed before reading any input or the workspace.  (The
-  // grid is at most one block per SM, so every block of this grid is resident.)
+  // this kernel's blocks exit, and it waits for this grid to complete).  (The grid is at most
+  // one block per SM, so every block of this grid is resident.)  The set-up below touches only
+  // this block's shared memory, TMEM and the kernel parameters, so it may overlap the kernel
+  // before this one; the wait before the first global access (block_seq_offsets) holds every
+  // read of an input or of the workspace until that kernel has completed.
   griddep_trigger();
-  griddep_wait();
 
   if (tid == 0) {
     for (int i = 0; i < P.PR; ++i) {
@@ -448,6 +449,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     tma_prefetch_desc(&qmap_l);
     if (a.d_rope > 0) tma_prefetch_desc(&qmap_r);
   }
+  griddep_wait();
   block_seq_offsets(a, off, m->scan_tmp);   // contains __syncthreads
   if (blockIdx.x == 0)
     for (int i = tid; i <= a.batch; i += kThreads) a.seq_off[i] = off[i];

@@ -41,6 +41,10 @@ __device__ __forceinline__ float block_reduce(float v, float* red) {
 __global__ void __launch_bounds__(kMergeThreads, 4) merge_kernel(DecodeArgs a) {
   __shared__ float w_s[kChunk];
   __shared__ float red[kMergeThreads / 32];
+  // Let the next kernel in the stream (the next layer's decode) launch once every block of
+  // this grid has started: its blocks then set up on the SMs this grid leaves and wait for
+  // this grid to complete before they read or write anything it uses.
+  griddep_trigger();
   griddep_wait();   // the decode's partials are complete and visible
   const int i = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
   const int64_t C = a.seq_off[a.batch] + (int64_t)a.split_x * a.batch;
