@@ -12,10 +12,11 @@
 // 64 tokens.  Warp roles (512 threads, four warpgroups with their own register budgets):
 //   warps 0-3  softmax: read S from TMEM, per-token scale, lazy online softmax, write P
 //              (f16) to shared memory, rescale O in TMEM when a max grows, write partials
-//   warps 4-11 convert: packed b-bit codes -> f16 operand tiles (UMMA 128-byte-swizzled,
-//              K-major) and their transpose into TMEM.  Two teams of four warps take
-//              alternate 128-feature groups; in a group, warp w owns 32 features (its TMEM
-//              lane quarter of C^T).
+//   warps 4-11 convert: 16-bit rows or packed b-bit codes -> f16 operand tiles (UMMA
+//              128-byte-swizzled, K-major) and their transpose into TMEM.  16-bit rows: all
+//              eight warps on every 128-feature group, 16 features each; packed
+//              (group-scaled) codes: two teams of four warps on alternate groups, 32 features
+//              each.  A warp's features are in its TMEM lane quarter of C^T.
 //   warp 12    TMA producer: 128-feature groups of 64 packed rows into a ring, and each
 //              tile's scales; the stream is read once, so it carries an evict-first L2 policy
 //   warp 13    score-MMA issuer (one thread) and TMEM owner
@@ -407,7 +408,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
 
   if (tid == 0) {
     for (int i = 0; i < P.PR; ++i) {
-      mbar_init(&b_pfull[i], kTeamWarps);   // the team converting the group
+      // every convert warp (16-bit rows), or the team converting the group (packed codes)
+      mbar_init(&b_pfull[i], kInPlace<BITS> ? kConvWarps : kTeamWarps);
       // score MMAs (commit), plus the convert warps where they read the slot after q_full
       mbar_init(&b_pempty[i], kInPlace<BITS> ? 1 : 1 + kTeamWarps);
       mbar_init(&b_tfull[i], 1);
@@ -714,9 +716,11 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   } else if (has_work && warp >= kConvWarp0) {
     regs_set<kRegsConvert>();
     // ------------------------------------------------------------------ convert
-    // Two teams of four warps take alternate groups (team cw / 4 converts the CTA's groups with
-    // the team's parity), so two groups are in flight; in its team's groups warp cw owns the 32
-    // features 32 cq .. 32 cq + 31 (cq = cw % 4), which are its own TMEM lane quarter of C^T.
+    // 16-bit rows: every warp converts every group, warp cw the 16 features 32 cq + 16 (cw / 4)
+    // .. + 15 (cq = cw % 4).  Packed codes: two teams of four warps take alternate groups (team
+    // cw / 4 converts the CTA's groups with the team's parity), so two groups are in flight; in
+    // its team's groups warp cw owns the 32 features 32 cq .. 32 cq + 31.  Either way a warp's
+    // features are in its own TMEM lane quarter of C^T.
     // The warps share no barrier among themselves (every hand-off is an mbarrier), so a warp
     // that stops on a failed wait leaves its loop alone; it then arrives on nothing more, and
     // everything downstream of the group it stopped at waits until it sees the abort word.
@@ -761,15 +765,22 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           for (int i = 0; i < 4; ++i) x[16 * h + 4 * tg + i] = d4[i];
         }
     };
-    auto stsm32 = [&](uint32_t base, const uint32_t (&x)[32]) {
+    // the same for 16 features (one half's offsets; register 4 tg + i: 16-token block tg)
+    auto ldsm16 = [&](uint32_t base, const uint32_t (&off)[4], uint32_t (&x)[16]) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
+      for (int tg = 0; tg < 4; ++tg) {
+        uint32_t d4[4];
+        ldsm_x4_trans(base + off[tg], d4);
 #pragma unroll
-        for (int tg = 0; tg < 4; ++tg) {
-          const uint32_t d4[4] = {x[16 * h + 4 * tg], x[16 * h + 4 * tg + 1],
-                                  x[16 * h + 4 * tg + 2], x[16 * h + 4 * tg + 3]};
-          stsm_x4_trans(base + aoff[h][tg], d4);
-        }
+        for (int i = 0; i < 4; ++i) x[4 * tg + i] = d4[i];
+      }
+    };
+    auto stsm16 = [&](uint32_t base, const uint32_t (&off)[4], const uint32_t (&x)[16]) {
+#pragma unroll
+      for (int tg = 0; tg < 4; ++tg) {
+        const uint32_t d4[4] = {x[4 * tg], x[4 * tg + 1], x[4 * tg + 2], x[4 * tg + 3]};
+        stsm_x4_trans(base + off[tg], d4);
+      }
     };
     // this warp's C^T: TMEM lanes 32 cq .. 32 cq + 31, columns of latent group p
     auto tmem_st32 = [&](uint32_t col, const uint32_t (&x)[32]) {
@@ -850,50 +861,60 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         ct_waited = true;
       };
       if constexpr (kInPlace<BITS>) {
-        // In place, 16-bit codes (or bf16 values) -> f16, in one pass through registers: each
-        // 8x8 block (8 tokens x 8 features) is loaded transposed, converted element by
-        // element, stored back transposed (row-major again, for the score MMAs; 16-bit codes
-        // as exact high and low parts in the stacked slot) and the same registers, now
-        // feature-major, go to C^T in TMEM.  The slot is not read after p_full, so only the
-        // score MMAs release it.
+        // In place, 16-bit codes (or bf16 values) -> f16, in one pass through registers, by all
+        // eight convert warps on every group: warp cw takes the 16 features of half hf = cw / 4
+        // of its lane quarter's 32 (a group's conversion then takes half as long as with one
+        // team of four).  Each 8x8 block (8 tokens x 8 features) is loaded transposed, converted
+        // element by element, stored back transposed (row-major again, for the score MMAs;
+        // 16-bit codes as exact high and low parts in the stacked slot) and the same registers,
+        // now feature-major, go to C^T in TMEM (lanes 32 cq + 16 hf ..).  The relocation from
+        // where TMA put the rows stays inside the warp's own 16-byte columns, all of which it
+        // reads before it writes any.  The slot is not read after p_full, so only the score MMAs
+        // release it.
+        const int hf = team;
+        uint32_t ao[4], ro[4];   // this warp's half of aoff / roff
+#pragma unroll
+        for (int tg = 0; tg < 4; ++tg) {
+          ao[tg] = hf ? aoff[1][tg] : aoff[0][tg];
+          ro[tg] = hf ? roff[1][tg] : roff[0][tg];
+        }
         for (int p = 0; p < P.NP; ++p) {
-          if (((p + gbase) & 1) == team) {
-            const uint32_t s = pr.slot;
-            fail = fail || !wait_warp(&b_tfull[s], pr.phase, abort, a.limit_ns);
-            const bool go = !fail && owns_group(p);
-            const uint32_t sbase = pairs_u + s * P.slot_bytes;
-            uint32_t x[32], xl[32];
-            if (go) {
-              ldsm32(sbase, roff, x);
-              if constexpr (BITS == 16) {
+          const uint32_t s = pr.slot;
+          fail = fail || !wait_warp(&b_tfull[s], pr.phase, abort, a.limit_ns);
+          const bool go = !fail && owns_group(p);
+          const uint32_t sbase = pairs_u + s * P.slot_bytes;
+          uint32_t x[16], xl[16];
+          if (go) {
+            ldsm16(sbase, ro, x);
+            if constexpr (BITS == 16) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) cvt_code16_split(x[i], x[i], xl[i]);
-              } else {
+              for (int i = 0; i < 16; ++i) cvt_code16_split(x[i], x[i], xl[i]);
+            } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = cvt_bf16x2(x[i]);
-                if (c.cnt < kTile) {
-                  // rows past the piece's end hold whatever the cache or scratch holds there
-                  // (as bf16 possibly a NaN, and P = 0 times NaN is NaN): zero them.  Register
-                  // 16h + 4tg + i holds tokens 16tg + 8(i%2) + 2(lane%4) + {0, 1}.
+              for (int i = 0; i < 16; ++i) x[i] = cvt_bf16x2(x[i]);
+              if (c.cnt < kTile) {
+                // rows past the piece's end hold whatever the cache or scratch holds there
+                // (as bf16 possibly a NaN, and P = 0 times NaN is NaN): zero them.  Register
+                // 4tg + i holds tokens 16tg + 8(i%2) + 2(lane%4) + {0, 1}.
 #pragma unroll
-                  for (int i = 0; i < 32; ++i) {
-                    const int t0 = 16 * ((i >> 2) & 3) + 8 * (i & 1) + 2 * (lane & 3);
-                    x[i] &= (t0 < c.cnt ? 0x0000FFFFu : 0u) | (t0 + 1 < c.cnt ? 0xFFFF0000u : 0u);
-                  }
+                for (int i = 0; i < 16; ++i) {
+                  const int t0 = 16 * (i >> 2) + 8 * (i & 1) + 2 * (lane & 3);
+                  x[i] &= (t0 < c.cnt ? 0x0000FFFFu : 0u) | (t0 + 1 < c.cnt ? 0xFFFF0000u : 0u);
                 }
               }
             }
-            if (go && !fail) {
-              stsm32(sbase, x);
-              if constexpr (BITS == 16) stsm32(sbase + kLoOff, xl);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0 && !fail) mbar_arrive(&b_pfull[s]);
-            if (p < P.NPd) {
-              if (!ct_waited) wait_ct();
-              if (go && !fail) tmem_st32(ct_col + 32u * p, x);
-            }
+          }
+          if (go && !fail) {
+            stsm16(sbase, ao, x);
+            if constexpr (BITS == 16) stsm16(sbase + kLoOff, ao, xl);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && !fail) mbar_arrive(&b_pfull[s]);
+          if (p < P.NPd) {
+            if (!ct_waited) wait_ct();
+            if (go && !fail)
+              tmem_st16x256b_x4(tmem + ((uint32_t)(32 * cq + 16 * hf) << 16) + ct_col + 32u * p, x);
           }
           pr.next(P.PR);
         }
