@@ -555,8 +555,8 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSuccess;
-  // Tensor-core launch over a codes plane: packed b <= 8 codes with token scales take the
-  // kernel specialised for them, everything else the general one.
+  // Tensor-core launch over a codes plane: codes with one scale per token take the kernel
+  // specialised for them, bf16 rows and group-scaled codes the general one.
   const bool packed = kvk::tc_packed_supported(L, A, dtype, n_heads);
   auto launch_tc = [&](const CUtensorMap& codes_map) {
     return packed ? kvk::launch_decode_tc_packed(a, codes_map, dtype, st)

@@ -1,5 +1,5 @@
-// kvk_decode_tc_packed.cu -- tensor-core (tcgen05) split decode over packed b-bit codes
-// (b in {2, 4, 8}, one fp16 scale per token): the plain decode of such layers.
+// kvk_decode_tc_packed.cu -- tensor-core (tcgen05) split decode over b-bit codes with one
+// fp16 scale per token (b in {2, 4, 8, 16}): the decode, and the fused append, of such layers.
 //
 // Computes the same partials as the CUDA-core kernel (kvk_decode_fma.cu) and the general
 // tensor-core kernel (kvk_decode_tc.cu): for every piece of a sequence that the CTA owns, the
@@ -9,23 +9,26 @@
 // attention over the dequantised cache; KV-Kaizen "Background": each decode step reads the
 // whole cache).
 //
-// Codes of at most 8 bits are exact in f16, so the scores need no high/low split and the
-// score MMA is M = 64.  This kernel keeps the conversion of every 128-feature group spread
-// over all eight convert warps (16 features each), which halves a group's conversion latency
-// against the general kernel's two alternating teams; measured on B200 at 32 x 8192 tokens,
-// 40 heads, d = 512, one layer takes 112 us at b = 8 here against 146 us in the general
-// kernel.  The general kernel keeps what this one lacks: 16-bit and bf16 rows and group
-// scales.
+// Scores are exact: codes of at most 8 bits are exact in f16 (score MMA M = 64); a 16-bit code
+// c is split into hi = f16(c) and lo = c - hi, both exact, stacked per 16-token block into one
+// M = 128 score MMA whose low-part rows land 16 TMEM lanes below the high-part rows (the
+// softmax adds the two).  The conversion of every 128-feature group is spread over all eight
+// convert warps (16 features each), and the softmax reads S with the 16x256b shape, two tokens
+// per thread; measured on B200 at 32 x 8192 tokens, 40 heads, d = 512, this kernel is faster
+// than the general one (kvk_decode_tc.cu) for every width it covers.  The general kernel keeps
+// what this one lacks: bf16 rows and group scales.
 //
 // One persistent CTA per SM walks its slice of the flattened token space (the split charges
 // each piece a fixed cost, so a CTA that starts a sequence takes fewer tokens) in tiles of
 // 64 tokens.  Warp roles (512 threads, four warpgroups with their own register budgets):
 //   warps 0-3  softmax: read S from TMEM, per-token scale, lazy online softmax, write P
 //              (f16) to shared memory, rescale O in TMEM when a max grows, write partials
-//   warps 4-11 convert: packed b-bit codes -> f16 operand tiles (UMMA 128-byte-swizzled,
-//              K-major) and their transpose into TMEM; staged query (power-of-two scaled).
+//   warps 4-11 convert: b-bit codes -> f16 operand tiles (UMMA 128-byte-swizzled, K-major;
+//              16-bit codes as stacked high and low parts) and their transpose into TMEM;
+//              staged query (power-of-two scaled).
 //              Two warps per SM sub-partition, 16 features of every 128-feature group each.
-//   warp 12    TMA producer: 128-feature groups of 64 packed rows into a ring, and each
+//   warp 12    TMA producer: 128-feature groups of 64 rows into a ring (16-bit rows straight
+//              into the group slots, narrower codes into a raw ring), and each
 //              tile's token scales; the stream is read once, so it carries an evict-first
 //              L2 policy
 //   warp 13    score-MMA issuer (one thread) and TMEM owner
@@ -35,13 +38,15 @@
 // Launched with 128 registers per thread; the softmax warpgroup raises its budget to
 // kRegsSoftmax, the conversion warpgroups lower theirs to kRegsConvert and the last
 // warpgroup to kRegsIssue (4 x 32 x (192 + 2 x 120 + 80) = 65536).
-// Per tile:  S^T[64 tok x N1 heads]  = C[64 x n] . Q^T         (M=64, A in smem, TMEM f32)
+// Per tile:  S^T[64 tok x N1 heads]  = C[64 x n] . Q^T   (M=64, or M=128 stacked x N2; A in
+//                                                          smem, TMEM f32)
 //            O^T[128 feat x N2 heads] += C^T[128 x 64] . P    (M=128 per 128 latent features,
 //                                                               A = C^T in TMEM)
 // Heads sit on N, so 40 heads cost N = 40 / 48, never M = 128.  The convert warps unpack each
 // 128-feature group from a raw ring into an f16 slot (UMMA 128-byte swizzled, K-major: the
-// score MMA's A) and put their 16 features of it, transposed with ldmatrix.trans, into TMEM
-// (tcgen05.st); the output MMA reads C^T from TMEM.
+// score MMA's A), or split 16-bit rows in place, and put their 16 features of it, transposed
+// with ldmatrix.trans, into TMEM (tcgen05.st); the output MMA reads C^T from TMEM (for 16-bit
+// codes the high parts: f16(code), relative 2^-12 on the output, inside its tolerance).
 // The transpose fragment orders the 16 tokens of each K step as 0,1,8,9,2,3,10,11,4,5,12,13,
 // 6,7,14,15; the softmax warps write P's K rows in that same order.
 // The per-token scale s_t multiplies the S row and is folded into P as p * s_t / S_run, with
@@ -82,6 +87,17 @@ __device__ __forceinline__ void regs_set() {
 constexpr int kTile = kTcTileTokens;   // 64
 constexpr int kAtom = 8192;            // 64 rows x 128 bytes (64 f16 features)
 constexpr int kPair = 2 * kAtom;       // 128 features
+// Group slot geometry.  Plain slots (b <= 8) hold each 64-feature atom's 64 f16 rows
+// contiguously.  16-bit codes use stacked slots: per 16-token block, the 16 rows of exact high
+// parts and then the 16 rows of low parts of the same tokens (4 KB blocks, low rows at +
+// kLoOff), so that one M = 128 score MMA yields both partial scores of 64 tokens.
+template <int BITS>
+constexpr bool kStacked = (BITS == 16);
+template <int BITS>
+constexpr uint32_t kAtomB = kStacked<BITS> ? 2u * kAtom : (uint32_t)kAtom;
+template <int BITS>
+constexpr uint32_t kSlotB = 2u * kAtomB<BITS>;
+constexpr uint32_t kLoOff = 2048;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol = 0;          // scores S^T, one buffer (N1 <= 64 columns)
 constexpr uint32_t kCtCol0 = 64;       // C^T double buffer: 64 + 128 b, latent group p at + 32 p
@@ -199,6 +215,19 @@ __device__ __forceinline__ bool wait_warp(uint64_t* b, uint32_t parity, uint32_t
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
+// Two 16-bit offset-binary codes, each split exactly into two f16 parts, hi = f16(code)
+// (rounded to nearest) and lo = code - hi: with hb, lb the code's bytes (exact in f16),
+// t = (hb - 128) * 256 - hi is an integer of magnitude <= 263 (so the fused multiply-add is
+// exact), and lo = t + lb an integer of magnitude <= 8 (f16 spacing is at most 16 below 2^15):
+// q . code = q . hi + q . lo exactly.
+__device__ __forceinline__ void cvt_code16_split(uint32_t w, uint32_t& hi, uint32_t& lo) {
+  const __half2 hs = __hsub2(bits_h2(__byte_perm(w, 0x64u, 0x4341u)), __float2half2_rn(1152.f));
+  const __half2 ls = __hsub2(bits_h2(__byte_perm(w, 0x64u, 0x4240u)), __float2half2_rn(1024.f));
+  const __half2 h = __hfma2(hs, __float2half2_rn(256.f), ls);
+  const __half2 t = __hfma2(hs, __float2half2_rn(256.f), __hneg2(h));
+  hi = h2_bits(h);
+  lo = h2_bits(__hadd2(t, ls));
+}
 // bytes of w selected by `sel` (each a field u < 1024) -> f16x2 of (u - bias), exact
 __device__ __forceinline__ uint32_t cvt_small(uint32_t w, uint32_t sel, __half2 bias) {
   return h2_bits(__hsub2(bits_h2(__byte_perm(w, 0x64u, sel)), bias));
@@ -303,7 +332,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.off_bar);
   uint64_t* b_pfull = bars;               // [PR] group converted, visible to the tensor core
   uint64_t* b_pempty = b_pfull + P.PR;    // [PR] group released by the MMAs
-  uint64_t* b_rfull = b_pempty + P.PR;    // [RR] packed group landed
+  uint64_t* b_tfull = b_pempty + P.PR;    // [PR] 16-bit: TMA landed in the group slot
+  uint64_t* b_rfull = b_tfull + P.PR;     // [RR] packed group landed
   uint64_t* b_rempty = b_rfull + P.RR;    // [RR] packed group consumed
   uint64_t* b_sfull = b_rempty + P.RR;    // scores ready in TMEM
   uint64_t* b_sempty = b_sfull + 1;       // scores read
@@ -337,8 +367,9 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
   if (tid == 0) {
     for (int i = 0; i < P.PR; ++i) {
       mbar_init(&b_pfull[i], kConvWarps);
-      // score MMAs (commit), plus the convert warps once they have read the slot back
-      mbar_init(&b_pempty[i], 1 + kConvWarps);
+      // score MMAs (commit), plus the convert warps where they read the slot back (b <= 8)
+      mbar_init(&b_pempty[i], kStacked<BITS> ? 1 : 1 + kConvWarps);
+      mbar_init(&b_tfull[i], 1);
     }
     for (int i = 0; i < P.RR; ++i) {
       mbar_init(&b_rfull[i], 1);
@@ -405,7 +436,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         cursor_start(c, seq0, off, a.batch, lo, hi);
         uint32_t cnt = 0;
         Ring rg;
-        const int slots = P.RR;
+        const int slots = kStacked<BITS> ? P.PR : P.RR;
         // hold the first cache loads until the first query is staged: its loads then do not
         // queue behind every CTA's ring fill
         mbar_wait(b_qfull, 0u, abort, a.limit_ns);
@@ -428,9 +459,22 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           }
           for (int p = 0; p < P.NP && ok; ++p) {
             const uint32_t s = rg.slot, ph = rg.phase;
-            if (!(ok = mbar_wait(&b_rempty[s], ph ^ 1u, abort, a.limit_ns))) break;
-            mbar_arrive_expect_tx(&b_rfull[s], P.raw_slot);
-            tma_load_2d_hint(raw + s * P.raw_slot, &tmap, p * 16 * BITS, row0, &b_rfull[s], pol);
+            if constexpr (kStacked<BITS>) {
+              // 16-bit rows land in the group slot itself: each atom's 64 rows contiguously at
+              // the start of the atom's place (the convert warps move them into the stacked
+              // layout); the slot is re-armed once the score MMAs have read it
+              if (!(ok = mbar_wait(&b_pempty[s], ph ^ 1u, abort, a.limit_ns))) break;
+              const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
+              mbar_arrive_expect_tx(&b_tfull[s], nat * kAtom);
+              for (int t = 0; t < nat; ++t)
+                tma_load_2d_hint(pairs + s * kSlotB<BITS> + t * kAtomB<BITS>, &tmap,
+                                 (2 * p + t) * 128, row0, &b_tfull[s], pol);
+            } else {
+              if (!(ok = mbar_wait(&b_rempty[s], ph ^ 1u, abort, a.limit_ns))) break;
+              mbar_arrive_expect_tx(&b_rfull[s], P.raw_slot);
+              tma_load_2d_hint(raw + s * P.raw_slot, &tmap, p * 16 * BITS, row0, &b_rfull[s],
+                               pol);
+            }
             ++cnt;
             rg.next(slots);
           }
@@ -445,7 +489,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         const uint32_t first = cnt > (uint32_t)slots ? cnt - slots : 0u;
         for (uint32_t k = first; k < cnt; ++k) {
           const uint32_t s = k % slots, ph = (k / slots) & 1u;
-          wait_noabort(&b_rfull[s], ph);
+          wait_noabort(kStacked<BITS> ? &b_tfull[s] : &b_rfull[s], ph);
         }
       }
     } else if (warp == kMmaWarp) {
@@ -473,7 +517,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           for (int t = 0; t < 2; ++t) {
             const int atom = 2 * p + t;
             if (atom * 64 >= a.n) break;
-            const uint64_t ad = a0 + ((s * kPair + t * kAtom) >> 4);
+            const uint64_t ad = a0 + ((s * kSlotB<BITS> + t * kAtomB<BITS>) >> 4);
             const uint64_t bd = b0 + ((atom * q_atom) >> 4);
             const int k0 = atom * 4;
             if (k0 + 4 <= P.NK16) {
@@ -585,6 +629,23 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     // fb = 32 cq + 16 ch (ch = cw / 4): TMEM lanes fb .. fb+15 of C^T.
     const int cw = warp - kConvWarp0;
     const int cq = cw & 3, ch = cw >> 2, fb = 32 * cq + 16 * ch;
+    // 16-bit codes: this lane's ldmatrix row address inside a stacked group slot, per 16-token
+    // block tg (token 16tg + 8((lane/8)%2) + lane%8, 16-byte chunk 4(cq%2) + 2ch + (lane/8)/2
+    // of atom cq/2), where TMA put the row (roff: the atom's 64 rows contiguous from the
+    // atom's start) and in the stacked layout (aoff; low part at + kLoOff).  Both keep the
+    // 128-byte swizzle phase (token % 8), so a warp's cells stay in its own 16-byte columns:
+    // it reads all of them (ldmatrix) before it writes any, and no other warp touches them.
+    uint32_t roff[4] = {}, aoff[4] = {};
+    if constexpr (kStacked<BITS>) {
+      const int mi = lane >> 3, r8 = lane & 7;
+      const uint32_t col = (uint32_t)(((4 * (cq & 1) + 2 * ch + (mi >> 1)) ^ r8) << 4);
+#pragma unroll
+      for (int tg = 0; tg < 4; ++tg) {
+        const uint32_t tok = (uint32_t)(16 * tg + 8 * (mi & 1) + r8);
+        roff[tg] = (uint32_t)(cq >> 1) * kAtomB<BITS> + tok * 128u + col;
+        aoff[tg] = (uint32_t)(cq >> 1) * kAtomB<BITS> + (tok >> 4) * 4096u + (tok & 15u) * 128u + col;
+      }
+    }
     Ring pr, rr;   // f16 group ring, packed group ring
     int last_piece = -1;
     bool fail = false;
@@ -671,12 +732,53 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       const int ctb = c.tile & 1;   // C^T buffer of this tile
       for (int p = 0; p < P.NP; ++p) {
         const uint32_t s = pr.slot, ph = pr.phase;
-        uint8_t* pair = pairs + s * kPair;
+        uint8_t* pair = pairs + s * kSlotB<BITS>;
         const int nat = ((2 * p + 1) * 64 < a.n) ? 2 : 1;
         // this warp owns features fb .. fb+15 of the group: atom cq/2, chunks
         // 4(cq%2) + 2ch + {0, 1} of every token row; it converts them and later transposes them
         const bool owns = (cq >> 1) < nat;
-        {
+        if constexpr (kStacked<BITS>) {
+          // In place, 16-bit codes -> exact f16 high and low parts, in one pass through
+          // registers: each 8x8 block (8 tokens x 8 features) is loaded transposed from where
+          // TMA put it, split element by element, stored back transposed into the stacked
+          // layout (high parts, and low parts kLoOff further), and the high parts, now
+          // feature-major, go to C^T in TMEM (lanes fb .. fb+15 of latent group p).  The slot is
+          // not read after p_full, so only the score MMAs release it.
+          fail = fail || !wait_warp(&b_tfull[s], ph, abort, a.limit_ns);
+          const bool go = !fail && owns;
+          const uint32_t sbase = smem_u32(pair);
+          uint32_t x[16], xl[16];
+          if (go) {
+#pragma unroll
+            for (int tg = 0; tg < 4; ++tg) {
+              uint32_t d4[4];
+              ldsm_x4_trans(sbase + roff[tg], d4);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) x[4 * tg + i] = d4[i];
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) cvt_code16_split(x[i], x[i], xl[i]);
+#pragma unroll
+            for (int tg = 0; tg < 4; ++tg) {
+              const uint32_t h4[4] = {x[4 * tg], x[4 * tg + 1], x[4 * tg + 2], x[4 * tg + 3]};
+              const uint32_t l4[4] = {xl[4 * tg], xl[4 * tg + 1], xl[4 * tg + 2], xl[4 * tg + 3]};
+              stsm_x4_trans(sbase + aoff[tg], h4);
+              stsm_x4_trans(sbase + kLoOff + aoff[tg], l4);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b_pfull[s]);
+          if (p < P.NPd) {
+            if (p == 0) {   // the output MMAs of tile - 2 have finished reading this buffer
+              fail = fail || !wait_warp(&b_ctempty[ctb], ((uint32_t)(c.tile >> 1) & 1u) ^ 1u,
+                                        abort, a.limit_ns);
+              tc_fence_after();
+            }
+            if (go && !fail)
+              tmem_st16x256b_x4(tmem + ((uint32_t)fb << 16) + kCtCol0 + 128u * ctb + 32u * p, x);
+          }
+        } else {
           const uint32_t rs = rr.slot, rph = rr.phase;
           fail = fail || !wait_warp(&b_rfull[rs], rph, abort, a.limit_ns);
           fail = fail || !wait_warp(&b_pempty[s], ph ^ 1u, abort, a.limit_ns);
@@ -788,30 +890,28 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
       const float ca = coef0 * s_a, cbf = coef0 * s_b;
       fail = fail || !wait_warp(b_sfull, (uint32_t)t & 1u, abort, a.limit_ns);
       tc_fence_after();
+      // S^T rows of this thread (16x256b shape over 16 lanes from `at`); with stacked 16-bit
+      // codes the low-part scores of the same tokens sit 16 lanes further and are added
+      auto load_s = [&](uint32_t at, float (&x)[4 * NB]) {
+        if constexpr (NB == 8) {
+          tmem_ld16x256b_x8(at, *reinterpret_cast<float(*)[32]>(x));
+        } else if constexpr (NB == 6) {   // columns 0-31 and 32-47
+          tmem_ld16x256b_x4(at, *reinterpret_cast<float(*)[16]>(x));
+          tmem_ld16x256b_x2(at + 32u, *reinterpret_cast<float(*)[8]>(x + 16));
+        } else if constexpr (NB == 4) {
+          tmem_ld16x256b_x4(at, *reinterpret_cast<float(*)[16]>(x));
+        } else {
+          tmem_ld16x256b_x2(at, *reinterpret_cast<float(*)[8]>(x));
+        }
+      };
       float x[4 * NB];
-      if constexpr (NB == 8) {
-        float v[32];
-        tmem_ld16x256b_x8(lb + kSCol, v);
+      load_s(lb + kSCol, x);
+      if constexpr (kStacked<BITS>) {
+        float xlo[4 * NB];
+        load_s(lb + (16u << 16) + kSCol, xlo);
+        tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = v[i];
-      } else if constexpr (NB == 6) {   // columns 0-31 and 32-47
-        float v[16], w[8];
-        tmem_ld16x256b_x4(lb + kSCol, v);
-        tmem_ld16x256b_x2(lb + kSCol + 32u, w);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = v[i];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[16 + i] = w[i];
-      } else if constexpr (NB == 4) {
-        float v[16];
-        tmem_ld16x256b_x4(lb + kSCol, v);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = v[i];
-      } else {
-        float v[8];
-        tmem_ld16x256b_x2(lb + kSCol, v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = v[i];
+        for (int i = 0; i < 4 * NB; ++i) x[i] += xlo[i];
       }
       tmem_wait_ld();
       tc_fence_before();
@@ -1010,7 +1110,8 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
   Plan pl;
   memset(&pl, 0, sizeof(pl));
   TcParams& P = pl.p;
-  if (b != 2 && b != 4 && b != 8) return pl;
+  if (b != 2 && b != 4 && b != 8 && b != 16) return pl;
+  const bool stacked = (b == 16);
   const int n = d + d_rope;
   P.N1 = (H + 7) / 8 * 8;
   P.N2 = (H + 15) / 16 * 16;
@@ -1026,40 +1127,52 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
   P.p_bytes = 8u * P.lbo_p;
   const size_t p_bytes = 2 * (size_t)P.p_bytes;
   const size_t misc_bytes = sizeof(Misc) + sizeof(int32_t) * (size_t)(batch + 1);
-  const int raw_slot = 64 * 16 * b;
+  const int raw_slot = stacked ? 0 : 64 * 16 * b;   // 16-bit rows land in the slots
+  const size_t slot_bytes = stacked ? 4u * kAtom : (size_t)kPair;
   P.raw_slot = raw_slot;
   // try the largest rings that fit
   const size_t fixed = align_up(q_bytes, 1024) + align_up(p_bytes, 1024);
   auto total_for = [&](int PR, int RR) {
     size_t off = fixed;
-    off += (size_t)PR * kPair;
+    off += (size_t)PR * slot_bytes;
     off = align_up(off + (size_t)RR * raw_slot, 1024);
-    off = align_up(off + (size_t)(2 * PR + 2 * RR + kFixedBars) * 8, 16);
+    off = align_up(off + (size_t)(3 * PR + 2 * RR + kFixedBars) * 8, 16);
     off += misc_bytes;
     return off + 1024;   // runtime alignment slack of the dynamic shared memory base
   };
-  // f16 slots for one and a half tiles of groups, and the largest raw ring that then fits
   int PR = 0, RR = 0;
-  const int want = P.NP + (P.NP + 1) / 2;
-  for (PR = want; PR >= P.NP; --PR) {
-    for (RR = 4 * P.NP; RR >= 2; --RR)
-      if (total_for(PR, RR) <= (size_t)kSmemLimit) break;
-    if (RR >= 2 && total_for(PR, RR) <= (size_t)kSmemLimit) break;
+  if (stacked) {
+    // TMA lands in the slots: at least a tile's groups
+    for (PR = 3 * P.NP; PR >= P.NP; --PR)
+      if (total_for(PR, 0) <= (size_t)kSmemLimit) break;
+    if (PR < P.NP) return pl;
+  } else {
+    // f16 slots for one and a half tiles of groups, and the largest raw ring that then fits
+    const int want = P.NP + (P.NP + 1) / 2;
+    for (PR = want; PR >= P.NP; --PR) {
+      for (RR = 4 * P.NP; RR >= 2; --RR)
+        if (total_for(PR, RR) <= (size_t)kSmemLimit) break;
+      if (RR >= 2 && total_for(PR, RR) <= (size_t)kSmemLimit) break;
+    }
+    if (PR < P.NP || RR < 2) return pl;
   }
-  if (PR < P.NP || RR < 2) return pl;
   P.PR = PR;
   P.RR = RR;
   size_t off = fixed;
   P.off_p = (uint32_t)align_up(q_bytes, 1024);
   P.off_pairs = (uint32_t)fixed;
-  off += (size_t)PR * kPair;
+  off += (size_t)PR * slot_bytes;
   P.off_raw = (uint32_t)off;
   off = align_up(off + (size_t)RR * raw_slot, 1024);
   P.off_bar = (uint32_t)off;
-  off = align_up(off + (size_t)(2 * PR + 2 * RR + kFixedBars) * 8, 16);
+  off = align_up(off + (size_t)(3 * PR + 2 * RR + kFixedBars) * 8, 16);
   P.off_misc = (uint32_t)off;
   pl.smem = off + misc_bytes + 1024;
-  P.idesc1 = sm100::idesc_f16(64, P.N1, false, false);
+  // score MMA: M = 64 tokens x N1 heads, or stacked M = 128 (high and low rows) x N2 heads
+  // (B rows past N1 are read from the next query atom, or from the P buffers after the last
+  // one, and give score columns of heads >= H, which the softmax ignores)
+  P.idesc1 = stacked ? sm100::idesc_f16(128, P.N2, false, false)
+                     : sm100::idesc_f16(64, P.N1, false, false);
   P.idesc2 = sm100::idesc_f16(128, P.N2, false, true);   // A = C^T from TMEM, B = P MN-major
   pl.ok = pl.smem <= (size_t)kSmemLimit;
   return pl;
@@ -1090,6 +1203,7 @@ int instance_regs_nh(int N2) {
 bool launch_regs_ok(int b, int N2) {
   int r = 0;
   switch (b) {
+    case 16: r = instance_regs_nh<16>(N2); break;
     case 8: r = instance_regs_nh<8>(N2); break;
     case 4: r = instance_regs_nh<4>(N2); break;
     case 2: r = instance_regs_nh<2>(N2); break;
@@ -1138,6 +1252,7 @@ cudaError_t launch_decode_tc_packed(const DecodeArgs& a, const CUtensorMap& tmap
   pl.p.a = a;
   pl.p.qdtype = dtype;
   switch (a.b) {
+    case 16: return launch_bits<16>(pl.p, tmap, pl.smem, a.G, st);
     case 8: return launch_bits<8>(pl.p, tmap, pl.smem, a.G, st);
     case 4: return launch_bits<4>(pl.p, tmap, pl.smem, a.G, st);
     case 2: return launch_bits<2>(pl.p, tmap, pl.smem, a.G, st);
