@@ -388,7 +388,8 @@ kvk_status kvk_quant_write_layers(kvk_layout* L, int n, const int32_t* layers,
 static int choose_path(const kvk_layout* L, const AnchorDesc& A, int dtype, int H) {
   if (L->path == KVK_PATH_CUDA_CORE) return KVK_PATH_CUDA_CORE;
   bool tc = kvk::tc_supported(L, A, dtype, H);
-  if (L->path == KVK_PATH_TENSOR) return tc ? KVK_PATH_TENSOR : -1;
+  if (L->path == KVK_PATH_TENSOR || L->path == KVK_PATH_TENSOR_GENERAL)
+    return tc ? KVK_PATH_TENSOR : -1;
   return tc ? KVK_PATH_TENSOR : KVK_PATH_CUDA_CORE;
 }
 
@@ -497,7 +498,7 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
                     make_codes_tmap(&keep_tmap, probe.dst_codes, (int64_t)batch * keep_stride,
                                     A.row_bytes, A.b, kvk::kTcTileTokens);
     if (!ok) {
-      if (L->path == KVK_PATH_TENSOR) return room ? KVK_ERR_UNSUPPORTED : KVK_ERR_WORKSPACE;
+      if (L->path != KVK_PATH_AUTO) return room ? KVK_ERR_UNSUPPORTED : KVK_ERR_WORKSPACE;
       path = KVK_PATH_CUDA_CORE;
     }
   }
@@ -514,7 +515,7 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
       ok = make_query_tmap(&qmap_r, q_rope, L->d_rope, n_heads, batch, q_rope_stride_head,
                            q_rope_stride_seq, rows);
     if (!ok) {
-      if (L->path == KVK_PATH_TENSOR) return KVK_ERR_UNSUPPORTED;
+      if (L->path != KVK_PATH_AUTO) return KVK_ERR_UNSUPPORTED;
       path = KVK_PATH_CUDA_CORE;
     }
   }
@@ -556,8 +557,10 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSuccess;
   // Tensor-core launch over a codes plane: codes with one scale per token take the kernel
-  // specialised for them, bf16 rows and group-scaled codes the general one.
-  const bool packed = kvk::tc_packed_supported(L, A, dtype, n_heads);
+  // specialised for them (unless the general one is asked for), bf16 rows and group-scaled
+  // codes the general one.
+  const bool packed =
+      L->path != KVK_PATH_TENSOR_GENERAL && kvk::tc_packed_supported(L, A, dtype, n_heads);
   auto launch_tc = [&](const CUtensorMap& codes_map) {
     return packed ? kvk::launch_decode_tc_packed(a, codes_map, dtype, st)
                   : kvk::launch_decode_tc(a, codes_map, qmap_l, qmap_r, dtype, st);
@@ -656,7 +659,7 @@ kvk_status kvk_read_status(kvk_layout* L, uint32_t* flags, int clear, kvk_stream
 }
 
 kvk_status kvk_set_decode_path(kvk_layout* L, int path) {
-  if (!L || path < KVK_PATH_AUTO || path > KVK_PATH_CUDA_CORE) return KVK_ERR_INVALID_ARG;
+  if (!L || path < KVK_PATH_AUTO || path > KVK_PATH_TENSOR_GENERAL) return KVK_ERR_INVALID_ARG;
   L->path = path;
   return KVK_OK;
 }

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "KVK_OK", 1: "KVK_ERR_INVALID_ARG", 2: "KVK_ERR_BAD_TABLE",
                 3: "KVK_ERR_BUDGET", 4: "KVK_ERR_INHERITING_LAYER", 5: "KVK_ERR_WORKSPACE",
                 6: "KVK_ERR_ALIGNMENT", 7: "KVK_ERR_CUDA", 8: "KVK_ERR_UNSUPPORTED"}
 KVK_F32, KVK_BF16, KVK_F16 = 0, 1, 2
-KVK_PATH_AUTO, KVK_PATH_TENSOR, KVK_PATH_CUDA_CORE = 0, 1, 2
+KVK_PATH_AUTO, KVK_PATH_TENSOR, KVK_PATH_CUDA_CORE, KVK_PATH_TENSOR_GENERAL = 0, 1, 2, 3
 KVK_FLAG_NONFINITE, KVK_FLAG_WRITE_RANGE, KVK_FLAG_SEQ_LEN, KVK_FLAG_KEEP_INDEX = 1, 2, 4, 8
 KVK_FLAG_TIMEOUT = 16
 

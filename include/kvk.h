@@ -74,6 +74,10 @@ typedef enum { KVK_F32 = 0, KVK_BF16 = 1, KVK_F16 = 2 } kvk_dtype;
 #define KVK_PATH_AUTO      0 /* tensor-core kernel where it applies, else the CUDA-core kernel  */
 #define KVK_PATH_TENSOR    1 /* tcgen05 kernel only (KVK_ERR_UNSUPPORTED where it cannot run)   */
 #define KVK_PATH_CUDA_CORE 2 /* FFMA kernel (any shape, any dtype)                                */
+/* The general tcgen05 kernel (the one bf16 rows and group-scaled codes take) also where the
+ * token-scale kernel would run (codes with one scale per token): a second tensor-core
+ * implementation of those widths to check against; KVK_ERR_UNSUPPORTED where it cannot run. */
+#define KVK_PATH_TENSOR_GENERAL 3
 
 /*
  * kvk_create_layout -- validate a per-layer plan and lay out its cache in an arena.

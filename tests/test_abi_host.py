@@ -144,6 +144,9 @@ def test_planning_layout_cannot_launch(kvk):
         assert lib.kvk_decode_path_for(handle, 0, 0, 8, 0, ctypes.byref(path)) == 0
         assert path.value == kvk.KVK_PATH_CUDA_CORE            # fp32 queries
         assert lib.kvk_set_decode_path(handle, 7) == 1
+        assert lib.kvk_set_decode_path(handle, kvk.KVK_PATH_TENSOR_GENERAL) == 0
+        assert lib.kvk_set_decode_path(handle, kvk.KVK_PATH_TENSOR_GENERAL + 1) == 1
+        assert lib.kvk_set_decode_path(handle, kvk.KVK_PATH_AUTO) == 0
         assert lib.kvk_set_decode_ctas(handle, -1) == 1
         del torch
     finally:

@@ -1,5 +1,6 @@
 """Tensor-core decode against the oracle where the benchmark runs it: long sequences, each CTA
-streaming many 64-token tiles (ring phases wrap, double buffers alternate, the output
+streaming many 64-token tiles (through the token-scale kernel the benchmark takes, and through
+the general tensor-core kernel, KVK_PATH_TENSOR_GENERAL) (ring phases wrap, double buffers alternate, the output
 accumulates across tiles, the lazy rescale and the running power-of-two scale fire) and CTA
 ranges that cross sequence boundaries; inputs drawn with the workloads' own distributions
 (per-channel std U(0.5, 2), Student-t(3), N(0, 1)).
@@ -83,18 +84,20 @@ def test_long_sequences_few_ctas_match_oracle(pkg, oracle_mod, b, d, wname):
     try:
         lay.quant_write(0, c.cuda(), kr.cuda(), torch.zeros(B, dtype=torch.int32, device="cuda"))
         assert lay.decode_path_for(1, torch.bfloat16, H) == pkg.KVK_PATH_TENSOR
-        lay.set_decode_path(pkg.KVK_PATH_TENSOR)
         lens = torch.tensor(LENS, dtype=torch.int32, device="cuda")
-        for ctas in (1, 3, 7, 0):
-            lay.set_decode_ctas(ctas)
-            lse = torch.empty(B, H, device="cuda")
-            out = lay.mla_decode(1, ql.cuda(), qr.cuda(), lens, sigma, lse=lse)
-            torch.cuda.synchronize()
-            o, l_ = out.cpu().numpy(), lse.cpu().numpy()
-            for i in range(B):
-                e = check_outputs(o[i], l_[i], refs[i][0], refs[i][1],
-                                  f"b={b} d={d} {wname} ctas={ctas} seq {i}")
-                _note(f"long b={b:2d} {w.latent_dist}", e)
+        for path in (pkg.KVK_PATH_TENSOR, pkg.KVK_PATH_TENSOR_GENERAL):
+            lay.set_decode_path(path)
+            kern = "token-scale" if path == pkg.KVK_PATH_TENSOR else "general"
+            for ctas in (1, 3, 7, 0):
+                lay.set_decode_ctas(ctas)
+                lse = torch.empty(B, H, device="cuda")
+                out = lay.mla_decode(1, ql.cuda(), qr.cuda(), lens, sigma, lse=lse)
+                torch.cuda.synchronize()
+                o, l_ = out.cpu().numpy(), lse.cpu().numpy()
+                for i in range(B):
+                    e = check_outputs(o[i], l_[i], refs[i][0], refs[i][1],
+                                      f"{kern} b={b} d={d} {wname} ctas={ctas} seq {i}")
+                    _note(f"long {kern} b={b:2d} {w.latent_dist}", e)
         assert lay.read_status() == 0
     finally:
         lay.close()
