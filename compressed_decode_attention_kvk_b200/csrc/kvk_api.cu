@@ -556,9 +556,9 @@ kvk_status decode_impl(kvk_layout* L, int layer, const void* q_lat, const void* 
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSuccess;
-  // Tensor-core launch over a codes plane: codes with one scale per token take the kernel
-  // specialised for them (unless the general one is asked for), bf16 rows and group-scaled
-  // codes the general one.
+  // Tensor-core launch over a codes plane: codes with one scale per token and bf16 rows take
+  // the kernel specialised for them (unless the general one is asked for), group-scaled codes
+  // the general one.
   const bool packed =
       L->path != KVK_PATH_TENSOR_GENERAL && kvk::tc_packed_supported(L, A, dtype, n_heads);
   auto launch_tc = [&](const CUtensorMap& codes_map) {

@@ -1,5 +1,6 @@
 // kvk_decode_tc_packed.cu -- tensor-core (tcgen05) split decode over b-bit codes with one
-// fp16 scale per token (b in {2, 4, 8, 16}): the decode, and the fused append, of such layers.
+// fp16 scale per token (b in {2, 4, 8, 16}) and over uncompressed bf16 rows: the decode, and
+// the fused append, of such layers.
 //
 // Computes the same partials as the CUDA-core kernel (kvk_decode_fma.cu) and the general
 // tensor-core kernel (kvk_decode_tc.cu): for every piece of a sequence that the CTA owns, the
@@ -16,7 +17,8 @@
 // convert warps (16 features each), and the softmax reads S with the 16x256b shape, two tokens
 // per thread; measured on B200 at 32 x 8192 tokens, 40 heads, d = 512, this kernel is faster
 // than the general one (kvk_decode_tc.cu) for every width it covers.  The general kernel keeps
-// what this one lacks: bf16 rows and group scales.
+// what this one lacks: group scales.  bf16 rows are exact in f16 (in its normal range) and are
+// converted in place; rows past a piece's end are zeroed (bf16 garbage can be NaN).
 //
 // One persistent CTA per SM walks its slice of the flattened token space (the split charges
 // each piece a fixed cost, so a CTA that starts a sequence takes fewer tokens) in tiles of
@@ -93,6 +95,9 @@ constexpr int kPair = 2 * kAtom;       // 128 features
 // kLoOff), so that one M = 128 score MMA yields both partial scores of 64 tokens.
 template <int BITS>
 constexpr bool kStacked = (BITS == 16);
+// 16-bit codes and bf16 rows are converted in place, in the group slot TMA filled
+template <int BITS>
+constexpr bool kInPlace = (BITS == 16 || BITS == KVK_BITS_BF16);
 template <int BITS>
 constexpr uint32_t kAtomB = kStacked<BITS> ? 2u * kAtom : (uint32_t)kAtom;
 template <int BITS>
@@ -227,6 +232,11 @@ __device__ __forceinline__ void cvt_code16_split(uint32_t w, uint32_t& hi, uint3
   const __half2 t = __hfma2(hs, __float2half2_rn(256.f), __hneg2(h));
   hi = h2_bits(h);
   lo = h2_bits(__hadd2(t, ls));
+}
+// two bf16 values -> f16x2, round to nearest: exact for values in the f16 normal range
+// (bf16 keeps 8 significant bits, f16 11); beyond +-65504 a value becomes +-inf
+__device__ __forceinline__ uint32_t cvt_bf16x2(uint32_t w) {
+  return h2_bits(__floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
 }
 // bytes of w selected by `sel` (each a field u < 1024) -> f16x2 of (u - bias), exact
 __device__ __forceinline__ uint32_t cvt_small(uint32_t w, uint32_t sel, __half2 bias) {
@@ -368,7 +378,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     for (int i = 0; i < P.PR; ++i) {
       mbar_init(&b_pfull[i], kConvWarps);
       // score MMAs (commit), plus the convert warps where they read the slot back (b <= 8)
-      mbar_init(&b_pempty[i], kStacked<BITS> ? 1 : 1 + kConvWarps);
+      mbar_init(&b_pempty[i], kInPlace<BITS> ? 1 : 1 + kConvWarps);
       mbar_init(&b_tfull[i], 1);
     }
     for (int i = 0; i < P.RR; ++i) {
@@ -436,7 +446,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         cursor_start(c, seq0, off, a.batch, lo, hi);
         uint32_t cnt = 0;
         Ring rg;
-        const int slots = kStacked<BITS> ? P.PR : P.RR;
+        const int slots = kInPlace<BITS> ? P.PR : P.RR;
         // hold the first cache loads until the first query is staged: its loads then do not
         // queue behind every CTA's ring fill
         mbar_wait(b_qfull, 0u, abort, a.limit_ns);
@@ -448,7 +458,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         while (c.valid && !abort_read(abort)) {
           const int row0 = c.seq * a.max_tokens + c.pos;
           bool ok = true;
-          {   // this tile's scale window (the arena has tail slack for the last one)
+          if constexpr (BITS != KVK_BITS_BF16) {   // this tile's scale window (the arena has
+                                                   // tail slack for the last one)
             const uintptr_t sp = reinterpret_cast<uintptr_t>(a.scales + row0);
             if (!(ok = mbar_wait(&b_scempty[sr.slot], sr.phase ^ 1u, abort, a.limit_ns))) break;
             mbar_arrive_expect_tx(&b_scfull[sr.slot], kScBytes);
@@ -459,7 +470,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
           }
           for (int p = 0; p < P.NP && ok; ++p) {
             const uint32_t s = rg.slot, ph = rg.phase;
-            if constexpr (kStacked<BITS>) {
+            if constexpr (kInPlace<BITS>) {
               // 16-bit rows land in the group slot itself: each atom's 64 rows contiguously at
               // the start of the atom's place (the convert warps move them into the stacked
               // layout); the slot is re-armed once the score MMAs have read it
@@ -489,7 +500,7 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         const uint32_t first = cnt > (uint32_t)slots ? cnt - slots : 0u;
         for (uint32_t k = first; k < cnt; ++k) {
           const uint32_t s = k % slots, ph = (k / slots) & 1u;
-          wait_noabort(kStacked<BITS> ? &b_tfull[s] : &b_rfull[s], ph);
+          wait_noabort(kInPlace<BITS> ? &b_tfull[s] : &b_rfull[s], ph);
         }
       }
     } else if (warp == kMmaWarp) {
@@ -636,14 +647,17 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     // 128-byte swizzle phase (token % 8), so a warp's cells stay in its own 16-byte columns:
     // it reads all of them (ldmatrix) before it writes any, and no other warp touches them.
     uint32_t roff[4] = {}, aoff[4] = {};
-    if constexpr (kStacked<BITS>) {
+    if constexpr (kInPlace<BITS>) {
       const int mi = lane >> 3, r8 = lane & 7;
       const uint32_t col = (uint32_t)(((4 * (cq & 1) + 2 * ch + (mi >> 1)) ^ r8) << 4);
 #pragma unroll
       for (int tg = 0; tg < 4; ++tg) {
         const uint32_t tok = (uint32_t)(16 * tg + 8 * (mi & 1) + r8);
         roff[tg] = (uint32_t)(cq >> 1) * kAtomB<BITS> + tok * 128u + col;
-        aoff[tg] = (uint32_t)(cq >> 1) * kAtomB<BITS> + (tok >> 4) * 4096u + (tok & 15u) * 128u + col;
+        // bf16 rows stay where TMA put them (a plain slot's layout)
+        aoff[tg] = kStacked<BITS> ? (uint32_t)(cq >> 1) * kAtomB<BITS> + (tok >> 4) * 4096u +
+                                        (tok & 15u) * 128u + col
+                                  : roff[tg];
       }
     }
     Ring pr, rr;   // f16 group ring, packed group ring
@@ -737,8 +751,8 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
         // this warp owns features fb .. fb+15 of the group: atom cq/2, chunks
         // 4(cq%2) + 2ch + {0, 1} of every token row; it converts them and later transposes them
         const bool owns = (cq >> 1) < nat;
-        if constexpr (kStacked<BITS>) {
-          // In place, 16-bit codes -> exact f16 high and low parts, in one pass through
+        if constexpr (kInPlace<BITS>) {
+          // In place, 16-bit codes -> exact f16 high and low parts (bf16 rows -> f16), in one pass through
           // registers: each 8x8 block (8 tokens x 8 features) is loaded transposed from where
           // TMA put it, split element by element, stored back transposed into the stacked
           // layout (high parts, and low parts kLoOff further), and the high parts, now
@@ -756,14 +770,31 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
 #pragma unroll
               for (int i = 0; i < 4; ++i) x[4 * tg + i] = d4[i];
             }
+            if constexpr (kStacked<BITS>) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) cvt_code16_split(x[i], x[i], xl[i]);
+              for (int i = 0; i < 16; ++i) cvt_code16_split(x[i], x[i], xl[i]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) x[i] = cvt_bf16x2(x[i]);
+              if (c.cnt < kTile) {
+                // rows past the piece's end hold whatever the cache or scratch holds there
+                // (as bf16 possibly a NaN, and P = 0 times NaN is NaN): zero them.  Register
+                // 4tg + i holds tokens 16tg + 8(i%2) + 2(lane%4) + {0, 1}.
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const int t0 = 16 * (i >> 2) + 8 * (i & 1) + 2 * (lane & 3);
+                  x[i] &= (t0 < c.cnt ? 0x0000FFFFu : 0u) | (t0 + 1 < c.cnt ? 0xFFFF0000u : 0u);
+                }
+              }
+            }
 #pragma unroll
             for (int tg = 0; tg < 4; ++tg) {
               const uint32_t h4[4] = {x[4 * tg], x[4 * tg + 1], x[4 * tg + 2], x[4 * tg + 3]};
-              const uint32_t l4[4] = {xl[4 * tg], xl[4 * tg + 1], xl[4 * tg + 2], xl[4 * tg + 3]};
               stsm_x4_trans(sbase + aoff[tg], h4);
-              stsm_x4_trans(sbase + kLoOff + aoff[tg], l4);
+              if constexpr (kStacked<BITS>) {
+                const uint32_t l4[4] = {xl[4 * tg], xl[4 * tg + 1], xl[4 * tg + 2], xl[4 * tg + 3]};
+                stsm_x4_trans(sbase + kLoOff + aoff[tg], l4);
+              }
             }
           }
           fence_proxy_async_smem();
@@ -860,7 +891,10 @@ decode_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUt
     while (c.valid) {
       const int t = c.tile, sb = t & 1;
       float s_a = 0.f, s_b = 0.f;
-      {
+      if constexpr (BITS == KVK_BITS_BF16) {   // uncompressed rows: unit token scale
+        s_a = (ra < c.cnt) ? 1.f : 0.f;
+        s_b = (rb < c.cnt) ? 1.f : 0.f;
+      } else {
         fail = fail || !wait_warp(&b_scfull[sr.slot], sr.phase, abort, a.limit_ns);
         const __half* w = reinterpret_cast<const __half*>(m->sc[sr.slot]) +
                           ((reinterpret_cast<uintptr_t>(a.scales + (int64_t)c.seq * a.max_tokens +
@@ -1110,8 +1144,9 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
   Plan pl;
   memset(&pl, 0, sizeof(pl));
   TcParams& P = pl.p;
-  if (b != 2 && b != 4 && b != 8 && b != 16) return pl;
+  if (b != 2 && b != 4 && b != 8 && b != 16 && b != KVK_BITS_BF16) return pl;
   const bool stacked = (b == 16);
+  const bool in_place = stacked || b == KVK_BITS_BF16;
   const int n = d + d_rope;
   P.N1 = (H + 7) / 8 * 8;
   P.N2 = (H + 15) / 16 * 16;
@@ -1127,7 +1162,7 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
   P.p_bytes = 8u * P.lbo_p;
   const size_t p_bytes = 2 * (size_t)P.p_bytes;
   const size_t misc_bytes = sizeof(Misc) + sizeof(int32_t) * (size_t)(batch + 1);
-  const int raw_slot = stacked ? 0 : 64 * 16 * b;   // 16-bit rows land in the slots
+  const int raw_slot = in_place ? 0 : 64 * 16 * b;   // 16-bit rows land in the slots
   const size_t slot_bytes = stacked ? 4u * kAtom : (size_t)kPair;
   P.raw_slot = raw_slot;
   // try the largest rings that fit
@@ -1141,7 +1176,7 @@ Plan make_plan(int d, int d_rope, int b, int H, int batch) {
     return off + 1024;   // runtime alignment slack of the dynamic shared memory base
   };
   int PR = 0, RR = 0;
-  if (stacked) {
+  if (in_place) {
     // TMA lands in the slots: at least a tile's groups
     for (PR = 3 * P.NP; PR >= P.NP; --PR)
       if (total_for(PR, 0) <= (size_t)kSmemLimit) break;
@@ -1204,6 +1239,7 @@ bool launch_regs_ok(int b, int N2) {
   int r = 0;
   switch (b) {
     case 16: r = instance_regs_nh<16>(N2); break;
+    case KVK_BITS_BF16: r = instance_regs_nh<KVK_BITS_BF16>(N2); break;
     case 8: r = instance_regs_nh<8>(N2); break;
     case 4: r = instance_regs_nh<4>(N2); break;
     case 2: r = instance_regs_nh<2>(N2); break;
@@ -1253,6 +1289,7 @@ cudaError_t launch_decode_tc_packed(const DecodeArgs& a, const CUtensorMap& tmap
   pl.p.qdtype = dtype;
   switch (a.b) {
     case 16: return launch_bits<16>(pl.p, tmap, pl.smem, a.G, st);
+    case KVK_BITS_BF16: return launch_bits<KVK_BITS_BF16>(pl.p, tmap, pl.smem, a.G, st);
     case 8: return launch_bits<8>(pl.p, tmap, pl.smem, a.G, st);
     case 4: return launch_bits<4>(pl.p, tmap, pl.smem, a.G, st);
     case 2: return launch_bits<2>(pl.p, tmap, pl.smem, a.G, st);
