@@ -32,7 +32,8 @@ def _paths(pkg, lay, dtype, H, has_keep=False):
     lay.set_decode_path(pkg.KVK_PATH_TENSOR)
     try:
         if lay.decode_path_for(0, dtype, H, has_keep) == pkg.KVK_PATH_TENSOR:
-            ps.append(pkg.KVK_PATH_TENSOR)
+            # the token-scale tensor-core kernel, and the general one forced
+            ps += [pkg.KVK_PATH_TENSOR, pkg.KVK_PATH_TENSOR_GENERAL]
     except pkg.KvkError:
         pass
     finally:
