@@ -29,10 +29,10 @@
 //              16-bit codes as stacked high and low parts) and their transpose into TMEM;
 //              staged query (power-of-two scaled).
 //              Two warps per SM sub-partition, 16 features of every 128-feature group each.
-//   warp 12    TMA producer: 128-feature groups of 64 rows into a ring (16-bit rows straight
-//              into the group slots, narrower codes into a raw ring), and each
-//              tile's token scales; the stream is read once, so it carries an evict-first
-//              L2 policy
+//   warp 12    TMA producer: 128-feature groups of 64 rows into a ring (16-bit codes and bf16
+//              rows straight into the group slots, narrower codes into a raw ring), and each
+//              tile's token scales (none for bf16 rows); the stream is read once, so it
+//              carries an evict-first L2 policy
 //   warp 13    score-MMA issuer (one thread) and TMEM owner
 //   warp 14    output-MMA issuer (one thread)
 //   warp 15    the fused append's new tokens; then warms L2 with the queries of the CTA's
@@ -46,14 +46,15 @@
 //                                                               A = C^T in TMEM)
 // Heads sit on N, so 40 heads cost N = 40 / 48, never M = 128.  The convert warps unpack each
 // 128-feature group from a raw ring into an f16 slot (UMMA 128-byte swizzled, K-major: the
-// score MMA's A), or split 16-bit rows in place, and put their 16 features of it, transposed
-// with ldmatrix.trans, into TMEM (tcgen05.st); the output MMA reads C^T from TMEM (for 16-bit
-// codes the high parts: f16(code), relative 2^-12 on the output, inside its tolerance).
+// score MMA's A), or convert 16-bit rows in place (codes split, bf16 rounded to f16), and put
+// their 16 features of it, transposed with ldmatrix.trans, into TMEM (tcgen05.st); the output
+// MMA reads C^T from TMEM (for 16-bit codes the high parts: f16(code), relative 2^-12 on the
+// output, inside its tolerance).
 // The transpose fragment orders the 16 tokens of each K step as 0,1,8,9,2,3,10,11,4,5,12,13,
 // 6,7,14,15; the softmax warps write P's K rows in that same order.
-// The per-token scale s_t multiplies the S row and is folded into P as p * s_t / S_run, with
-// S_run a running power of two >= every scale seen so far (when it grows, O is rescaled by the
-// exact ratio).
+// The per-token scale s_t (1 for bf16 rows) multiplies the S row and is folded into P as
+// p * s_t / S_run, with S_run a running power of two >= every scale seen so far (when it grows,
+// O is rescaled by the exact ratio).
 // Every wait is bounded (the call's wait limit); on expiry the kernel records
 // KVK_FLAG_TIMEOUT, drains its own TMA loads and MMAs, frees TMEM and exits.
 #include <string.h>
