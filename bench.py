@@ -90,7 +90,7 @@ def barrier(pg, device=None):
 # Sources whose code makes up the dominant decode kernel (the token-scale tensor-core kernel
 # that 16-bit layers take, and the headers it includes); the traffic record is tied to a
 # comment- and whitespace-insensitive hash.
-KERNEL_SOURCES = ("compressed_decode_attention_kvk_b200/csrc/kvk_decode_tc_packed.cu",
+KERNEL_SOURCES = ("compressed_decode_attention_kvk_b200/csrc/kvk_decode_tc_token.cu",
                   "compressed_decode_attention_kvk_b200/csrc/kvk_quant_common.cuh",
                   "compressed_decode_attention_kvk_b200/csrc/kvk_sm100.cuh",
                   "compressed_decode_attention_kvk_b200/csrc/kvk_decode_common.cuh",

@@ -1,4 +1,4 @@
-// kvk_decode_tc_packed.cu -- tensor-core (tcgen05) split decode over b-bit codes with one
+// kvk_decode_tc_token.cu -- tensor-core (tcgen05) split decode over b-bit codes with one
 // fp16 scale per token (b in {2, 4, 8, 16}) and over uncompressed bf16 rows: the decode, and
 // the fused append, of such layers.
 //

@@ -146,7 +146,7 @@ cudaError_t launch_decode_fma(const DecodeArgs& a, int dtype, cudaStream_t strea
 cudaError_t launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tmap, const CUtensorMap& qmap_l,
                              const CUtensorMap& qmap_r, int dtype, cudaStream_t st);
 bool tc_supported(const kvk_layout* L, const AnchorDesc& A, int dtype, int H);
-// The token-scale tensor-core kernel (kvk_decode_tc_packed.cu): decode (and fused append) of
+// The token-scale tensor-core kernel (kvk_decode_tc_token.cu): decode (and fused append) of
 // b in {2, 4, 8, 16} codes with one scale per token and of bf16 rows; the query read with
 // 16-byte loads (rows
 // 16-byte aligned, as the general kernel's query tensor maps require).
